@@ -1,0 +1,201 @@
+/*
+ * pa.h — C ABI of the B200 (sm_100a) paged KV attention library (libpa.so).
+ *
+ * Three operations, all asynchronous on the caller's CUDA stream:
+ *
+ *   pa_write_kv            scatter this step's K/V rows into a block-paged cache
+ *   pa_attention_varlen    softmax attention of packed variable-length queries
+ *                          over the paged cache (prefill, decode, chunked
+ *                          prefill and any mix of them in one batch)
+ *   pa_attention_smallseq  one query per batch entry over a handful (<= 16) of
+ *                          contiguous keys
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Element type: bfloat16 for every Q/K/V/cache/output tensor (passed as
+ *    void*, 2 bytes per element).  Index tensors are int32 unless stated.
+ *  - Layout: token-major ("NHD"), dense, innermost dimension last:
+ *      q, out           [num_tokens, num_q_heads, head_dim]
+ *      k, v (new rows)  [num_tokens, num_kv_heads, head_dim]
+ *      k_cache, v_cache [num_blocks, block_size, num_kv_heads, head_dim]
+ *  - Pointers are device pointers unless stated, 16-byte aligned.
+ *  - The caller owns every buffer, including the workspace.  The library
+ *    allocates no device memory and keeps no state between calls beyond a
+ *    per-device table of attributes (SM count) and lazily-resolved driver
+ *    entry points.
+ *  - `stream` is a cudaStream_t passed as void*; NULL means the legacy default
+ *    stream.  No call synchronises except pa_get_error.
+ *  - `out` must not alias any input.
+ *
+ * Errors
+ * ------
+ *  Problems visible on the host (null pointers, non-positive sizes,
+ *  num_q_heads % num_kv_heads != 0, unsupported head_dim or block_size,
+ *  misaligned pointers, a workspace that is too small) are reported by the
+ *  return value BEFORE anything is launched or written — the reject-before-
+ *  write rule of TensorRT-LLM PR "CSA2 Vanilla sparse attention"
+ *  (description, "rejected before anything is written").
+ *  Problems only the device can see (a slot or block id outside the pool,
+ *  inconsistent lengths, a query longer than its sequence, an exceeded length
+ *  hint, a bounded wait that gave up) never fault: the kernel skips the
+ *  offending row or reads zeros instead, and ORs a bit into a sticky 32-bit
+ *  error word held in the first bytes of the workspace.  pa_get_error reads
+ *  and clears it.
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,  /* host-visible bad argument; nothing was launched */
+  PA_ERR_UNSUPPORTED = 2,  /* valid request outside what this build supports */
+  PA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+  PA_ERR_DEVICE_INDEX = 4, /* pa_get_error: the device saw a bad index/length */
+  PA_ERR_TIMEOUT = 5       /* pa_get_error: a bounded device wait gave up */
+} pa_status;
+
+/* Bits of the device error word (pa_get_error's *bits). */
+#define PA_DEVERR_SLOT      0x1u  /* slot_mapping entry >= num_blocks*block_size */
+#define PA_DEVERR_BLOCK     0x2u  /* block-table entry outside [0, num_blocks)   */
+#define PA_DEVERR_LENGTHS   0x4u  /* query_start_loc / seq_lens / cu_seqlens bad */
+#define PA_DEVERR_QLEN      0x8u  /* a sequence has more queries than keys       */
+#define PA_DEVERR_HINT      0x10u /* a length exceeded max_query_len/max_seq_len */
+#define PA_DEVERR_TIMEOUT   0x20u /* a bounded wait inside a kernel gave up      */
+
+/* Bytes at the start of every workspace reserved for the error word. */
+#define PA_ERROR_WORD_BYTES 256
+
+/*
+ * pa_write_kv — KV-cache write through slot_mapping.
+ *
+ * Defined by vllm-spyre PR #853 "Pytorch Native Attention on Spyre",
+ * description, step 1: every new token's key/value row is written into the
+ * paged cache at the slot slot_mapping names; slot s is block s / block_size,
+ * offset s % block_size (the vLLM v1 convention).
+ *
+ *  k, v          [num_tokens, num_kv_heads, head_dim] bf16 (read)
+ *  slot_mapping  [num_tokens] int64 (read).  slot < 0 marks a padding token:
+ *                its row is skipped.  slot >= num_blocks*block_size: row
+ *                skipped and PA_DEVERR_SLOT raised.
+ *  k_cache, v_cache [num_blocks, block_size, num_kv_heads, head_dim] bf16,
+ *                written in place; slots not named are left unchanged.
+ *  workspace     NULL, or >= PA_ERROR_WORD_BYTES zero-initialised bytes whose
+ *                error word receives PA_DEVERR_SLOT.
+ * Two tokens naming the same slot is invalid input; the cache then holds one
+ * of the candidate rows.  head_dim must be a multiple of 8.
+ */
+pa_status pa_write_kv(const void* k, const void* v, const int64_t* slot_mapping,
+                      int64_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                      void* k_cache, void* v_cache, int64_t num_blocks,
+                      int32_t block_size, void* workspace, void* stream);
+
+/*
+ * pa_attention_varlen_workspace_size — bytes of workspace pa_attention_varlen
+ * needs for these sizes (a function of the arguments only).  The workspace
+ * must be zero-initialised once before its first use (the error word must
+ * start at zero); afterwards it can be reused by consecutive calls on the
+ * same stream without clearing.
+ */
+size_t pa_attention_varlen_workspace_size(int32_t num_seqs, int64_t num_q_tokens,
+                                          int32_t num_q_heads, int32_t num_kv_heads,
+                                          int32_t head_dim);
+
+/*
+ * pa_attention_varlen — paged softmax attention over packed varlen queries.
+ *
+ * Defined by vllm-spyre PR #853, description, steps 2-6 (keys of a sequence
+ * reached through its block list; a boolean mask of padding validity and, for
+ * prefill, causality; softmax attention per sequence; only real tokens
+ * written) with grouped-query heads as the repeat_interleave expansion of the
+ * same description, and causal alignment bottom-right as in vllm-omni
+ * PR #9244 (kernel-semantics review).  For sequence s with
+ * Lq = query_start_loc[s+1] - query_start_loc[s] queries and Lkv = seq_lens[s]
+ * keys, query i (token query_start_loc[s] + i) and query head h see keys
+ * j < Lkv, and with causal != 0 only j <= (Lkv - Lq) + i; they read KV head
+ * h / (num_q_heads / num_kv_heads); key j lives in block
+ * block_tables[s][j / block_size], offset j % block_size.
+ *   out = softmax(scale * q . K^T over the visible keys) . V
+ * A row with no visible key is written as zeros (TensorRT-LLM "CSA2 Vanilla
+ * sparse attention", description: an empty selection gives zeros).
+ * seq_lens counts every key of the sequence, this step's tokens included.
+ * Sequences with Lq == 1 take the split-KV decode kernel; all others the
+ * tensor-core prefill kernel; both may appear in one call.
+ *
+ *  q                [num_q_tokens, num_q_heads, head_dim] bf16
+ *  k_cache, v_cache [num_blocks, block_size, num_kv_heads, head_dim] bf16
+ *  block_tables     [num_seqs, max_blocks_per_seq] int32; entries past a
+ *                   sequence's last needed block are never read
+ *  seq_lens         [num_seqs] int32
+ *  query_start_loc  [num_seqs + 1] int32, non-decreasing, starting at 0,
+ *                   ending at <= num_q_tokens
+ *  max_query_len    host hint: >= every Lq (1 means a pure decode batch, and
+ *                   the prefill kernel is not launched).  A violated hint
+ *                   raises PA_DEVERR_HINT.
+ *  max_seq_len      host hint: >= every Lkv; checked like max_query_len.
+ *  scale            multiplies q . k (usually 1/sqrt(head_dim))
+ *  causal           0 or 1
+ *  out              [num_q_tokens, num_q_heads, head_dim] bf16, written for
+ *                   every token that belongs to a sequence
+ *  workspace        device buffer of >= workspace_size bytes (see above)
+ * Supported: head_dim in {64, 128}; block_size == 16;
+ * num_q_heads / num_kv_heads <= 16 (decode packs a GQA group into one tile).
+ */
+pa_status pa_attention_varlen(const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* block_tables, int32_t max_blocks_per_seq,
+                              const int32_t* seq_lens, const int32_t* query_start_loc,
+                              int32_t num_seqs, int64_t num_q_tokens,
+                              int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                              int32_t block_size, int64_t num_blocks,
+                              int32_t max_query_len, int32_t max_seq_len, float scale,
+                              int32_t causal, void* out, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/*
+ * pa_attention_smallseq — s_q = 1 cross attention over short contiguous KV.
+ *
+ * Defined by ROCm/TransformerEngine PR #461 "CK varlen cross attention for
+ * small-seq", description: one query per batch entry, keys and values packed
+ * THD with cu_seqlens_kv (entry b owns rows cu_seqlens_kv[b] ..
+ * cu_seqlens_kv[b+1]-1), no causal mask, max_seqlen_kv <= 16; the batch is
+ * the number of query tokens.  An empty entry gives zeros.
+ *
+ *  q, out   [batch, num_q_heads, head_dim] bf16
+ *  k, v     [cu_seqlens_kv[batch], num_kv_heads, head_dim] bf16
+ *  cu_seqlens_kv [batch + 1] int32, non-decreasing from 0
+ *  max_seqlen_kv host hint, 0..16 (> 16: PA_ERR_UNSUPPORTED — use
+ *           pa_attention_varlen); an entry longer than the hint raises
+ *           PA_DEVERR_HINT and only its first max_seqlen_kv keys are used.
+ *  workspace NULL or >= PA_ERROR_WORD_BYTES zero-initialised bytes (error word)
+ * Supported: head_dim in {64, 128}.
+ */
+pa_status pa_attention_smallseq(const void* q, const void* k, const void* v,
+                                const int32_t* cu_seqlens_kv, int32_t batch,
+                                int32_t num_q_heads, int32_t num_kv_heads,
+                                int32_t head_dim, int32_t max_seqlen_kv, float scale,
+                                void* out, void* workspace, void* stream);
+
+/*
+ * pa_get_error — synchronise `stream`, read the workspace's error word into
+ * *bits (may be NULL), clear it, and map it to a status: PA_OK when zero,
+ * PA_ERR_TIMEOUT when PA_DEVERR_TIMEOUT is set, PA_ERR_DEVICE_INDEX otherwise.
+ */
+pa_status pa_get_error(void* workspace, void* stream, uint32_t* bits);
+
+/* Static description of a status code. */
+const char* pa_status_string(pa_status status);
+
+/* Library version string, e.g. "pa 0.1 sm_100a". */
+const char* pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H */

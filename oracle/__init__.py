@@ -1,0 +1,173 @@
+"""Reference oracle (fp64 CPU) for paged KV attention — test infrastructure.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` leg of
+``bench.py`` may import this package.  The product path never calls it.
+
+The arithmetic lives in ``oracle.c`` (plain C, double precision); this module
+only compiles it with gcc and marshals numpy arrays into it.  Inputs are
+bfloat16 bit patterns held in ``uint16`` arrays; outputs are ``float64``.
+
+Definitions followed (see the header of ``oracle.c`` for each passage):
+
+* cache write — vllm-spyre PR #853 "Pytorch Native Attention on Spyre",
+  description, step 1 (slot_mapping scatter);
+* masked softmax attention with GQA — same description, steps 4-6 and the
+  repeat_interleave paragraph; bottom-right causal alignment — vllm-omni
+  PR #9244, kernel-semantics review; empty rows give zeros — TensorRT-LLM
+  "CSA2 Vanilla sparse attention", description;
+* small-seq cross attention — ROCm/TransformerEngine PR #461, description.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        p = ctypes.c_void_p
+        i32, i64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_double
+        lib.oracle_num_threads.restype = i32
+        lib.oracle_write_kv.restype = i64
+        lib.oracle_write_kv.argtypes = [p, p, p, i64, i32, i32, p, p, i64, i32]
+        lib.oracle_attention_varlen.restype = i32
+        lib.oracle_attention_varlen.argtypes = [
+            p, p, p, p, p, p, i32, i32, i32, i32, f64, i32, p, i64, p]
+        lib.oracle_attention_varlen_paged.restype = i32
+        lib.oracle_attention_varlen_paged.argtypes = [
+            p, p, p, p, i32, p, p, i32, i32, i32, i32, i32, i64, f64, i32, p, i64, p]
+        lib.oracle_attention_weights.restype = i64
+        lib.oracle_attention_weights.argtypes = [
+            p, p, p, p, p, p, i32, i32, i32, i32, f64, i32, i64, i32, p]
+        lib.oracle_attention_smallseq.restype = i32
+        lib.oracle_attention_smallseq.argtypes = [p, p, p, p, i32, i32, i32, i32, f64, p]
+        _lib = lib
+    return _lib
+
+
+def _arr(a, dtype):
+    a = np.ascontiguousarray(a)
+    if a.dtype != dtype:
+        raise TypeError(f"expected {np.dtype(dtype)}, got {a.dtype}")
+    return a
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def write_kv(k, v, slot_mapping, k_cache, v_cache, block_size):
+    """Literal slot-by-slot write, in place on the uint16 cache arrays.
+
+    k, v: [T, Hkv, D] uint16; slot_mapping: [T] int64;
+    caches: [NB, BS, Hkv, D] uint16.  Returns the count of out-of-pool slots.
+    """
+    k, v = _arr(k, np.uint16), _arr(v, np.uint16)
+    sm = _arr(slot_mapping, np.int64)
+    if not (k_cache.flags.c_contiguous and v_cache.flags.c_contiguous):
+        raise ValueError("caches must be contiguous")
+    t, hkv, d = k.shape
+    nb = k_cache.shape[0]
+    return int(_load().oracle_write_kv(_ptr(k), _ptr(v), _ptr(sm), t, hkv, d,
+                                       _ptr(k_cache), _ptr(v_cache), nb, block_size))
+
+
+def attention_varlen(q, k_seq, v_seq, kv_offsets, seq_lens, query_start_loc,
+                     num_kv_heads, scale, causal, rows=None):
+    """Logical-form attention; returns float64 [T, Hq, D] (rows not asked for are 0)."""
+    q = _arr(q, np.uint16)
+    k_seq, v_seq = _arr(k_seq, np.uint16), _arr(v_seq, np.uint16)
+    kv_offsets = _arr(kv_offsets, np.int64)
+    seq_lens = _arr(seq_lens, np.int32)
+    qsl = _arr(query_start_loc, np.int32)
+    t, hq, d = q.shape
+    out = np.zeros((t, hq, d), dtype=np.float64)
+    rows_a = None if rows is None else _arr(rows, np.int64)
+    rc = _load().oracle_attention_varlen(
+        _ptr(q), _ptr(k_seq), _ptr(v_seq), _ptr(kv_offsets), _ptr(seq_lens), _ptr(qsl),
+        len(seq_lens), hq, num_kv_heads, d, float(scale), int(bool(causal)),
+        _ptr(rows_a), 0 if rows_a is None else len(rows_a), _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_attention_varlen failed ({rc})")
+    return out
+
+
+def attention_varlen_paged(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc,
+                           num_kv_heads, scale, causal, rows=None):
+    """Paged-form attention through the block table; returns float64 [T, Hq, D]."""
+    q = _arr(q, np.uint16)
+    k_cache, v_cache = _arr(k_cache, np.uint16), _arr(v_cache, np.uint16)
+    bt = _arr(block_tables, np.int32)
+    seq_lens = _arr(seq_lens, np.int32)
+    qsl = _arr(query_start_loc, np.int32)
+    t, hq, d = q.shape
+    nb, bs = k_cache.shape[0], k_cache.shape[1]
+    out = np.zeros((t, hq, d), dtype=np.float64)
+    rows_a = None if rows is None else _arr(rows, np.int64)
+    rc = _load().oracle_attention_varlen_paged(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(bt), bt.shape[1], _ptr(seq_lens),
+        _ptr(qsl), len(seq_lens), hq, num_kv_heads, d, bs, nb, float(scale),
+        int(bool(causal)), _ptr(rows_a), 0 if rows_a is None else len(rows_a), _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_attention_varlen_paged failed ({rc})")
+    return out
+
+
+def attention_weights(q, k_seq, v_seq, kv_offsets, seq_lens, query_start_loc,
+                      num_kv_heads, scale, causal, token, head):
+    """Softmax weights of one (token, head) row over its sequence's keys."""
+    q = _arr(q, np.uint16)
+    k_seq, v_seq = _arr(k_seq, np.uint16), _arr(v_seq, np.uint16)
+    kv_offsets = _arr(kv_offsets, np.int64)
+    seq_lens = _arr(seq_lens, np.int32)
+    qsl = _arr(query_start_loc, np.int32)
+    t, hq, d = q.shape
+    s = int(np.searchsorted(qsl, token, side="right") - 1)
+    w = np.zeros(max(int(seq_lens[s]), 1), dtype=np.float64)
+    n = _load().oracle_attention_weights(
+        _ptr(q), _ptr(k_seq), _ptr(v_seq), _ptr(kv_offsets), _ptr(seq_lens), _ptr(qsl),
+        len(seq_lens), hq, num_kv_heads, d, float(scale), int(bool(causal)),
+        int(token), int(head), _ptr(w))
+    if n < 0:
+        raise ValueError("oracle_attention_weights failed")
+    return w[: int(seq_lens[s])], int(n)
+
+
+def attention_smallseq(q, k, v, cu_seqlens_kv, num_kv_heads, scale):
+    """s_q = 1 cross attention over contiguous THD keys; returns float64 [B, Hq, D]."""
+    q = _arr(q, np.uint16)
+    k, v = _arr(k, np.uint16), _arr(v, np.uint16)
+    cu = _arr(cu_seqlens_kv, np.int32)
+    b, hq, d = q.shape
+    out = np.zeros((b, hq, d), dtype=np.float64)
+    rc = _load().oracle_attention_smallseq(_ptr(q), _ptr(k), _ptr(v), _ptr(cu), b, hq,
+                                           num_kv_heads, d, float(scale), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_attention_smallseq failed")
+    return out
