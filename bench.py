@@ -1,0 +1,492 @@
+"""Benchmark: one step = KV scatter of this step's tokens + paged attention.
+
+Default workload (N = 1): the decode batch — 64 sequences x 1 query, context
+uniform in [256, 4096], Hq 32 / Hkv 8, head_dim 128, block 16, bf16 — on
+which the headline HBM-bandwidth metric is quoted.  With --gpus N (launched
+by torchrun, one process per GPU) every rank runs its own independent decode
+batch (different seed): weak scaling, no collective on the data path; ranks
+only meet at the barriers around the timed region and in one MAX reduction of
+the elapsed time.
+
+Prints ONE JSON line (rank 0).  ``--impl reference`` times the fp64 CPU
+oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "paged-attn decode HBM GB/s + prefill TFLOP/s (fraction of B200 roofline)"
+WORKLOAD = ("decode_batch: 64 seqs x 1 query token, context U[256,4096], Hq 32 / Hkv 8, "
+            "head_dim 128, block 16, bf16, shuffled block tables; step = scatter of the 64 new "
+            "K/V rows + split-KV decode attention")
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work (what the method must move / compute)
+# ---------------------------------------------------------------------------
+
+def scatter_bytes(case) -> int:
+    t = int(case.k_new.shape[0])
+    return t * case.num_kv_heads * case.head_dim * 2 * 4 + 8 * t
+
+
+def attention_bytes(case) -> int:
+    """K + V of every visible key once per KV head, plus Q, O and the tables read."""
+    lens = case.seq_lens.cpu().to(torch.int64)
+    kv = int(lens.sum()) * case.num_kv_heads * case.head_dim * 2 * 2
+    qo = 2 * case.num_q_tokens * case.num_q_heads * case.head_dim * 2
+    tables = int(((lens + case.block_size - 1) // case.block_size).sum()) * 4
+    meta = 4 * (2 * case.num_seqs + 1)
+    return kv + qo + tables + meta
+
+
+def visible_pairs(case) -> int:
+    lens = case.seq_lens.cpu().tolist()
+    ql = case.query_lens.cpu().tolist()
+    tot = 0
+    for L, q in zip(lens, ql):
+        if not case.causal:
+            tot += L * q
+            continue
+        for i in range(q):
+            tot += max(0, min(L, L - q + i + 1))
+    return tot
+
+
+def attention_flops(case) -> int:
+    return 4 * case.head_dim * case.num_q_heads * visible_pairs(case)
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.dev = device_index
+
+    def _id(self):
+        try:
+            u = torch.cuda.get_device_properties(self.dev).uuid
+            s = str(u)
+            return s if s.startswith("GPU-") else "GPU-" + s
+        except Exception:
+            return str(self.dev)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self._id(), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(
+            d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def device_case(case, dev):
+    import dataclasses
+    kw = {}
+    for f in dataclasses.fields(case):
+        v = getattr(case, f.name)
+        kw[f.name] = v.to(dev) if isinstance(v, torch.Tensor) else v
+    return type(case)(**kw)
+
+
+def time_varlen_component(pa, case, iters=20, warmup=3, with_scatter=False):
+    """Average device time (ms) of one attention_varlen call on `case` (device tensors)."""
+    ws = pa.varlen_workspace(case.num_seqs, case.num_q_tokens, case.num_q_heads,
+                             case.num_kv_heads, case.head_dim)
+    out = torch.empty_like(case.q)
+
+    def run():
+        if with_scatter:
+            pa.write_kv(case.k_new, case.v_new, case.slot_mapping, case.k_cache, case.v_cache)
+        pa.attention_varlen(case.q, case.k_cache, case.v_cache, case.block_tables, case.seq_lens,
+                            case.query_start_loc, case.num_kv_heads, case.scale, case.causal, out,
+                            max_query_len=case.max_query_len, max_seq_len=case.max_seq_len,
+                            workspace=ws)
+
+    if not with_scatter:
+        pa.write_kv(case.k_new, case.v_new, case.slot_mapping, case.k_cache, case.v_cache)
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(iters)]
+    for a, b in evs:
+        a.record()
+        run()
+        b.record()
+    torch.cuda.synchronize()
+    st, bits = pa.get_error(ws)
+    if st != 0:
+        raise RuntimeError(f"device error word {bits:#x}")
+    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+
+def components(pa, hbm_peak, tc_peak, peak_kind):
+    """Secondary single-GPU measurements on the other workloads (device time per call)."""
+    res = {}
+    dev = torch.device("cuda")
+    vc = workloads.varlen_prefill(device=dev, keep_logical=False)
+    ms = time_varlen_component(pa, vc)
+    tf = attention_flops(vc) / (ms * 1e-3) / 1e12
+    res["varlen_prefill"] = {"ms": round(ms, 4), "tflops": round(tf, 1),
+                             "frac": round(tf / tc_peak, 3), "peak": tc_peak,
+                             "unit": "TFLOP/s", "of": peak_kind}
+    del vc
+    ss = workloads.smallseq_batch(device=dev)
+    out = torch.empty_like(ss.q)
+    for _ in range(3):
+        pa.attention_smallseq(ss.q, ss.k, ss.v, ss.cu_seqlens_kv, ss.scale, out)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(20):
+        pa.attention_smallseq(ss.q, ss.k, ss.v, ss.cu_seqlens_kv, ss.scale, out)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / 20
+    nbytes = (ss.k.numel() + ss.v.numel() + ss.q.numel() + out.numel()) * 2 + 4 * (ss.batch + 1)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    res["smallseq_batch"] = {"ms": round(ms, 4), "gbs": round(gbs, 1),
+                             "frac": round(gbs / hbm_peak, 3), "unit": "GB/s", "of": peak_kind}
+    del ss, out
+    mx = workloads.mixed_step(device=dev, keep_logical=False)
+    ms = time_varlen_component(pa, mx, iters=10)
+    nbytes = attention_bytes(mx)
+    fl = attention_flops(mx)
+    # serial roofline: decode bytes at the HBM peak plus prefill FLOPs at the tensor peak
+    dec_bytes = sum(int(l) for l, q in zip(mx.seq_lens.tolist(), mx.query_lens.tolist()) if q == 1)
+    dec_bytes *= mx.num_kv_heads * mx.head_dim * 4
+    pre_fl = fl - 4 * mx.head_dim * mx.num_q_heads * sum(
+        int(l) for l, q in zip(mx.seq_lens.tolist(), mx.query_lens.tolist()) if q == 1)
+    t_roof = dec_bytes / (hbm_peak * 1e9) + pre_fl / (tc_peak * 1e12)
+    res["mixed_step"] = {"ms": round(ms, 4), "roofline_ms": round(t_roof * 1e3, 4),
+                         "frac_serial": round(t_roof / (ms * 1e-3), 3),
+                         "decode_gb": round(dec_bytes / 1e9, 2), "prefill_tflop": round(pre_fl / 1e12, 3),
+                         "of": peak_kind}
+    del mx
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_ours(args, rank, world, local_rank):
+    import paged_kv_gqa_reshape_b200 as pa
+
+    pa.load()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    hbm_peak, tc_peak, tc_sust, peak_kind = measured_peaks()
+
+    case = workloads.decode_batch(device=dev, seed=1002 + rank, keep_logical=False)
+    ws = pa.varlen_workspace(case.num_seqs, case.num_q_tokens, case.num_q_heads,
+                             case.num_kv_heads, case.head_dim, device=dev)
+    out = torch.empty_like(case.q)
+    mql, msl = case.max_query_len, case.max_seq_len
+
+    def step(attn_events=None):
+        pa.write_kv(case.k_new, case.v_new, case.slot_mapping, case.k_cache, case.v_cache,
+                    workspace=ws)
+        if attn_events is not None:
+            attn_events[0].record()
+        pa.attention_varlen(case.q, case.k_cache, case.v_cache, case.block_tables, case.seq_lens,
+                            case.query_start_loc, case.num_kv_heads, case.scale, case.causal, out,
+                            max_query_len=mql, max_seq_len=msl, workspace=ws)
+        if attn_events is not None:
+            attn_events[1].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, bits = pa.get_error(ws)
+    if st != 0:
+        raise RuntimeError(f"device error word {bits:#x} after warm-up")
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    st, bits = pa.get_error(ws)
+    if st != 0:
+        raise RuntimeError(f"device error word {bits:#x} in the timed region")
+
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    max_ms = float(t.item())
+    bytes_step = scatter_bytes(case) + attention_bytes(case)
+    total_bytes = bytes_step * args.steps * world
+    value = total_bytes / (max_ms * 1e-3) / 1e9
+
+    # end to end through the public API: pinned host inputs in, output back, every step
+    e2e = run_e2e(pa, case, args, dev, ws)
+    if world > 1:
+        te = torch.tensor([e2e["ms"]], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
+        e2e["ms"] = float(te.item())
+    e2e_value = bytes_step * args.steps * world / (e2e["ms"] * 1e-3) / 1e9
+
+    attn_bytes = attention_bytes(case)
+    achieved = attn_bytes / (attn_ms * 1e-3) / 1e9
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16; per-rank seed 1002+rank)",
+        "config": {"workload": WORKLOAD, "global_batch": 64 * world, "seq_len": "256-4096",
+                   "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
+                   "l2": "inputs larger than L2 (0.57 GB of K/V per step vs 126 MB L2)"},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
+                     "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                     "traffic": args.traffic,
+                     "kernel": "pa_attention_varlen (plan + split-KV decode), per-call events",
+                     "peak_kind": peak_kind},
+        "clocks": clk,
+        "gpu_launches": 3 * args.steps,
+    }
+    return result, case
+
+
+def run_e2e(pa, case, args, dev, ws):
+    """The same step through the public API with host-resident inputs/outputs."""
+    names = ["q", "k_new", "v_new", "slot_mapping", "block_tables", "seq_lens", "query_start_loc"]
+    host = {n: getattr(case, n).cpu().pin_memory() for n in names}
+    devt = {n: torch.empty_like(getattr(case, n)) for n in names}
+    out_h = torch.empty(case.q.shape, dtype=case.q.dtype).pin_memory()
+    out_d = torch.empty_like(case.q)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+    steps = max(1, min(args.steps, 500))
+
+    def step():
+        for n in names:
+            devt[n].copy_(host[n], non_blocking=True)
+        pa.write_kv(devt["k_new"], devt["v_new"], devt["slot_mapping"], case.k_cache,
+                    case.v_cache, workspace=ws)
+        pa.attention_varlen(devt["q"], case.k_cache, case.v_cache, devt["block_tables"],
+                            devt["seq_lens"], devt["query_start_loc"], case.num_kv_heads,
+                            case.scale, case.causal, out_d, max_query_len=case.max_query_len,
+                            max_seq_len=case.max_seq_len, workspace=ws)
+        out_h.copy_(out_d, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) * args.steps / steps
+    return {"ms": ms, "h2d": h2d, "d2h": d2h}
+
+
+# ---------------------------------------------------------------------------
+# oracle legs (CPU)
+# ---------------------------------------------------------------------------
+
+def oracle_decode_sample(num_seqs, seed=1002):
+    """A bounded sample of the decode workload for the CPU oracle."""
+    return workloads.decode_batch(num_seqs=num_seqs, seed=seed)
+
+
+def time_oracle_step(case):
+    import oracle
+    kc = workloads.bf16_bits(case.k_cache).copy()
+    vc = workloads.bf16_bits(case.v_cache).copy()
+    q = workloads.bf16_bits(case.q)
+    kn, vn = workloads.bf16_bits(case.k_new), workloads.bf16_bits(case.v_new)
+    kl, vl = workloads.bf16_bits(case.k_logical), workloads.bf16_bits(case.v_logical)
+    t0 = time.perf_counter()
+    oracle.write_kv(kn, vn, case.slot_mapping.numpy(), kc, vc, case.block_size)
+    oracle.attention_varlen(q, kl, vl, case.kv_offsets.numpy(), case.seq_lens.numpy(),
+                            case.query_start_loc.numpy(), case.num_kv_heads, case.scale,
+                            case.causal)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(budget_s=12.0):
+    import oracle
+    oracle.build()
+    case = oracle_decode_sample(64)
+    nbytes = scatter_bytes(case) + attention_bytes(case)
+    times = []
+    t_begin = time.perf_counter()
+    while not times or (time.perf_counter() - t_begin < budget_s and len(times) < 20):
+        times.append(time_oracle_step(case))
+    gbs = nbytes * len(times) / sum(times) / 1e9
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"the full 64-sequence decode batch (seed 1002), {len(times)} passes of "
+                      f"oracle write_kv + fp64 attention ({sum(times):.1f} s)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+    oracle.build()
+    # each step: one decode sequence of the workload (cycling), so K steps stay bounded
+    full = oracle_decode_sample(64)
+    sub = []
+    import dataclasses
+    for s in range(64):
+        sub.append(oracle_decode_sample(1, seed=1002 + 1000 * (s + 1)))
+    for _ in range(min(args.warmup, 3)):
+        time_oracle_step(sub[0])
+    times, nbytes = [], 0
+    for i in range(args.steps):
+        c = sub[i % len(sub)]
+        times.append(time_oracle_step(c))
+        nbytes += scatter_bytes(c) + attention_bytes(c)
+    total = sum(times)
+    gbs = nbytes / total / 1e9
+    del full
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": 64, "seq_len": "256-4096",
+                   "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": "each step: one decode sequence drawn from the workload's "
+                                   "distribution (context U[256,4096]), oracle write + attention"},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-components", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="dram bytes per dominant-kernel launch from an ncu capture, if current")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        result, case = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            hbm_peak, tc_peak, tc_sust, peak_kind = measured_peaks()
+            if world == 1 and not args.no_components:
+                del case
+                torch.cuda.empty_cache()
+                import paged_kv_gqa_reshape_b200 as pa
+                result["components"] = components(pa, hbm_peak, tc_peak, peak_kind)
+            if world == 1 and not args.no_cpu_baseline:
+                result["cpu_baseline"] = cpu_baseline()
+            print(json.dumps(result), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

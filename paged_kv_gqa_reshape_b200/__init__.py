@@ -1,0 +1,234 @@
+"""B200-native paged KV attention: Python binding of libpa.so (include/pa.h).
+
+This module only marshals arguments: it checks tensor dtypes/shapes, passes
+raw device pointers and the current CUDA stream to the C ABI, and turns a
+non-zero status into an exception.  Every step of the computation runs in
+the library's sm_100a kernels; there is no fallback path.  If the library
+cannot be loaded the calls raise.
+
+Calls (names as in the C ABI, without the ``pa_`` prefix):
+
+* ``write_kv(k, v, slot_mapping, k_cache, v_cache)``
+* ``attention_varlen(q, k_cache, v_cache, block_tables, seq_lens,
+  query_start_loc, num_kv_heads, scale, causal, out)``
+* ``attention_smallseq(q, k, v, cu_seqlens_kv, scale, out)``
+* ``get_error(workspace)`` / ``status_string(status)``
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "PaError", "library_path", "load", "write_kv", "attention_varlen", "attention_smallseq",
+    "varlen_workspace_size", "varlen_workspace", "error_workspace", "get_error",
+    "status_string", "version", "EXPORTED_SYMBOLS",
+    "DEVERR_SLOT", "DEVERR_BLOCK", "DEVERR_LENGTHS", "DEVERR_QLEN", "DEVERR_HINT",
+    "DEVERR_TIMEOUT", "ERROR_WORD_BYTES",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+PA_OK = 0
+DEVERR_SLOT, DEVERR_BLOCK, DEVERR_LENGTHS = 0x1, 0x2, 0x4
+DEVERR_QLEN, DEVERR_HINT, DEVERR_TIMEOUT = 0x8, 0x10, 0x20
+ERROR_WORD_BYTES = 256
+
+EXPORTED_SYMBOLS = (
+    "pa_write_kv", "pa_attention_varlen_workspace_size", "pa_attention_varlen",
+    "pa_attention_smallseq", "pa_get_error", "pa_status_string", "pa_version",
+)
+
+_lib = None
+_lock = threading.Lock()
+
+
+class PaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)}")
+        self.status = status
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libpa.so")
+
+
+def load(build_if_missing: bool = True):
+    """Load libpa.so (building it with nvcc first if it is missing or stale)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if build_if_missing:
+            from . import _build
+            try:
+                _build.build()
+            except Exception as e:  # the library must exist: no fallback
+                if not os.path.exists(library_path()):
+                    raise RuntimeError(f"libpa.so is missing and could not be built: {e}") from e
+        try:
+            lib = ctypes.CDLL(library_path())
+        except OSError as e:
+            raise RuntimeError(f"cannot load the CUDA library {library_path()}: {e}") from e
+        p, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+        lib.pa_write_kv.restype = ctypes.c_int
+        lib.pa_write_kv.argtypes = [p, p, p, i64, i32, i32, p, p, i64, i32, p, p]
+        lib.pa_attention_varlen_workspace_size.restype = ctypes.c_size_t
+        lib.pa_attention_varlen_workspace_size.argtypes = [i32, i64, i32, i32, i32]
+        lib.pa_attention_varlen.restype = ctypes.c_int
+        lib.pa_attention_varlen.argtypes = [
+            p, p, p, p, i32, p, p, i32, i64, i32, i32, i32, i32, i64, i32, i32,
+            ctypes.c_float, i32, p, p, ctypes.c_size_t, p]
+        lib.pa_attention_smallseq.restype = ctypes.c_int
+        lib.pa_attention_smallseq.argtypes = [p, p, p, p, i32, i32, i32, i32, i32,
+                                              ctypes.c_float, p, p, p]
+        lib.pa_get_error.restype = ctypes.c_int
+        lib.pa_get_error.argtypes = [p, p, ctypes.POINTER(ctypes.c_uint32)]
+        lib.pa_status_string.restype = ctypes.c_char_p
+        lib.pa_status_string.argtypes = [ctypes.c_int]
+        lib.pa_version.restype = ctypes.c_char_p
+        lib.pa_version.argtypes = []
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load().pa_status_string(int(status)).decode()
+
+
+def version() -> str:
+    return load().pa_version().decode()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(t: torch.Tensor, name: str, dtype, ndim: Optional[int] = None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+
+
+def _raise(status: int, where: str):
+    if status != PA_OK:
+        raise PaError(status, where)
+
+
+def error_workspace(device=None) -> torch.Tensor:
+    """A zeroed workspace holding only the device error word."""
+    return torch.zeros(ERROR_WORD_BYTES, dtype=torch.uint8, device=device or "cuda")
+
+
+def varlen_workspace_size(num_seqs, num_q_tokens, num_q_heads, num_kv_heads, head_dim) -> int:
+    return int(load().pa_attention_varlen_workspace_size(num_seqs, num_q_tokens, num_q_heads,
+                                                         num_kv_heads, head_dim))
+
+
+def varlen_workspace(num_seqs, num_q_tokens, num_q_heads, num_kv_heads, head_dim,
+                     device=None) -> torch.Tensor:
+    """A zero-initialised workspace for attention_varlen with these sizes."""
+    n = varlen_workspace_size(num_seqs, num_q_tokens, num_q_heads, num_kv_heads, head_dim)
+    return torch.zeros(max(n, ERROR_WORD_BYTES), dtype=torch.uint8, device=device or "cuda")
+
+
+def write_kv(k, v, slot_mapping, k_cache, v_cache, workspace=None, stream=None):
+    """Scatter k/v [T, Hkv, D] into the paged caches at slot_mapping (int64 [T])."""
+    _check(k, "k", torch.bfloat16, 3)
+    _check(v, "v", torch.bfloat16, 3)
+    _check(slot_mapping, "slot_mapping", torch.int64, 1)
+    _check(k_cache, "k_cache", torch.bfloat16, 4)
+    _check(v_cache, "v_cache", torch.bfloat16, 4)
+    t, hkv, d = k.shape
+    if v.shape != k.shape or slot_mapping.shape[0] != t:
+        raise ValueError("k, v and slot_mapping disagree on the token count / shape")
+    nb, bs, hkv_c, d_c = k_cache.shape
+    if v_cache.shape != k_cache.shape or hkv_c != hkv or d_c != d:
+        raise ValueError("cache shape does not match k/v")
+    ws = workspace.data_ptr() if workspace is not None else None
+    st = load().pa_write_kv(k.data_ptr(), v.data_ptr(), slot_mapping.data_ptr(), t, hkv, d,
+                            k_cache.data_ptr(), v_cache.data_ptr(), nb, bs, ws, _stream(stream))
+    _raise(st, "pa_write_kv")
+
+
+def attention_varlen(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc,
+                     num_kv_heads, scale, causal, out, max_query_len=None, max_seq_len=None,
+                     workspace=None, stream=None):
+    """Paged varlen attention; writes out [T, Hq, D] (bf16).
+
+    max_query_len / max_seq_len are host-side hints (the metadata builder's
+    maxima); when omitted the safe bounds (all tokens / the block table's
+    reach) are used, which never forces a device synchronisation.
+    """
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_cache, "k_cache", torch.bfloat16, 4)
+    _check(v_cache, "v_cache", torch.bfloat16, 4)
+    _check(block_tables, "block_tables", torch.int32, 2)
+    _check(seq_lens, "seq_lens", torch.int32, 1)
+    _check(query_start_loc, "query_start_loc", torch.int32, 1)
+    _check(out, "out", torch.bfloat16, 3)
+    t, hq, d = q.shape
+    nb, bs, hkv, d_c = k_cache.shape
+    if hkv != num_kv_heads or d_c != d or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shape does not match q / num_kv_heads")
+    if out.shape != q.shape:
+        raise ValueError("out must have q's shape")
+    s = seq_lens.shape[0]
+    if query_start_loc.shape[0] != s + 1 or block_tables.shape[0] != s:
+        raise ValueError("seq_lens, query_start_loc and block_tables disagree on num_seqs")
+    mb = block_tables.shape[1]
+    mql = t if max_query_len is None else int(max_query_len)
+    msl = mb * bs if max_seq_len is None else int(max_seq_len)
+    if workspace is None:
+        workspace = varlen_workspace(s, t, hq, hkv, d, device=q.device)
+    st = load().pa_attention_varlen(
+        q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(), mb,
+        seq_lens.data_ptr(), query_start_loc.data_ptr(), s, t, hq, hkv, d, bs, nb, mql, msl,
+        float(scale), int(bool(causal)), out.data_ptr(), workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _raise(st, "pa_attention_varlen")
+    return out
+
+
+def attention_smallseq(q, k, v, cu_seqlens_kv, scale, out, max_seqlen_kv=16, workspace=None,
+                       stream=None):
+    """s_q = 1 attention over <= 16 contiguous keys per entry; writes out [B, Hq, D]."""
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k, "k", torch.bfloat16, 3)
+    _check(v, "v", torch.bfloat16, 3)
+    _check(cu_seqlens_kv, "cu_seqlens_kv", torch.int32, 1)
+    _check(out, "out", torch.bfloat16, 3)
+    b, hq, d = q.shape
+    _, hkv, d_k = k.shape
+    if d_k != d or v.shape != k.shape or out.shape != q.shape or cu_seqlens_kv.shape[0] != b + 1:
+        raise ValueError("inconsistent small-seq shapes")
+    ws = workspace.data_ptr() if workspace is not None else None
+    st = load().pa_attention_smallseq(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                      cu_seqlens_kv.data_ptr(), b, hq, hkv, d,
+                                      int(max_seqlen_kv), float(scale), out.data_ptr(), ws,
+                                      _stream(stream))
+    _raise(st, "pa_attention_smallseq")
+    return out
+
+
+def get_error(workspace, stream=None):
+    """Synchronise, read and clear the workspace's device error word: (status, bits)."""
+    bits = ctypes.c_uint32(0)
+    st = load().pa_get_error(workspace.data_ptr(), _stream(stream), ctypes.byref(bits))
+    return int(st), int(bits.value)

@@ -1,0 +1,279 @@
+// C ABI (include/pa.h): argument checks, workspace layout, launches.
+//
+// Every host-visible problem is rejected before anything is launched or
+// written (the reject-before-write rule of TensorRT-LLM PR "CSA2 Vanilla
+// sparse attention", description).  The library allocates no device memory;
+// its only state is a per-device SM count and the lazily resolved driver
+// entry point used to encode TMA tensor maps.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/pa.h"
+#include "kernels.h"
+#include "layout.h"
+
+namespace {
+
+using pa::WorkspaceLayout;
+
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices];
+std::mutex g_mu;
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_sm_count[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    g_sm_count[dev] = n;
+  }
+  return g_sm_count[dev];
+}
+
+bool log_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("PA_LOG");
+    v = (e && *e && strcmp(e, "0") != 0) ? 1 : 0;
+  }
+  return v == 1;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- cuTensorMapEncodeTiled through the runtime's driver entry point ------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// bf16 tensor map with a 128-byte swizzle; dims/strides innermost first.
+bool make_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+              const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t estride[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+                  dims, strides_bytes, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pa_status_string(pa_status s) {
+  switch (s) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG: bad argument (nothing was launched)";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: request outside this build's support";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA: a CUDA call failed";
+    case PA_ERR_DEVICE_INDEX: return "PA_ERR_DEVICE_INDEX: the device saw a bad index or length";
+    case PA_ERR_TIMEOUT: return "PA_ERR_TIMEOUT: a bounded device wait gave up";
+  }
+  return "pa: unknown status";
+}
+
+const char* pa_version(void) { return "pa 0.1 sm_100a"; }
+
+pa_status pa_write_kv(const void* k, const void* v, const int64_t* slot_mapping,
+                      int64_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                      void* k_cache, void* v_cache, int64_t num_blocks, int32_t block_size,
+                      void* workspace, void* stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || head_dim % 8 != 0 ||
+      num_blocks <= 0 || block_size <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+    return PA_ERR_INVALID_ARG;
+  const int row_vecs = num_kv_heads * head_dim / 8;
+  uint32_t* err = workspace ? static_cast<uint32_t*>(workspace) : nullptr;
+  cudaError_t e = pa::launch_write_kv(k, v, slot_mapping, num_tokens, row_vecs, k_cache, v_cache,
+                                      num_blocks * (int64_t)block_size, err, sm_count(),
+                                      static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+size_t pa_attention_varlen_workspace_size(int32_t num_seqs, int64_t num_q_tokens,
+                                          int32_t num_q_heads, int32_t num_kv_heads,
+                                          int32_t head_dim) {
+  if (num_seqs < 0 || num_q_tokens < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+    return 0;
+  return pa::make_layout(num_seqs, num_q_tokens, num_q_heads, num_kv_heads, head_dim).total;
+}
+
+pa_status pa_attention_varlen(const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* block_tables, int32_t max_blocks_per_seq,
+                              const int32_t* seq_lens, const int32_t* query_start_loc,
+                              int32_t num_seqs, int64_t num_q_tokens, int32_t num_q_heads,
+                              int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                              int64_t num_blocks, int32_t max_query_len, int32_t max_seq_len,
+                              float scale, int32_t causal, void* out, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  // ---- host-visible checks (nothing launched yet) ----
+  if (num_seqs < 0 || num_q_tokens < 0 || num_q_tokens > 0x7fffffffll || num_q_heads <= 0 ||
+      num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || max_blocks_per_seq <= 0 ||
+      num_blocks <= 0 || num_blocks > 0x7fffffffll || max_query_len < 0 || max_seq_len < 0 ||
+      (causal != 0 && causal != 1) || !isfinite(scale))
+    return PA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (block_size != pa::kPageKeys) return PA_ERR_UNSUPPORTED;
+  const int group = num_q_heads / num_kv_heads;
+  if (group > 16) return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0 || num_q_tokens == 0) return PA_OK;
+  if (!q || !k_cache || !v_cache || !block_tables || !seq_lens || !query_start_loc || !out ||
+      !workspace)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+      (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(query_start_loc) & 3u))
+    return PA_ERR_INVALID_ARG;
+  const WorkspaceLayout L =
+      pa::make_layout(num_seqs, num_q_tokens, num_q_heads, num_kv_heads, head_dim);
+  if (workspace_bytes < L.total) return PA_ERR_INVALID_ARG;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  const int nsm = sm_count();
+  const float scale_log2 = scale * 1.4426950408889634f;
+  const bool run_prefill = max_query_len > 1;
+
+  CUtensorMap q_map, k_map, v_map;
+  if (run_prefill) {
+    const cuuint32_t box_q[3] = {64, 1, (cuuint32_t)pa::kPrefillTileM};
+    const cuuint64_t dq[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_q_heads,
+                              (cuuint64_t)num_q_tokens};
+    const cuuint64_t sq[2] = {(cuuint64_t)head_dim * 2, (cuuint64_t)num_q_heads * head_dim * 2};
+    const cuuint32_t box_kv[4] = {64, 1, (cuuint32_t)pa::kPageKeys, 1};
+    const cuuint64_t dkv[4] = {(cuuint64_t)head_dim, (cuuint64_t)num_kv_heads,
+                               (cuuint64_t)block_size, (cuuint64_t)num_blocks};
+    const cuuint64_t skv[3] = {(cuuint64_t)head_dim * 2, (cuuint64_t)num_kv_heads * head_dim * 2,
+                               (cuuint64_t)block_size * num_kv_heads * head_dim * 2};
+    if (!make_map(&q_map, q, 3, dq, sq, box_q) || !make_map(&k_map, k_cache, 4, dkv, skv, box_kv) ||
+        !make_map(&v_map, v_cache, 4, dkv, skv, box_kv))
+      return PA_ERR_CUDA;
+  }
+
+  const int target_items = nsm * 2 * 4 < pa::kDecodeMaxItems ? nsm * 2 * 4 : pa::kDecodeMaxItems;
+  pa::launch_plan(query_start_loc, seq_lens, num_seqs, num_q_tokens, max_blocks_per_seq,
+                  block_size, max_query_len, max_seq_len, causal, num_kv_heads, target_items, ws,
+                  L, st);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return PA_ERR_CUDA;
+
+  if (run_prefill) {
+    pa::PrefillParams pp{};
+    pp.block_tables = block_tables;
+    pp.max_blocks_per_seq = max_blocks_per_seq;
+    pp.num_q_heads = num_q_heads;
+    pp.num_kv_heads = num_kv_heads;
+    pp.group = group;
+    pp.num_blocks = num_blocks;
+    pp.num_q_tokens = num_q_tokens;
+    pp.scale_log2 = scale_log2;
+    pp.causal = causal;
+    pp.out = static_cast<__nv_bfloat16*>(out);
+    pp.ws = ws;
+    pp.L = L;
+    e = pa::launch_prefill(pp, q_map, k_map, v_map, head_dim, nsm, st);
+    if (e != cudaSuccess) return PA_ERR_CUDA;
+  }
+
+  pa::DecodeParams dp{};
+  dp.q = static_cast<const __nv_bfloat16*>(q);
+  dp.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
+  dp.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
+  dp.block_tables = block_tables;
+  dp.max_blocks_per_seq = max_blocks_per_seq;
+  dp.num_q_heads = num_q_heads;
+  dp.num_kv_heads = num_kv_heads;
+  dp.group = group;
+  dp.num_blocks = num_blocks;
+  dp.scale_log2 = scale_log2;
+  dp.out = static_cast<__nv_bfloat16*>(out);
+  dp.ws = ws;
+  dp.L = L;
+  e = pa::launch_decode(dp, head_dim, nsm * 2, st);
+  if (log_enabled())
+    fprintf(stderr, "[pa] varlen S=%d T=%lld Hq=%d Hkv=%d D=%d prefill=%d sms=%d\n", num_seqs,
+            (long long)num_q_tokens, num_q_heads, num_kv_heads, head_dim, (int)run_prefill, nsm);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_attention_smallseq(const void* q, const void* k, const void* v,
+                                const int32_t* cu_seqlens_kv, int32_t batch, int32_t num_q_heads,
+                                int32_t num_kv_heads, int32_t head_dim, int32_t max_seqlen_kv,
+                                float scale, void* out, void* workspace, void* stream) {
+  if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
+      max_seqlen_kv < 0 || !isfinite(scale))
+    return PA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (max_seqlen_kv > 16) return PA_ERR_UNSUPPORTED;
+  if (batch == 0) return PA_OK;
+  if (!q || !k || !v || !cu_seqlens_kv || !out) return PA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_kv) & 3u) || (workspace && !aligned16(workspace)))
+    return PA_ERR_INVALID_ARG;
+  pa::SmallSeqParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.cu_seqlens_kv = cu_seqlens_kv;
+  p.batch = batch;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.group = num_q_heads / num_kv_heads;
+  p.max_seqlen_kv = max_seqlen_kv;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.err = static_cast<uint32_t*>(workspace);
+  cudaError_t e = pa::launch_smallseq(p, head_dim, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_get_error(void* workspace, void* stream, uint32_t* bits) {
+  if (bits) *bits = 0;
+  if (!workspace) return PA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof word, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, sizeof word, st) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return PA_ERR_CUDA;
+  if (bits) *bits = word;
+  if (word == 0) return PA_OK;
+  return (word & PA_DEVERR_TIMEOUT) ? PA_ERR_TIMEOUT : PA_ERR_DEVICE_INDEX;
+}
+
+}  // extern "C"

@@ -1,0 +1,80 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "layout.h"
+
+namespace pa {
+
+// ---- KV scatter ------------------------------------------------------------
+cudaError_t launch_write_kv(const void* k, const void* v, const int64_t* slot_mapping,
+                            int64_t num_tokens, int row_vecs, void* k_cache, void* v_cache,
+                            int64_t num_slots, uint32_t* err, int num_sms, cudaStream_t stream);
+
+// ---- plan ------------------------------------------------------------------
+void launch_plan(const int32_t* query_start_loc, const int32_t* seq_lens, int num_seqs,
+                 long long num_q_tokens, int max_blocks_per_seq, int block_size,
+                 int max_query_len, int max_seq_len, int causal, int num_kv_heads,
+                 int target_items, unsigned char* ws, const WorkspaceLayout& L,
+                 cudaStream_t stream);
+
+// ---- split-KV decode -------------------------------------------------------
+struct DecodeParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k_cache;
+  const __nv_bfloat16* v_cache;
+  const int32_t* block_tables;
+  int max_blocks_per_seq;
+  int num_q_heads;
+  int num_kv_heads;
+  int group;  // num_q_heads / num_kv_heads, <= 16
+  long long num_blocks;
+  float scale_log2;  // scale * log2(e)
+  __nv_bfloat16* out;
+  unsigned char* ws;
+  WorkspaceLayout L;
+};
+cudaError_t launch_decode(const DecodeParams& p, int head_dim, int grid, cudaStream_t stream);
+
+// ---- tcgen05 prefill ------------------------------------------------------
+struct PrefillParams {
+  const int32_t* block_tables;
+  int max_blocks_per_seq;
+  int num_q_heads;
+  int num_kv_heads;
+  int group;
+  long long num_blocks;
+  long long num_q_tokens;
+  float scale_log2;
+  int causal;
+  __nv_bfloat16* out;
+  unsigned char* ws;
+  WorkspaceLayout L;
+};
+// Tensor maps are built by the host layer (they need the driver entry point).
+cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& q_map,
+                           const CUtensorMap& k_map, const CUtensorMap& v_map, int head_dim,
+                           int grid, cudaStream_t stream);
+
+// ---- small-seq -------------------------------------------------------------
+struct SmallSeqParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const int32_t* cu_seqlens_kv;
+  int batch;
+  int num_q_heads;
+  int num_kv_heads;
+  int group;
+  int max_seqlen_kv;
+  float scale_log2;
+  __nv_bfloat16* out;
+  uint32_t* err;
+};
+cudaError_t launch_smallseq(const SmallSeqParams& p, int head_dim, cudaStream_t stream);
+
+}  // namespace pa

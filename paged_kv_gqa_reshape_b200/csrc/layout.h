@@ -1,0 +1,80 @@
+// Workspace layout and per-call work plan shared by the host API and the
+// kernels.  Everything here is sized from call arguments only, so the host
+// can size the workspace without touching the device.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+namespace pa {
+
+constexpr int kPrefillTileM = 128;      // query rows per prefill tile (tcgen05 M)
+constexpr int kPrefillTileN = 128;      // keys per prefill KV tile (tcgen05 N)
+constexpr int kDecodeWarps = 4;         // warps per decode CTA
+constexpr int kPageKeys = 16;           // block_size this build supports
+constexpr int kDecodeMinChunk = 256;    // smallest split-KV chunk (keys)
+constexpr int kDecodeMaxItems = 4096;   // upper bound on planned (seq, chunk) pairs beyond S
+constexpr int kCostBuckets = 4096;      // prefill tiles are sorted by KV-tile count
+
+// Sanitised geometry of one sequence, written by the plan kernel.  The
+// attention kernels read lengths only from here, never from the raw inputs.
+struct SeqInfo {
+  int32_t q_start;    // first query token of the sequence
+  int32_t q_len;      // number of query tokens (0 if the sequence is skipped)
+  int32_t kv_len;     // number of keys (clamped to the block table's reach)
+  int32_t n_chunks;   // decode only: split-KV chunks (0 for non-decode sequences)
+  int32_t pair_base;  // decode only: index of the first (seq, chunk) pair
+  int32_t chunk_len;  // decode only: keys per chunk (multiple of 64)
+  int32_t pad0, pad1;
+};
+
+struct PlanHeader {
+  int32_t num_prefill_tiles;  // entries in the prefill tile list
+  int32_t num_decode_pairs;   // entries in the decode (seq, chunk) list
+  int32_t total_decode_keys;
+  int32_t pad[61];
+};
+
+struct WorkspaceLayout {
+  size_t err;        // uint32 error word (PA_ERROR_WORD_BYTES reserved)
+  size_t header;     // PlanHeader
+  size_t seq_info;   // SeqInfo[num_seqs]
+  size_t tiles;      // int2[max_tiles]   (seq, first query row of the tile)
+  size_t pairs;      // int2[max_pairs]   (seq, chunk)
+  size_t counters;   // int32[num_seqs * num_kv_heads]  split-KV arrival counters
+  size_t lse;        // float[max_pairs * num_q_heads]   log2-sum-exp per partial
+  size_t partial;    // float[max_pairs * num_q_heads * head_dim]
+  size_t total;
+  int64_t max_tiles;
+  int64_t max_pairs;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline WorkspaceLayout make_layout(int64_t num_seqs, int64_t num_q_tokens, int64_t num_q_heads,
+                                   int64_t num_kv_heads, int64_t head_dim) {
+  WorkspaceLayout L{};
+  size_t off = 0;
+  L.err = off;
+  off += 256;
+  L.header = off;
+  off += sizeof(PlanHeader);
+  L.seq_info = off;
+  off = align_up(off + sizeof(SeqInfo) * (size_t)num_seqs, 256);
+  L.max_tiles = (num_q_tokens + kPrefillTileM - 1) / kPrefillTileM + num_seqs;
+  L.tiles = off;
+  off = align_up(off + 8 * (size_t)L.max_tiles, 256);
+  L.max_pairs = kDecodeMaxItems + num_seqs;
+  L.pairs = off;
+  off = align_up(off + 8 * (size_t)L.max_pairs, 256);
+  L.counters = off;
+  off = align_up(off + 4 * (size_t)(num_seqs * num_kv_heads), 256);
+  L.lse = off;
+  off = align_up(off + 4 * (size_t)(L.max_pairs * num_q_heads), 256);
+  L.partial = off;
+  off = align_up(off + 4 * (size_t)(L.max_pairs * num_q_heads * head_dim), 256);
+  L.total = off;
+  return L;
+}
+
+}  // namespace pa

@@ -1,0 +1,220 @@
+// Work planning on the device (one CTA), so no length ever travels to the host.
+//
+// Reads query_start_loc and seq_lens, sanitises them into SeqInfo, and builds
+//  - the prefill tile list: one entry per 128-query-row tile of every
+//    sequence with more than one query, ordered by descending KV-tile count
+//    (longest work first, for the persistent prefill grid);
+//  - the decode list: one (seq, chunk) pair per split-KV chunk of every
+//    single-query sequence, with a chunk length chosen from the total decode
+//    key count so that the decode grid gets a few items per CTA;
+//  - zeroed split-KV arrival counters.
+// This plays the role of the device-side runtime length reduction of
+// ROCm/TransformerEngine PR #461 (description: the real maximum is found on
+// the device before routing), without any host synchronisation.
+#include "common.cuh"
+#include "layout.h"
+
+namespace pa {
+
+namespace {
+
+constexpr int kPlanThreads = 1024;
+
+// Block-wide exclusive scan of one int per thread; returns the block total.
+__device__ int block_exclusive_scan(int v, int* out_excl, int* s_warp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_warp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = (lane < (int)(blockDim.x >> 5)) ? s_warp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    s_warp[lane] = w;  // inclusive warp totals
+  }
+  __syncthreads();
+  int warp_prefix = warp ? s_warp[warp - 1] : 0;
+  *out_excl = warp_prefix + x - v;
+  int total = s_warp[(blockDim.x >> 5) - 1];
+  __syncthreads();
+  return total;
+}
+
+__device__ __forceinline__ int tile_cost(const SeqInfo& si, int row0, int causal) {
+  int last_row = min(si.q_len, row0 + kPrefillTileM) - 1;
+  int vis = si.kv_len;
+  if (causal) vis = max(0, min(si.kv_len, si.kv_len - si.q_len + last_row + 1));
+  return (vis + kPrefillTileN - 1) / kPrefillTileN;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kPlanThreads, 1)
+    plan_kernel(const int32_t* __restrict__ query_start_loc, const int32_t* __restrict__ seq_lens,
+                int num_seqs, long long num_q_tokens, int max_blocks_per_seq, int block_size,
+                int max_query_len, int max_seq_len, int causal, int num_kv_heads,
+                int target_items, unsigned char* ws, WorkspaceLayout L) {
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws + L.err);
+  PlanHeader* hdr = reinterpret_cast<PlanHeader*>(ws + L.header);
+  SeqInfo* info = reinterpret_cast<SeqInfo*>(ws + L.seq_info);
+  int2* tiles = reinterpret_cast<int2*>(ws + L.tiles);
+  int2* pairs = reinterpret_cast<int2*>(ws + L.pairs);
+  int32_t* counters = reinterpret_cast<int32_t*>(ws + L.counters);
+
+  __shared__ int s_warp[32];
+  __shared__ unsigned long long s_dec_keys;
+  __shared__ int s_hist[kCostBuckets];
+  __shared__ int s_carry;
+  __shared__ uint32_t s_err;
+
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    s_dec_keys = 0;
+    s_err = 0;
+  }
+  for (int i = tid; i < kCostBuckets; i += blockDim.x) s_hist[i] = 0;
+  for (long long i = tid; i < (long long)num_seqs * num_kv_heads; i += blockDim.x)
+    counters[i] = 0;
+  __syncthreads();
+
+  // ---- pass 1: sanitise lengths, total decode keys -------------------------
+  const long long reach = (long long)max_blocks_per_seq * block_size;
+  for (int s = tid; s < num_seqs; s += blockDim.x) {
+    uint32_t e = 0;
+    long long qs = query_start_loc[s], qe = query_start_loc[s + 1];
+    long long kv = seq_lens[s];
+    if (qs < 0 || qe < qs || qe > num_q_tokens) {
+      e |= PA_DEVERR_LENGTHS;
+      qe = qs = max(0ll, min(qs, num_q_tokens));
+    }
+    if (kv < 0) {
+      e |= PA_DEVERR_LENGTHS;
+      kv = 0;
+    }
+    if (kv > reach) {
+      e |= PA_DEVERR_LENGTHS;
+      kv = reach;
+    }
+    long long ql = qe - qs;
+    if (ql > kv) e |= PA_DEVERR_QLEN;
+    if (ql > max_query_len || kv > max_seq_len) e |= PA_DEVERR_HINT;
+    SeqInfo si;
+    si.q_start = (int)qs;
+    si.q_len = (int)ql;
+    si.kv_len = (int)kv;
+    si.n_chunks = 0;
+    si.pair_base = 0;
+    si.chunk_len = 0;
+    si.pad0 = si.pad1 = 0;
+    info[s] = si;
+    if (ql == 1) atomicAdd(&s_dec_keys, (unsigned long long)kv);
+    if (e) atomicOr(&s_err, e);
+  }
+  __syncthreads();
+
+  // split-KV chunk: enough chunks for ~target_items (seq, chunk, kv-head)
+  // items, never below kDecodeMinChunk keys, always a multiple of 64 keys
+  long long want = ((long long)s_dec_keys * num_kv_heads + target_items - 1) / max(target_items, 1);
+  int chunk = (int)max((long long)kDecodeMinChunk, min(want, (long long)1 << 30));
+  chunk = (chunk + 63) / 64 * 64;
+
+  // ---- pass 2: chunk counts, tile histogram ---------------------------------
+  if (tid == 0) s_carry = 0;
+  __syncthreads();
+  for (int base = 0; base < num_seqs; base += blockDim.x) {
+    int s = base + tid;
+    int n_chunks = 0;
+    SeqInfo si;
+    if (s < num_seqs) {
+      si = info[s];
+      if (si.q_len == 1) n_chunks = max(1, (si.kv_len + chunk - 1) / chunk);
+      if (si.q_len > 1) {
+        for (int r = 0; r < si.q_len; r += kPrefillTileM) {
+          int c = tile_cost(si, r, causal);
+          atomicAdd(&s_hist[kCostBuckets - 1 - min(c, kCostBuckets - 1)], 1);
+        }
+      }
+    }
+    int excl;
+    int total = block_exclusive_scan(n_chunks, &excl, s_warp);
+    if (s < num_seqs && n_chunks) {
+      int pb = s_carry + excl;
+      info[s].n_chunks = n_chunks;
+      info[s].pair_base = pb;
+      info[s].chunk_len = chunk;
+      for (int c = 0; c < n_chunks; ++c)
+        if ((long long)(pb + c) < (long long)L.max_pairs) pairs[pb + c] = make_int2(s, c);
+    }
+    __syncthreads();
+    if (tid == 0) s_carry += total;
+    __syncthreads();
+  }
+  int num_pairs = s_carry;
+  if ((long long)num_pairs > (long long)L.max_pairs) {  // cannot happen for target_items <= kDecodeMaxItems
+    if (tid == 0) atomicOr(&s_err, PA_DEVERR_LENGTHS);
+    num_pairs = (int)L.max_pairs;
+  }
+
+  // ---- pass 3: counting sort of prefill tiles by descending cost -----------
+  // exclusive scan of the histogram (bucket 0 = most expensive)
+  {
+    constexpr int per = kCostBuckets / kPlanThreads;
+    int local[per];
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < per; ++i) {
+      local[i] = s_hist[tid * per + i];
+      sum += local[i];
+    }
+    int excl;
+    block_exclusive_scan(sum, &excl, s_warp);
+#pragma unroll
+    for (int i = 0; i < per; ++i) {
+      s_hist[tid * per + i] = excl;
+      excl += local[i];
+    }
+  }
+  __syncthreads();
+  int num_tiles = 0;
+  for (int s = tid; s < num_seqs; s += blockDim.x) {
+    SeqInfo si = info[s];
+    if (si.q_len > 1) {
+      for (int r = 0; r < si.q_len; r += kPrefillTileM) {
+        int c = tile_cost(si, r, causal);
+        int pos = atomicAdd(&s_hist[kCostBuckets - 1 - min(c, kCostBuckets - 1)], 1);
+        if ((long long)pos < (long long)L.max_tiles) tiles[pos] = make_int2(s, r);  // overlapping query ranges can overflow
+        else atomicOr(&s_err, PA_DEVERR_LENGTHS);
+      }
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    // the last bucket's running cursor ends at the number of tiles
+    num_tiles = (int)min((long long)s_hist[kCostBuckets - 1], (long long)L.max_tiles);
+    hdr->num_prefill_tiles = num_tiles;
+    hdr->num_decode_pairs = num_pairs;
+    hdr->total_decode_keys = (int)min(s_dec_keys, (unsigned long long)0x7fffffff);
+    if (s_err) atomicOr(err, s_err);
+  }
+}
+
+void launch_plan(const int32_t* query_start_loc, const int32_t* seq_lens, int num_seqs,
+                 long long num_q_tokens, int max_blocks_per_seq, int block_size,
+                 int max_query_len, int max_seq_len, int causal, int num_kv_heads,
+                 int target_items, unsigned char* ws, const WorkspaceLayout& L,
+                 cudaStream_t stream) {
+  plan_kernel<<<1, kPlanThreads, 0, stream>>>(query_start_loc, seq_lens, num_seqs, num_q_tokens,
+                                              max_blocks_per_seq, block_size, max_query_len,
+                                              max_seq_len, causal, num_kv_heads, target_items,
+                                              ws, L);
+}
+
+}  // namespace pa

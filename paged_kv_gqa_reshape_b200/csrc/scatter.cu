@@ -1,0 +1,78 @@
+// KV-cache write through slot_mapping (the cache-update step of vllm-spyre
+// PR #853 "Pytorch Native Attention on Spyre", description, step 1).
+//
+// One warp per token: it reads the token's K and V rows (num_kv_heads *
+// head_dim bf16 each, contiguous) with 16-byte loads and stores them to slot
+// slot_mapping[t] of the caches, whose rows are contiguous too
+// ([num_blocks, block_size, Hkv, D] => slot s starts at s * Hkv * D).  Pure
+// bandwidth: every byte is read once and written once.  A negative slot marks
+// a padding token (skipped); a slot beyond the pool is skipped and reported.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace pa {
+
+__global__ void __launch_bounds__(256) write_kv_kernel(const uint4* __restrict__ k,
+                                                       const uint4* __restrict__ v,
+                                                       const int64_t* __restrict__ slot_mapping,
+                                                       long long num_tokens, int row_vecs,
+                                                       uint4* __restrict__ k_cache,
+                                                       uint4* __restrict__ v_cache,
+                                                       long long num_slots, uint32_t* err) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long t = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       t < num_tokens; t += warps) {
+    const long long slot = slot_mapping[t];
+    if (slot < 0) continue;
+    if (slot >= num_slots) {
+      if (lane == 0) raise_error(err, PA_DEVERR_SLOT);
+      continue;
+    }
+    const uint4* ks = k + t * row_vecs;
+    const uint4* vs = v + t * row_vecs;
+    uint4* kd = k_cache + slot * row_vecs;
+    uint4* vd = v_cache + slot * row_vecs;
+    // issue all loads of this lane before its stores (row_vecs <= 32 * 8 here)
+    constexpr int kMaxPerLane = 8;
+    uint4 kr[kMaxPerLane], vr[kMaxPerLane];
+#pragma unroll
+    for (int i = 0; i < kMaxPerLane; ++i) {
+      const int idx = i * 32 + lane;
+      if (idx < row_vecs) {
+        kr[i] = __ldcs(ks + idx);
+        vr[i] = __ldcs(vs + idx);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxPerLane; ++i) {
+      const int idx = i * 32 + lane;
+      if (idx < row_vecs) {
+        kd[idx] = kr[i];
+        vd[idx] = vr[i];
+      }
+    }
+    // rows wider than 32 * 8 vectors (Hkv * D > 2048) continue here
+    for (int idx = kMaxPerLane * 32 + lane; idx < row_vecs; idx += 32) {
+      kd[idx] = __ldcs(ks + idx);
+      vd[idx] = __ldcs(vs + idx);
+    }
+  }
+}
+
+cudaError_t launch_write_kv(const void* k, const void* v, const int64_t* slot_mapping,
+                            int64_t num_tokens, int row_vecs, void* k_cache, void* v_cache,
+                            int64_t num_slots, uint32_t* err, int num_sms, cudaStream_t stream) {
+  if (num_tokens <= 0) return cudaSuccess;
+  const int threads = 256;
+  const long long warps_needed = num_tokens;
+  long long blocks = (warps_needed + (threads / 32) - 1) / (threads / 32);
+  const long long cap = (long long)num_sms * 8;  // 8 resident 256-thread CTAs per SM
+  if (blocks > cap) blocks = cap;
+  write_kv_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
+      static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping, num_tokens,
+      row_vecs, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), num_slots, err);
+  return cudaGetLastError();
+}
+
+}  // namespace pa

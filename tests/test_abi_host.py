@@ -1,0 +1,115 @@
+"""CPU-only checks of the C ABI: the library builds, loads and exports every
+symbol include/pa.h declares, and host-visible argument errors are rejected
+before anything is launched (no GPU needed for any of this)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import paged_kv_gqa_reshape_b200 as pa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    with open(os.path.join(ROOT, "include", "pa.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_exported_set():
+    assert declared_symbols() == sorted(pa.EXPORTED_SYMBOLS)
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = pa.load()
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_status_strings_and_version():
+    assert pa.status_string(0) == "PA_OK"
+    for s in range(1, 6):
+        assert pa.status_string(s).startswith("PA_ERR_")
+    assert "sm_100a" in pa.version()
+
+
+def test_workspace_size_is_a_function_of_the_arguments():
+    a = pa.varlen_workspace_size(64, 64, 32, 8, 128)
+    b = pa.varlen_workspace_size(64, 64, 32, 8, 128)
+    assert a == b and a > 256
+    assert pa.varlen_workspace_size(256, 4344, 64, 8, 128) > a
+    assert pa.varlen_workspace_size(-1, 1, 1, 1, 64) == 0
+
+
+def _varlen(lib, **over):
+    args = dict(q=1 << 12, kc=1 << 12, vc=1 << 12, bt=1 << 12, mb=4, sl=1 << 12, qsl=1 << 12,
+                S=2, T=4, Hq=4, Hkv=2, D=64, BS=16, NB=8, mql=4, msl=64, scale=0.125,
+                causal=1, out=1 << 12, ws=1 << 12, wsb=1 << 30, stream=None)
+    args.update(over)
+    return lib.pa_attention_varlen(*args.values())
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(Hq=6, Hkv=4), 1),           # Hq % Hkv != 0
+    (dict(Hkv=0), 1),
+    (dict(D=96), 2),                  # unsupported head_dim
+    (dict(BS=32), 2),                 # unsupported block size
+    (dict(Hq=34, Hkv=2), 2),          # GQA group > 16
+    (dict(causal=2), 1),
+    (dict(scale=float("nan")), 1),
+    (dict(q=0), 1),                   # null pointer
+    (dict(q=(1 << 12) + 2), 1),       # misaligned
+    (dict(wsb=16), 1),                # workspace too small
+    (dict(NB=0), 1),
+])
+def test_varlen_rejects_before_launch(over, expect):
+    assert _varlen(pa.load(), **over) == expect
+
+
+def test_varlen_empty_batch_is_a_no_op():
+    assert _varlen(pa.load(), S=0) == 0
+    assert _varlen(pa.load(), T=0) == 0
+
+
+def test_write_kv_rejects_before_launch():
+    lib = pa.load()
+    ok = dict(k=1 << 12, v=1 << 12, sm=1 << 12, T=3, Hkv=2, D=64, kc=1 << 12, vc=1 << 12,
+              NB=4, BS=16, ws=None, stream=None)
+    for over in (dict(D=60), dict(Hkv=0), dict(NB=0), dict(k=0), dict(kc=(1 << 12) + 8),
+                 dict(T=-1)):
+        a = dict(ok)
+        a.update(over)
+        assert lib.pa_write_kv(*a.values()) == 1, over
+    a = dict(ok)
+    a["T"] = 0
+    assert lib.pa_write_kv(*a.values()) == 0
+
+
+def test_smallseq_rejects_before_launch():
+    lib = pa.load()
+    ok = dict(q=1 << 12, k=1 << 12, v=1 << 12, cu=1 << 12, B=4, Hq=4, Hkv=4, D=128, mx=16,
+              scale=0.1, out=1 << 12, ws=None, stream=None)
+    for over, expect in ((dict(mx=17), 2), (dict(D=80), 2), (dict(Hq=6), 1), (dict(cu=0), 1),
+                         (dict(out=(1 << 12) + 4), 1)):
+        a = dict(ok)
+        a.update(over)
+        assert lib.pa_attention_smallseq(*a.values()) == expect, over
+    a = dict(ok)
+    a["B"] = 0
+    assert lib.pa_attention_smallseq(*a.values()) == 0
+
+
+def test_python_binding_rejects_cpu_and_wrong_dtypes():
+    q = torch.zeros(4, 4, 64, dtype=torch.bfloat16)
+    kc = torch.zeros(8, 16, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        pa.attention_varlen(q, kc, kc, torch.zeros(2, 2, dtype=torch.int32),
+                            torch.zeros(2, dtype=torch.int32), torch.zeros(3, dtype=torch.int32),
+                            2, 0.1, True, q)
+    with pytest.raises(TypeError):
+        pa.write_kv(q.float(), q, torch.zeros(4, dtype=torch.int64), kc, kc)
