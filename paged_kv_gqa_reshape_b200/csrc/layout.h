@@ -13,7 +13,7 @@ constexpr int kPrefillTileN = 128;      // keys per prefill KV tile (tcgen05 N)
 constexpr int kDecodeWarps = 4;         // warps per decode CTA
 constexpr int kPageKeys = 16;           // block_size this build supports
 constexpr int kDecodeMinChunk = 256;    // smallest split-KV chunk (keys)
-constexpr int kDecodeMaxItems = 4096;   // upper bound on planned (seq, chunk) pairs beyond S
+constexpr int kDecodeMaxItems = 4096;   // upper bound on the plan's (seq, chunk, kv-head) target
 constexpr int kCostBuckets = 4096;      // prefill tiles are sorted by KV-tile count
 
 // Sanitised geometry of one sequence, written by the plan kernel.  The
@@ -64,7 +64,10 @@ inline WorkspaceLayout make_layout(int64_t num_seqs, int64_t num_q_tokens, int64
   L.max_tiles = (num_q_tokens + kPrefillTileM - 1) / kPrefillTileM + num_seqs;
   L.tiles = off;
   off = align_up(off + 8 * (size_t)L.max_tiles, 256);
-  L.max_pairs = kDecodeMaxItems + num_seqs;
+  // The plan picks chunk >= total_decode_keys * Hkv / target_items with
+  // target_items <= kDecodeMaxItems, so sum_s ceil(L_s / chunk) <=
+  // target_items / Hkv + num_seqs.
+  L.max_pairs = (kDecodeMaxItems + num_kv_heads - 1) / num_kv_heads + num_seqs;
   L.pairs = off;
   off = align_up(off + 8 * (size_t)L.max_pairs, 256);
   L.counters = off;
