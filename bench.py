@@ -86,22 +86,41 @@ class ClockSampler:
         self.proc = None
         self.dev = device_index
 
-    def _id(self):
+    def _ids(self):
+        ids = []
         try:
-            u = torch.cuda.get_device_properties(self.dev).uuid
-            s = str(u)
-            return s if s.startswith("GPU-") else "GPU-" + s
+            u = str(torch.cuda.get_device_properties(self.dev).uuid)
+            ids.append(u if u.startswith("GPU-") else "GPU-" + u)
         except Exception:
-            return str(self.dev)
+            pass
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            parts = [x.strip() for x in vis.split(",") if x.strip()]
+            if self.dev < len(parts):
+                ids.append(parts[self.dev])
+        ids.append(str(self.dev))
+        return ids
 
     def start(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", self._id(), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "50"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except Exception:
-            self.proc = None
+        self.proc = None
+        for ident in self._ids():
+            try:
+                probe = subprocess.run(["nvidia-smi", "-i", ident, "--query-gpu=clocks.sm",
+                                        "--format=csv,noheader,nounits"],
+                                       capture_output=True, text=True, timeout=20)
+            except Exception:
+                continue
+            if probe.returncode != 0 or not probe.stdout.strip():
+                continue
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", ident, "--query-gpu=" + self.FIELDS,
+                     "--format=csv,noheader,nounits", "-lms", "50"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                time.sleep(0.3)  # let the first sample land before the timed region
+            except Exception:
+                self.proc = None
+            return
 
     def stop(self):
         if self.proc is None:
@@ -329,6 +348,62 @@ def run_ours(args, rank, world, local_rank):
     return result, case
 
 
+def run_single_workload(args):
+    """--workload NAME (not the headline): time NAME's step on one GPU.
+
+    Used to profile the other workloads' kernels with committed code only;
+    prints one JSON line with that workload's own throughput.
+    """
+    import paged_kv_gqa_reshape_b200 as pa
+
+    pa.load()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    hbm_peak, tc_peak, _, peak_kind = measured_peaks()
+    name = args.workload
+    if name == "smallseq_batch":
+        ss = workloads.smallseq_batch(device=dev)
+        out = torch.empty_like(ss.q)
+
+        def step():
+            pa.attention_smallseq(ss.q, ss.k, ss.v, ss.cu_seqlens_kv, ss.scale, out)
+        work = (ss.k.numel() + ss.v.numel() + ss.q.numel() + out.numel()) * 2 + 4 * (ss.batch + 1)
+        unit, scale_div, peak = "GB/s", 1e9, hbm_peak
+    else:
+        case = workloads.NAMED[name](device=dev, keep_logical=False) if name != "tiny_prefill" \
+            else workloads.tiny_prefill(device=dev)
+        ws = pa.varlen_workspace(case.num_seqs, case.num_q_tokens, case.num_q_heads,
+                                 case.num_kv_heads, case.head_dim, device=dev)
+        out = torch.empty_like(case.q)
+
+        def step():
+            pa.write_kv(case.k_new, case.v_new, case.slot_mapping, case.k_cache, case.v_cache,
+                        workspace=ws)
+            pa.attention_varlen(case.q, case.k_cache, case.v_cache, case.block_tables,
+                                case.seq_lens, case.query_start_loc, case.num_kv_heads,
+                                case.scale, case.causal, out, max_query_len=case.max_query_len,
+                                max_seq_len=case.max_seq_len, workspace=ws)
+        if case.max_query_len > 1:
+            work, unit, scale_div, peak = attention_flops(case), "TFLOP/s", 1e12, tc_peak
+        else:
+            work = scatter_bytes(case) + attention_bytes(case)
+            unit, scale_div, peak = "GB/s", 1e9, hbm_peak
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / args.steps
+    v = work / (ms * 1e-3) / scale_div
+    return {"workload": name, "value": round(v, 2), "unit": unit, "ms_per_step": round(ms, 5),
+            "steps": args.steps, "warmup": args.warmup, "frac": round(v / peak, 4),
+            "peak": peak, "peak_kind": peak_kind}
+
+
 def run_e2e(pa, case, args, dev, ws):
     """The same step through the public API with host-resident inputs/outputs."""
     names = ["q", "k_new", "v_new", "slot_mapping", "block_tables", "seq_lens", "query_start_loc"]
@@ -449,6 +524,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-components", action="store_true")
+    ap.add_argument("--workload", default="decode_batch", choices=sorted(workloads.NAMED),
+                    help="decode_batch is the headline; the others time one workload alone")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per dominant-kernel launch from an ncu capture, if current")
     args = ap.parse_args()
@@ -463,6 +540,10 @@ def main():
         res = run_reference(args, rank, world)
         if res is not None:
             print(json.dumps(res), flush=True)
+        return
+
+    if args.workload != "decode_batch":
+        print(json.dumps(run_single_workload(args)), flush=True)
         return
 
     if world > 1:
