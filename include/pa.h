@@ -158,6 +158,39 @@ pa_status pa_attention_varlen(const void* q, const void* k_cache, const void* v_
                               size_t workspace_bytes, void* stream);
 
 /*
+ * pa_attention_varlen_static — pa_attention_varlen for callers that cannot
+ * allocate device memory.  This is an addition of this library: the pages it
+ * follows have no counterpart.
+ *
+ * Some callers may not call cudaMalloc: a host program that owns all device
+ * memory through its own pool allocator and forbids other allocations, or a
+ * latency-critical serving path where cudaMalloc/cudaFree would synchronise
+ * the device.  This variant takes the same arguments as pa_attention_varlen
+ * minus the workspace, runs the same kernels, and keeps its scratch in a
+ * file-scope device array of PA_STATIC_SCRATCH_BYTES bytes that every GPU
+ * loading the library holds until the process exits.  It allocates nothing.
+ *
+ *  - Sizes whose pa_attention_varlen_workspace_size() exceeds
+ *    PA_STATIC_SCRATCH_BYTES return PA_ERR_UNSUPPORTED before any launch.
+ *  - The first call on a device looks up the array's device address with
+ *    that device current; make it before any stream capture.
+ *  - All calls share the array (it keeps the last call's contents; each call
+ *    rebuilds what it needs).  Calls whose executions overlap on the GPU race
+ *    on it: issue them on one stream, one host thread at a time.
+ *  - Device-side index errors are handled as in pa_attention_varlen but
+ *    cannot be read back (there is no caller workspace for pa_get_error).
+ */
+#define PA_STATIC_SCRATCH_BYTES (32u << 20)
+pa_status pa_attention_varlen_static(const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                     const int32_t* seq_lens, const int32_t* query_start_loc,
+                                     int32_t num_seqs, int64_t num_q_tokens,
+                                     int32_t num_q_heads, int32_t num_kv_heads,
+                                     int32_t head_dim, int32_t block_size, int64_t num_blocks,
+                                     int32_t max_query_len, int32_t max_seq_len, float scale,
+                                     int32_t causal, void* out, void* stream);
+
+/*
  * pa_attention_smallseq — s_q = 1 cross attention over short contiguous KV.
  *
  * Defined by ROCm/TransformerEngine PR #461 "CK varlen cross attention for

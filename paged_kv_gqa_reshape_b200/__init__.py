@@ -25,6 +25,7 @@ import torch
 
 __all__ = [
     "PaError", "library_path", "load", "write_kv", "attention_varlen", "attention_smallseq",
+    "attention_varlen_static", "STATIC_SCRATCH_BYTES",
     "varlen_workspace_size", "varlen_workspace", "error_workspace", "get_error",
     "status_string", "version", "EXPORTED_SYMBOLS",
     "DEVERR_SLOT", "DEVERR_BLOCK", "DEVERR_LENGTHS", "DEVERR_QLEN", "DEVERR_HINT",
@@ -36,10 +37,12 @@ PA_OK = 0
 DEVERR_SLOT, DEVERR_BLOCK, DEVERR_LENGTHS = 0x1, 0x2, 0x4
 DEVERR_QLEN, DEVERR_HINT, DEVERR_TIMEOUT = 0x8, 0x10, 0x20
 ERROR_WORD_BYTES = 256
+STATIC_SCRATCH_BYTES = 32 << 20  # PA_STATIC_SCRATCH_BYTES
 
 EXPORTED_SYMBOLS = (
     "pa_write_kv", "pa_attention_varlen_workspace_size", "pa_attention_varlen",
     "pa_attention_smallseq", "pa_get_error", "pa_status_string", "pa_version",
+    "pa_attention_varlen_static",
 )
 
 _lib = None
@@ -84,6 +87,10 @@ def load(build_if_missing: bool = True):
         lib.pa_attention_varlen.argtypes = [
             p, p, p, p, i32, p, p, i32, i64, i32, i32, i32, i32, i64, i32, i32,
             ctypes.c_float, i32, p, p, ctypes.c_size_t, p]
+        lib.pa_attention_varlen_static.restype = ctypes.c_int
+        lib.pa_attention_varlen_static.argtypes = [
+            p, p, p, p, i32, p, p, i32, i64, i32, i32, i32, i32, i64, i32, i32,
+            ctypes.c_float, i32, p, p]
         lib.pa_attention_smallseq.restype = ctypes.c_int
         lib.pa_attention_smallseq.argtypes = [p, p, p, p, i32, i32, i32, i32, i32,
                                               ctypes.c_float, p, p, p]
@@ -203,6 +210,45 @@ def attention_varlen(q, k_cache, v_cache, block_tables, seq_lens, query_start_lo
         float(scale), int(bool(causal)), out.data_ptr(), workspace.data_ptr(),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _raise(st, "pa_attention_varlen")
+    return out
+
+
+def attention_varlen_static(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc,
+                            num_kv_heads, scale, causal, out, max_query_len=None,
+                            max_seq_len=None, stream=None):
+    """attention_varlen for callers that cannot allocate device memory.
+
+    Takes no workspace: the library keeps the scratch in a fixed device array
+    of STATIC_SCRATCH_BYTES (32 MiB) per GPU.  Meant for hosts that own all
+    device memory through their own allocator, or paths where cudaMalloc would
+    synchronise the device.  Sizes needing more scratch raise (status
+    PA_ERR_UNSUPPORTED); calls that overlap on the GPU race on the shared
+    array; device-side index errors cannot be read back.  The first call on a
+    device looks up the array's address and should come before any stream
+    capture.
+    """
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_cache, "k_cache", torch.bfloat16, 4)
+    _check(v_cache, "v_cache", torch.bfloat16, 4)
+    _check(block_tables, "block_tables", torch.int32, 2)
+    _check(seq_lens, "seq_lens", torch.int32, 1)
+    _check(query_start_loc, "query_start_loc", torch.int32, 1)
+    _check(out, "out", torch.bfloat16, 3)
+    t, hq, d = q.shape
+    nb, bs, hkv, d_c = k_cache.shape
+    if hkv != num_kv_heads or d_c != d or v_cache.shape != k_cache.shape or out.shape != q.shape:
+        raise ValueError("inconsistent shapes")
+    s = seq_lens.shape[0]
+    if query_start_loc.shape[0] != s + 1 or block_tables.shape[0] != s:
+        raise ValueError("seq_lens, query_start_loc and block_tables disagree on num_seqs")
+    mb = block_tables.shape[1]
+    mql = t if max_query_len is None else int(max_query_len)
+    msl = mb * bs if max_seq_len is None else int(max_seq_len)
+    st = load().pa_attention_varlen_static(
+        q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(), mb,
+        seq_lens.data_ptr(), query_start_loc.data_ptr(), s, t, hq, hkv, d, bs, nb, mql, msl,
+        float(scale), int(bool(causal)), out.data_ptr(), _stream(stream))
+    _raise(st, "pa_attention_varlen_static")
     return out
 
 

@@ -1,0 +1,84 @@
+// pa_attention_varlen_static: paged varlen attention for callers that cannot
+// allocate device memory.
+//
+// Some callers may not call cudaMalloc at all: a host program that owns every
+// byte of device memory through its own pool allocator and forbids any other
+// allocation, or a latency-critical serving path where cudaMalloc/cudaFree
+// would synchronise the device.  Such callers still pass their inputs and
+// outputs, but cannot hand over a workspace.  This entry point runs exactly
+// the same kernels as pa_attention_varlen, with the workspace placed in a
+// file-scope device array of PA_STATIC_SCRATCH_BYTES bytes instead.
+//
+// Properties the caller must know:
+//  - Every GPU that loads this library holds the array until the process
+//    exits, whether or not this entry point is ever called.
+//  - The first call on a device looks up the array's device address
+//    (cudaGetSymbolAddress) with that device current, and caches it; make that
+//    first call before any stream capture.
+//  - All calls share the one array, which keeps the last call's contents.  The
+//    plan kernel rebuilds every list and zeroes every split-KV counter at the
+//    start of each call, and this entry point clears the error word, so no
+//    state leaks from one call to the next; but calls whose executions
+//    overlap on the GPU (different streams, or different host threads) race
+//    on the array and must not be issued.
+//  - Device-side index errors are handled as in pa_attention_varlen (rows
+//    skipped, reads zero-filled) but cannot be read back: the error word lives
+//    in the shared array, not in a caller buffer.
+//  - Sizes whose workspace would exceed PA_STATIC_SCRATCH_BYTES are rejected
+//    with PA_ERR_UNSUPPORTED before anything is launched.
+// Nothing here calls cudaMalloc, cudaFree or any allocating library routine.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "../../include/pa.h"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// The scratch area: one copy per device that loads the library.
+static __device__ __align__(256) unsigned char g_pa_static_scratch[PA_STATIC_SCRATCH_BYTES];
+
+void* g_scratch_addr[kMaxDevices];  // device address of the array, per device
+std::mutex g_scratch_mu;
+
+// Device address of the current device's copy of the array (looked up once
+// per device; the array's name in host code is only a host-side stand-in).
+pa_status scratch_address(void** addr) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_pa_static_scratch) != cudaSuccess || p == nullptr)
+      return PA_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *addr = g_scratch_addr[dev];
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" pa_status pa_attention_varlen_static(
+    const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+    int32_t max_blocks_per_seq, const int32_t* seq_lens, const int32_t* query_start_loc,
+    int32_t num_seqs, int64_t num_q_tokens, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t block_size, int64_t num_blocks, int32_t max_query_len,
+    int32_t max_seq_len, float scale, int32_t causal, void* out, void* stream) {
+  const size_t need = pa_attention_varlen_workspace_size(num_seqs, num_q_tokens, num_q_heads,
+                                                         num_kv_heads, head_dim);
+  if (need > (size_t)PA_STATIC_SCRATCH_BYTES) return PA_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  pa_status st = scratch_address(&scratch);
+  if (st != PA_OK) return st;
+  if (need > 0 && num_seqs > 0 && num_q_tokens > 0 &&
+      cudaMemsetAsync(scratch, 0, sizeof(uint32_t), static_cast<cudaStream_t>(stream)) !=
+          cudaSuccess)
+    return PA_ERR_CUDA;
+  return pa_attention_varlen(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                             query_start_loc, num_seqs, num_q_tokens, num_q_heads, num_kv_heads,
+                             head_dim, block_size, num_blocks, max_query_len, max_seq_len, scale,
+                             causal, out, scratch, (size_t)PA_STATIC_SCRATCH_BYTES, stream);
+}
