@@ -185,12 +185,16 @@ pa_status pa_attention_varlen(const void* q, const void* k_cache, const void* v_
       return PA_ERR_CUDA;
   }
 
-  const int target_items = nsm * 2 * 4 < pa::kDecodeMaxItems ? nsm * 2 * 4 : pa::kDecodeMaxItems;
-  pa::launch_plan(query_start_loc, seq_lens, num_seqs, num_q_tokens, max_blocks_per_seq,
-                  block_size, max_query_len, max_seq_len, causal, num_kv_heads, target_items, ws,
-                  L, st);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return PA_ERR_CUDA;
+  // decode CTAs compute their page ranges themselves for up to
+  // kSelfPlanMaxSeqs sequences; beyond that the plan kernel writes the prefix
+  const bool self_plan = num_seqs <= pa::kSelfPlanMaxSeqs;
+  cudaError_t e = cudaSuccess;
+  if (run_prefill || !self_plan) {
+    pa::launch_plan(query_start_loc, seq_lens, num_seqs, num_q_tokens, max_blocks_per_seq,
+                    block_size, max_query_len, max_seq_len, causal, num_kv_heads, ws, L, st);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return PA_ERR_CUDA;
+  }
 
   if (run_prefill) {
     pa::PrefillParams pp{};
@@ -215,7 +219,14 @@ pa_status pa_attention_varlen(const void* q, const void* k_cache, const void* v_
   dp.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
   dp.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
   dp.block_tables = block_tables;
+  dp.query_start_loc = query_start_loc;
+  dp.seq_lens = seq_lens;
+  dp.num_seqs = num_seqs;
+  dp.num_q_tokens = num_q_tokens;
+  dp.max_query_len = max_query_len;
   dp.max_blocks_per_seq = max_blocks_per_seq;
+  dp.max_seq_len = max_seq_len;
+  dp.self_plan = self_plan ? 1 : 0;
   dp.num_q_heads = num_q_heads;
   dp.num_kv_heads = num_kv_heads;
   dp.group = group;
@@ -224,7 +235,7 @@ pa_status pa_attention_varlen(const void* q, const void* k_cache, const void* v_
   dp.out = static_cast<__nv_bfloat16*>(out);
   dp.ws = ws;
   dp.L = L;
-  e = pa::launch_decode(dp, head_dim, nsm * 2, st);
+  e = pa::launch_decode(dp, head_dim, nsm, st);
   if (log_enabled())
     fprintf(stderr, "[pa] varlen S=%d T=%lld Hq=%d Hkv=%d D=%d prefill=%d sms=%d\n", num_seqs,
             (long long)num_q_tokens, num_q_heads, num_kv_heads, head_dim, (int)run_prefill, nsm);

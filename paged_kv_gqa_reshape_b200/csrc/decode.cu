@@ -1,28 +1,42 @@
 // Split-KV decode attention over the paged cache (single-query sequences).
 //
-// Work item = (sequence, key chunk, KV head).  One CTA of 4 warps owns an
-// item; its warps take the chunk's 16-key pages round-robin.  The query rows
-// of the KV head's whole GQA group (g = Hq/Hkv <= 16 heads of the one decode
-// token) form the M = 16 rows of an m16n8k16 bf16 tile, so each K/V page is
-// read from HBM once for all g heads (the repeat_interleave expansion of
+// Work split: the pages (16 keys) of all single-query sequences are laid end
+// to end and cut into gridDim.x / groups equal contiguous ranges, one per
+// resident CTA and group of HPC KV heads, so every CTA streams the same
+// number of pages (+-1) whatever the length mix; a sequence cut by a range
+// boundary is finished by a split-KV merge.  (The per-page ranges replace
+// fixed-size work items, whose last item set the finish time.)  Warp w of a
+// CTA computes KV head (group * HPC + w); its query heads' GQA group is
+// served by one pass over the pages, so the repeat_interleave expansion of
 // vllm-spyre PR #853 "Pytorch Native Attention on Spyre" is never
-// materialised).  Decode is HBM-bound: the contraction is ~g FLOP per byte,
-// so the legacy mma.sync path keeps up with the 16-key pages and tcgen05's
-// minimum M of 64 would buy nothing.
+// materialised.
 //
-// Memory path: every warp streams its pages through a private NSTAGE-deep
-// ring of cp.async 16-byte copies (XOR-swizzled rows, conflict-free ldmatrix),
-// and its producer runs ahead across item boundaries, so the ring never
-// drains between items.  Keys past the sequence end are zero-filled instead
-// of read; a block id outside the pool is reported and read as zeros.
+// Memory path: each 16-slot page is copied by the whole CTA as the
+// contiguous rows it is in HBM (slot r holds [Hkv, D]), through an
+// NSTAGE-deep shared-memory ring of cp.async 16-byte copies (rows
+// XOR-swizzled for conflict-free ldmatrix).  The copies run NSTAGE pages
+// ahead across sequence boundaries; one barrier per page publishes the page
+// that landed and frees the one before it.  Keys past the sequence end are
+// zero-filled instead of read; a block id outside the pool is reported and
+// read as zeros.
 //
-// Per page: S = Q.K^T (fp32), masked, online softmax in the log2 domain
-// (scale folded with log2 e), P rounded to bf16, O += P.V.  At item end the
-// four warps' (max, sum, O) states are merged through shared memory.  A
-// sequence with one chunk writes bf16 output directly; otherwise the chunk
-// writes a normalised fp32 partial plus its log2-sum-exp, and the last CTA to
-// finish a (sequence, KV head) merges all chunks (arrival counter + fences),
-// so no separate combine launch is needed.
+// Per page each warp computes S^T = K . Q^T with mma.sync m16n8k16: the
+// page's 16 keys are the M rows and the group's query heads the N columns
+// (8 per n-tile), so a GQA group of 8 fills the tile exactly.  The online
+// softmax runs per head column in the log2 domain (scale folded with log2 e);
+// P^T is rounded to bf16 and turned into the B operand of O^T += V^T . P^T
+// with movmatrix.  Decode moves ~g FLOP per byte, so it is HBM-bound: the
+// legacy mma path keeps up and tcgen05's M >= 64 would buy nothing.
+//
+// Planning: with up to kSelfPlanMaxSeqs sequences every CTA computes the
+// page prefix itself from query_start_loc / seq_lens (one pass + a block scan
+// into shared memory), so a pure decode batch needs no plan launch; beyond
+// that it reads the prefix the plan kernel wrote.
+//
+// Output: a sequence inside one range writes bf16 directly.  Otherwise each
+// range's segment writes its normalised fp32 partial and log2-sum-exp per head
+// into slot (range + sequence), and the last warp to finish a (sequence, KV
+// head) merges the segments (arrival counter + fences, reset after use).
 #include <math.h>
 
 #include "common.cuh"
@@ -31,391 +45,467 @@
 
 namespace pa {
 
-
-
-template <int D, int NSTAGE>
+template <int D, int HPC, int NSTAGE>
 struct DecodeShape {
-  static constexpr int kChunks = D / 8;               // 16-byte chunks per row
-  static constexpr int kPageElems = kPageKeys * D;    // one page of one KV head
-  static constexpr int kWarpStageBytes = 2 * kPageElems * 2;  // K + V
-  static constexpr int kRingBytes = kDecodeWarps * NSTAGE * kWarpStageBytes;
-  static __host__ __device__ constexpr int combine_bytes(int g) {
-    return kDecodeWarps * g * (2 + D) * 4;
-  }
-  static __host__ __device__ constexpr int smem_bytes(int g) {
-    return kRingBytes + combine_bytes(g);
+  static constexpr int kChunks = D / 8;                     // 16-byte chunks per row
+  static constexpr int kHeadPage = kPageKeys * D;           // one head's page (elements)
+  static constexpr int kTensorStage = HPC * kHeadPage;      // K (or V) of one stage
+  static constexpr int kStageBytes = 2 * kTensorStage * 2;  // K + V
+  static constexpr int kRingBytes = NSTAGE * kStageBytes;
+  static constexpr int kPlanBytes = (2 * kSelfPlanMaxSeqs + 1) * 4;
+  static constexpr int smem_bytes(bool self_plan) {
+    return kRingBytes + (self_plan ? kPlanBytes : 0);
   }
 };
 
 namespace {
 
-// The item a producer or consumer is working on.
-struct Item {
-  int seq;
-  int kvh;
-  int chunk;
-  int first_key;  // first key of the chunk
-  int n_keys;     // keys in the chunk
-  int n_pages;
-  int kv_len;
-};
-
-__device__ __forceinline__ Item load_item(int item, const int2* pairs, const SeqInfo* info,
-                                          int num_kv_heads) {
-  Item it;
-  int2 pr = pairs[item / num_kv_heads];
-  it.seq = pr.x;
-  it.chunk = pr.y;
-  it.kvh = item % num_kv_heads;
-  SeqInfo si = info[pr.x];
-  it.kv_len = si.kv_len;
-  it.first_key = pr.y * si.chunk_len;
-  it.n_keys = max(0, min(si.chunk_len, si.kv_len - it.first_key));
-  it.n_pages = (it.n_keys + kPageKeys - 1) / kPageKeys;
-  return it;
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
 }
 
 }  // namespace
 
-template <int D, int NSTAGE>
-__global__ void __launch_bounds__(kDecodeWarps * 32, 2) decode_kernel(DecodeParams p) {
-  using Shape = DecodeShape<D, NSTAGE>;
+template <int D, int HPC, int NSTAGE, int NGT>
+__global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams p) {
+  using Shape = DecodeShape<D, HPC, NSTAGE>;
   constexpr int CH = Shape::kChunks;
-  constexpr int KSTEPS = D / 16;
-  constexpr int NT = D / 8;  // output n-tiles of 8 columns
+  constexpr int KSTEPS = D / 16;  // k-steps of S^T = K . Q^T and m-tiles of O^T
+  constexpr int NT = HPC * 32;    // threads per CTA
+  constexpr unsigned FULL = 0xffffffffu;
 
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
+  const int tid = threadIdx.x;
   const int g = p.group;
   const int Hkv = p.num_kv_heads;
+  const int groups = Hkv / HPC;
+  const int S = p.num_seqs;
+  const int hg = blockIdx.x % groups;           // KV-head group of this CTA
+  const long long c = blockIdx.x / groups;      // page range of this CTA
+  const long long G = gridDim.x / groups;       // page ranges per group
+  const int kvh = hg * HPC + warp;              // this warp's KV head
+  const int head0 = kvh * g;                    // its first query head
 
   unsigned char* ws = p.ws;
   uint32_t* err = reinterpret_cast<uint32_t*>(ws + p.L.err);
-  const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(ws + p.L.header);
   const SeqInfo* info = reinterpret_cast<const SeqInfo*>(ws + p.L.seq_info);
-  const int2* pairs = reinterpret_cast<const int2*>(ws + p.L.pairs);
+  const int32_t* g_pfx = reinterpret_cast<const int32_t*>(ws + p.L.page_pfx);
   int32_t* counters = reinterpret_cast<int32_t*>(ws + p.L.counters);
   float* lse_buf = reinterpret_cast<float*>(ws + p.L.lse);
   float* part_buf = reinterpret_cast<float*>(ws + p.L.partial);
 
-  const int num_items = hdr->num_decode_pairs * Hkv;
+  __nv_bfloat16* ring = reinterpret_cast<__nv_bfloat16*>(smem);
+  int* s_pg = reinterpret_cast<int*>(smem + Shape::kRingBytes);  // [S + 1] page prefix
+  int* s_kv = s_pg + kSelfPlanMaxSeqs + 1;                       // [S] decode kv_len or -1
+  __shared__ uint32_t s_err;
+  __shared__ int s_scan[HPC];
+  __shared__ int s_carry;
 
-  __nv_bfloat16* ring =
-      reinterpret_cast<__nv_bfloat16*>(smem) + (size_t)warp * NSTAGE * 2 * Shape::kPageElems;
-  float* comb_m = reinterpret_cast<float*>(smem + Shape::kRingBytes);
-  float* comb_l = comb_m + kDecodeWarps * g;
-  float* comb_o = comb_l + kDecodeWarps * g;
-  __shared__ int s_last;
-
-  const size_t row_stride = (size_t)Hkv * D;  // elements between consecutive slots
-
-  // ---------------- producer: this warp's page stream ----------------------
-  int p_item = blockIdx.x;
-  int p_page = warp;
-  Item pit;
-  if (p_item < num_items) pit = load_item(p_item, pairs, info, Hkv);
-  auto p_skip_empty = [&]() {
-    while (p_item < num_items && p_page >= pit.n_pages) {
-      p_item += gridDim.x;
-      p_page = warp;
-      if (p_item < num_items) pit = load_item(p_item, pairs, info, Hkv);
-    }
-  };
-  p_skip_empty();
-
-  auto issue = [&](int slot) {
-    if (p_item < num_items) {
-      const int key0 = pit.first_key + p_page * kPageKeys;
-      const int32_t* table = p.block_tables + (size_t)pit.seq * p.max_blocks_per_seq;
-      const long long block = table[key0 / kPageKeys];
-      const bool block_ok = block >= 0 && block < p.num_blocks;
-      if (!block_ok && lane == 0) raise_error(err, PA_DEVERR_BLOCK);
-      const long long safe_block = block_ok ? block : 0;
-      __nv_bfloat16* kdst = ring + slot * 2 * Shape::kPageElems;
-      __nv_bfloat16* vdst = kdst + Shape::kPageElems;
-      const size_t base = ((size_t)safe_block * kPageKeys * Hkv + pit.kvh) * D;
-#pragma unroll
-      for (int i = 0; i < kPageKeys * CH / 32; ++i) {
-        const int idx = i * 32 + lane;
-        const int r = idx / CH, c = idx % CH;
-        const bool ok = block_ok && (key0 + r < pit.kv_len);
-        const size_t src = base + (size_t)r * row_stride + c * 8;
-        const int dst = r * D + ((c ^ (r & 7)) * 8);
-        cp_async_16(smem_u32(kdst + dst), p.k_cache + (ok ? src : 0), ok);
-        cp_async_16(smem_u32(vdst + dst), p.v_cache + (ok ? src : 0), ok);
-      }
-      p_page += kDecodeWarps;
-      p_skip_empty();
-    }
-    cp_async_commit();
-  };
-
-#pragma unroll
-  for (int s = 0; s < NSTAGE; ++s) issue(s);
-  int c_slot = 0;
-
-  const int gr = lane >> 2;  // fragment row (head within the group)
-  const int tq = lane & 3;   // fragment column pair
-
-  for (int c_item = blockIdx.x; c_item < num_items; c_item += gridDim.x) {
-    const Item it = load_item(c_item, pairs, info, Hkv);
-    const SeqInfo si = info[it.seq];
-    const int tok = si.q_start;
-
-    // Q fragments (A operand) for the group's rows; rows >= g are zero.
-    uint32_t qa[KSTEPS][4];
-    {
-      const uint32_t* q32 = reinterpret_cast<const uint32_t*>(p.q);
-      const size_t row0 = ((size_t)tok * p.num_q_heads + (size_t)it.kvh * g + gr) * D;
-      const size_t row1 = row0 + (size_t)8 * D;
-#pragma unroll
-      for (int ks = 0; ks < KSTEPS; ++ks) {
-        const int col = ks * 16 + tq * 2;
-        qa[ks][0] = gr < g ? q32[(row0 + col) / 2] : 0u;
-        qa[ks][1] = gr + 8 < g ? q32[(row1 + col) / 2] : 0u;
-        qa[ks][2] = gr < g ? q32[(row0 + col + 8) / 2] : 0u;
-        qa[ks][3] = gr + 8 < g ? q32[(row1 + col + 8) / 2] : 0u;
-      }
-    }
-
-    float o[NT][4];
-#pragma unroll
-    for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-
-    for (int pg = warp; pg < it.n_pages; pg += kDecodeWarps) {
-      cp_async_wait<NSTAGE - 1>();
-      __syncwarp();
-      const __nv_bfloat16* ks_ = ring + c_slot * 2 * Shape::kPageElems;
-      const __nv_bfloat16* vs_ = ks_ + Shape::kPageElems;
-      const uint32_t kbase = smem_u32(ks_), vbase = smem_u32(vs_);
-
-      // ---- S = Q . K^T for 16 keys (two n-tiles of 8) ----
-      float s[2][4];
-#pragma unroll
-      for (int n = 0; n < 2; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
-      {
-        const int mi = lane >> 3, rr = lane & 7;
-        const int key = (mi >> 1) * 8 + rr;
-#pragma unroll
-        for (int ks = 0; ks < KSTEPS; ++ks) {
-          const int chunk = ks * 2 + (mi & 1);
-          const uint32_t addr = kbase + (key * D + ((chunk ^ (key & 7)) * 8)) * 2;
-          uint32_t b0, b1, b2, b3;
-          ldmatrix_x4(addr, b0, b1, b2, b3);
-          mma_bf16_16816(s[0], qa[ks], b0, b1);
-          mma_bf16_16816(s[1], qa[ks], b2, b3);
-        }
-      }
-      // ---- mask + online softmax (log2 domain) ----
-      const int key0 = it.first_key + pg * kPageKeys;
-      float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-      for (int n = 0; n < 2; ++n) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int key = key0 + n * 8 + tq * 2 + (e & 1);
-          float v = s[n][e] * p.scale_log2;
-          if (key >= it.kv_len) v = -INFINITY;
-          s[n][e] = v;
-        }
-        mx0 = fmaxf(mx0, fmaxf(s[n][0], s[n][1]));
-        mx1 = fmaxf(mx1, fmaxf(s[n][2], s[n][3]));
-      }
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-      const float base0 = mn0 == -INFINITY ? 0.f : mn0;
-      const float base1 = mn1 == -INFINITY ? 0.f : mn1;
-      const float a0 = fast_exp2(m0 - base0), a1 = fast_exp2(m1 - base1);
-      m0 = mn0;
-      m1 = mn1;
-      float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-      for (int n = 0; n < 2; ++n) {
-        s[n][0] = fast_exp2(s[n][0] - base0);
-        s[n][1] = fast_exp2(s[n][1] - base0);
-        s[n][2] = fast_exp2(s[n][2] - base1);
-        s[n][3] = fast_exp2(s[n][3] - base1);
-        rs0 += s[n][0] + s[n][1];
-        rs1 += s[n][2] + s[n][3];
-      }
-      l0 = l0 * a0 + rs0;
-      l1 = l1 * a1 + rs1;
-#pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        o[n][0] *= a0;
-        o[n][1] *= a0;
-        o[n][2] *= a1;
-        o[n][3] *= a1;
-      }
-      uint32_t pa[4];
-      pa[0] = pack_bf16x2(s[0][0], s[0][1]);
-      pa[1] = pack_bf16x2(s[0][2], s[0][3]);
-      pa[2] = pack_bf16x2(s[1][0], s[1][1]);
-      pa[3] = pack_bf16x2(s[1][2], s[1][3]);
-      // ---- O += P . V ----
-      {
-        const int mi = lane >> 3, rr = lane & 7;
-        const int key = (mi & 1) * 8 + rr;
-#pragma unroll
-        for (int dp = 0; dp < D / 16; ++dp) {
-          const int chunk = dp * 2 + (mi >> 1);
-          const uint32_t addr = vbase + (key * D + ((chunk ^ (key & 7)) * 8)) * 2;
-          uint32_t b0, b1, b2, b3;
-          ldmatrix_x4_trans(addr, b0, b1, b2, b3);
-          mma_bf16_16816(o[2 * dp], pa, b0, b1);
-          mma_bf16_16816(o[2 * dp + 1], pa, b2, b3);
-        }
-      }
-      __syncwarp();
-      issue(c_slot);  // refill the slot just consumed (may belong to a later item)
-      c_slot = (c_slot + 1 == NSTAGE) ? 0 : c_slot + 1;
-    }
-
-    // ---- merge the four warps' states ----
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    if (tq == 0) {
-      if (gr < g) {
-        comb_m[warp * g + gr] = m0;
-        comb_l[warp * g + gr] = l0;
-      }
-      if (gr + 8 < g) {
-        comb_m[warp * g + gr + 8] = m1;
-        comb_l[warp * g + gr + 8] = l1;
-      }
-    }
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      const int d = n * 8 + tq * 2;
-      if (gr < g) {
-        comb_o[(warp * g + gr) * D + d] = o[n][0];
-        comb_o[(warp * g + gr) * D + d + 1] = o[n][1];
-      }
-      if (gr + 8 < g) {
-        comb_o[(warp * g + gr + 8) * D + d] = o[n][2];
-        comb_o[(warp * g + gr + 8) * D + d + 1] = o[n][3];
-      }
+  // ------------------------------- plan ------------------------------------
+  if (p.self_plan) {
+    if (tid == 0) {
+      s_err = 0;
+      s_carry = 0;
     }
     __syncthreads();
+    const long long reach = (long long)p.max_blocks_per_seq * kPageKeys;
+    uint32_t e = 0;
+    for (int s = tid; s < S; s += NT) {
+      const long long qs = p.query_start_loc[s], qe = p.query_start_loc[s + 1];
+      long long kv = p.seq_lens[s];
+      const bool bad_q = qs < 0 || qe < qs || qe > p.num_q_tokens;
+      if (bad_q) e |= PA_DEVERR_LENGTHS;
+      if (kv < 0) {
+        e |= PA_DEVERR_LENGTHS;
+        kv = 0;
+      }
+      if (kv > reach) {
+        e |= PA_DEVERR_LENGTHS;
+        kv = reach;
+      }
+      if (!bad_q && (qe - qs > p.max_query_len || kv > p.max_seq_len)) e |= PA_DEVERR_HINT;
+      const bool dec = !bad_q && qe - qs == 1;
+      if (dec && kv == 0) e |= PA_DEVERR_QLEN;
+      s_kv[s] = dec ? (int)kv : -1;
+    }
+    if (e) atomicOr(&s_err, e);
+    __syncthreads();
+    for (int base = 0; base < S; base += NT) {
+      const int s = base + tid;
+      const int n = (s < S && s_kv[s] > 0) ? (s_kv[s] + kPageKeys - 1) / kPageKeys : 0;
+      int x = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(FULL, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane == 31) s_scan[warp] = x;
+      __syncthreads();
+      int before = s_carry;
+      for (int w = 0; w < warp; ++w) before += s_scan[w];
+      if (s < S) s_pg[s] = before + x - n;
+      __syncthreads();
+      if (tid == 0) {
+        int tot = 0;
+        for (int w = 0; w < HPC; ++w) tot += s_scan[w];
+        s_carry += tot;
+      }
+      __syncthreads();
+    }
+    if (tid == 0) s_pg[S] = s_carry;
+    __syncthreads();
+    if (blockIdx.x == 0 && tid == 0 && s_err) atomicOr(err, s_err);
+  }
+  auto pfx = [&](int s) -> long long { return p.self_plan ? s_pg[s] : __ldg(g_pfx + s); };
+  auto seq_kv = [&](int s) -> int { return p.self_plan ? s_kv[s] : info[s].kv_len; };
+  auto seq_q = [&](int s) -> int { return p.self_plan ? p.query_start_loc[s] : info[s].q_start; };
+  auto is_decode = [&](int s) -> bool { return p.self_plan ? s_kv[s] >= 0 : info[s].q_len == 1; };
 
-    const int n_chunks = si.n_chunks;
-    const int pair = si.pair_base + it.chunk;
-    for (int e = threadIdx.x; e < g * (D / 8); e += blockDim.x) {
-      const int r = e / (D / 8);
-      const int d0 = (e % (D / 8)) * 8;
-      float M = -INFINITY;
+  const long long P = pfx(S);
+
+  // single-query sequences with no key: zero output rows (spread over the ranges)
+  for (long long s = c; s < S; s += G) {
+    if (is_decode((int)s) && seq_kv((int)s) == 0) {
+      __nv_bfloat16* o0 = p.out + ((size_t)seq_q((int)s) * p.num_q_heads + head0) * D;
+      for (int i = lane; i < g * D; i += 32) o0[i] = __float2bfloat16_rn(0.f);
+    }
+  }
+  if (P == 0) return;
+
+  // min(G, P) ranges, so that every range holds at least one page and every
+  // range counted by a sequence's merge really produces a partial
+  const long long R = G < P ? G : P;
+  if (c >= R) return;
+  const long long b0 = c * P / R, b1 = (c + 1) * P / R;  // this CTA's pages [b0, b1)
+  // range holding page x: the largest c' with c' * P / R <= x
+  auto range_of = [&](long long x) -> long long { return ((x + 1) * R - 1) / P; };
+  // the sequence holding page x: the last s with pfx(s) <= x
+  auto seq_of = [&](long long x) -> int {
+    int lo = 0, hi = S - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pfx(mid) <= x)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    return lo;
+  };
+  if (b0 >= b1) return;
+
+  // ---------------- producer: pages [x_p, b1) in order ----------------------
+  const size_t row_stride = (size_t)Hkv * D;
+  long long x_p = b0;
+  int seq_p = seq_of(b0);
+  long long p_first = pfx(seq_p), p_end = pfx(seq_p + 1);
+  int p_kv = seq_kv(seq_p);
+  long long x = b0;  // consumer position
+  auto issue_page = [&]() {
+    const int stage = (int)((x_p - b0) % NSTAGE);
+    const int key0 = (int)(x_p - p_first) * kPageKeys;
+    const long long block =
+        p.block_tables[(size_t)seq_p * p.max_blocks_per_seq + (x_p - p_first)];
+    const bool block_ok = block >= 0 && block < p.num_blocks;
+    if (!block_ok && tid == 0) raise_error(err, PA_DEVERR_BLOCK);
+    const size_t base = ((size_t)(block_ok ? block : 0) * kPageKeys * Hkv + (size_t)hg * HPC) * D;
+    __nv_bfloat16* kdst = ring + (size_t)stage * 2 * Shape::kTensorStage;
+    __nv_bfloat16* vdst = kdst + Shape::kTensorStage;
 #pragma unroll
-      for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, comb_m[w * g + r]);
-      float f[kDecodeWarps];
-      float Lsum = 0.f;
+    for (int i = 0; i < CH / 2; ++i) {
+      const int ci = i * NT + tid;  // chunk index within the page's K (or V) rows
+      const int r = ci / (HPC * CH);
+      const int rem = ci - r * (HPC * CH);
+      const int h = rem / CH, cc = rem - h * CH;
+      const bool ok = block_ok && (key0 + r < p_kv);
+      const size_t src = base + (size_t)r * row_stride + h * D + cc * 8;
+      const int dst = (h * kPageKeys + r) * D + ((cc ^ (r & 7)) * 8);
+      cp_async_16(smem_u32(kdst + dst), p.k_cache + (ok ? src : 0), ok);
+      cp_async_16(smem_u32(vdst + dst), p.v_cache + (ok ? src : 0), ok);
+    }
+    cp_async_commit();
+    ++x_p;
+    if (x_p < b1 && x_p >= p_end) {  // next sequence with pages
+      do {
+        ++seq_p;
+      } while (pfx(seq_p + 1) <= x_p);
+      p_first = pfx(seq_p);
+      p_end = pfx(seq_p + 1);
+      p_kv = seq_kv(seq_p);
+    }
+  };
+  auto fill = [&]() {
+    while (x_p - x < NSTAGE && x_p < b1) issue_page();
+  };
+  fill();
+
+  const int gq = lane >> 2;  // fragment group: key row of S^T / d row of O^T / head of B
+  const int tq = lane & 3;   // fragment column pair: heads 2tq, 2tq+1
+  const uint32_t* q32 = reinterpret_cast<const uint32_t*>(p.q);
+
+  int seq = seq_of(b0);
+  while (x < b1) {
+    const long long seg_first = pfx(seq), seg_last = pfx(seq + 1);
+    const long long seg_end = seg_last < b1 ? seg_last : b1;
+    const int seg_kv = seq_kv(seq);
+    const int seg_q = seq_q(seq);
+    const long long c_first = range_of(seg_first), c_last = range_of(seg_last - 1);
+    const int n_chunks = (int)(c_last - c_first + 1);
+    const int pair_base = (int)c_first + seq;
+
+    // Q^T as the B operand (k = d, n = head): heads nt*8 + gq of the group
+    uint32_t qb[NGT][KSTEPS][2];
 #pragma unroll
-      for (int w = 0; w < kDecodeWarps; ++w) {
-        const float mw = comb_m[w * g + r];
-        f[w] = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
-        Lsum += comb_l[w * g + r] * f[w];
-      }
-      const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-      float acc[8];
+    for (int nt = 0; nt < NGT; ++nt) {
+      const int hl = nt * 8 + gq;
+      const bool hv = hl < g;
+      const size_t row = ((size_t)seg_q * p.num_q_heads + head0 + (hv ? hl : 0)) * D;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float a = 0.f;
-#pragma unroll
-        for (int w = 0; w < kDecodeWarps; ++w) a += comb_o[(w * g + r) * D + d0 + j] * f[w];
-        acc[j] = a * inv;
-      }
-      const int head = it.kvh * g + r;
-      if (n_chunks <= 1) {
-        uint4 v;
-        v.x = pack_bf16x2(acc[0], acc[1]);
-        v.y = pack_bf16x2(acc[2], acc[3]);
-        v.z = pack_bf16x2(acc[4], acc[5]);
-        v.w = pack_bf16x2(acc[6], acc[7]);
-        *reinterpret_cast<uint4*>(p.out + ((size_t)tok * p.num_q_heads + head) * D + d0) = v;
-      } else {
-        float* dst = part_buf + ((size_t)pair * p.num_q_heads + head) * D + d0;
-        *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-        if (d0 == 0)
-          lse_buf[(size_t)pair * p.num_q_heads + head] =
-              Lsum > 0.f ? M + log2f(Lsum) : -INFINITY;
+      for (int ks = 0; ks < KSTEPS; ++ks) {
+        qb[nt][ks][0] = hv ? q32[(row + ks * 16 + 2 * tq) / 2] : 0u;
+        qb[nt][ks][1] = hv ? q32[(row + ks * 16 + 2 * tq + 8) / 2] : 0u;
       }
     }
+    float o[NGT][KSTEPS][4];
+    float m[NGT][2], l[NGT][2];
+#pragma unroll
+    for (int nt = 0; nt < NGT; ++nt) {
+      m[nt][0] = m[nt][1] = -INFINITY;
+      l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < KSTEPS; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
+    }
 
-    if (n_chunks > 1) {
-      // split-KV merge by the last CTA to finish this (sequence, KV head)
-      __threadfence();
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        const int old = atomicAdd(&counters[it.seq * Hkv + it.kvh], 1);
-        s_last = (old == n_chunks - 1);
+    for (; x < seg_end; ++x) {
+      cp_async_wait_dyn((int)(x_p - x - 1));  // my copies of page x have landed
+      __syncthreads();  // everyone's have, and page x-1's stage is free
+      fill();
+      const __nv_bfloat16* kst =
+          ring + (size_t)((x - b0) % NSTAGE) * 2 * Shape::kTensorStage + warp * Shape::kHeadPage;
+      const uint32_t kbase = smem_u32(kst), vbase = smem_u32(kst + Shape::kTensorStage);
+      const int mi = lane >> 3, rr = lane & 7;
+
+      // ---- S^T = K . Q^T : 16 keys x 8 heads per n-tile ----
+      float sc[NGT][4];
+#pragma unroll
+      for (int nt = 0; nt < NGT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+      {
+        const int key = (mi & 1) * 8 + rr;
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+          const int chunk = ks * 2 + (mi >> 1);
+          uint32_t a[4];
+          ldmatrix_x4(kbase + (key * D + ((chunk ^ (key & 7)) * 8)) * 2, a[0], a[1], a[2], a[3]);
+#pragma unroll
+          for (int nt = 0; nt < NGT; ++nt) mma_bf16_16816(sc[nt], a, qb[nt][ks][0], qb[nt][ks][1]);
+        }
       }
-      __syncthreads();
-      if (s_last) {
-        __threadfence();
-        const int pb = si.pair_base;
-        for (int e = threadIdx.x; e < g * (D / 8); e += blockDim.x) {
-          const int r = e / (D / 8);
-          const int d0 = (e % (D / 8)) * 8;
-          const int head = it.kvh * g + r;
-          float M = -INFINITY;
-          for (int c = 0; c < n_chunks; ++c)
-            M = fmaxf(M, __ldcg(lse_buf + (size_t)(pb + c) * p.num_q_heads + head));
-          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          float wsum = 0.f;
-          if (M != -INFINITY) {
-            for (int c = 0; c < n_chunks; ++c) {
-              const float lc = __ldcg(lse_buf + (size_t)(pb + c) * p.num_q_heads + head);
-              const float w = (lc == -INFINITY) ? 0.f : fast_exp2(lc - M);
-              wsum += w;
-              const float* src = part_buf + ((size_t)(pb + c) * p.num_q_heads + head) * D + d0;
-              const float4 x0 = __ldcg(reinterpret_cast<const float4*>(src));
-              const float4 x1 = __ldcg(reinterpret_cast<const float4*>(src + 4));
-              acc[0] += w * x0.x;
-              acc[1] += w * x0.y;
-              acc[2] += w * x0.z;
-              acc[3] += w * x0.w;
-              acc[4] += w * x1.x;
-              acc[5] += w * x1.y;
-              acc[6] += w * x1.z;
-              acc[7] += w * x1.w;
-            }
-          }
-          const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-          uint4 v;
-          v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-          v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-          v.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
-          v.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
-          *reinterpret_cast<uint4*>(p.out + ((size_t)tok * p.num_q_heads + head) * D + d0) = v;
+      // ---- mask, online softmax per head column ----
+      const int key0 = (int)(x - seg_first) * kPageKeys;
+      const bool ok0 = key0 + gq < seg_kv, ok1 = key0 + gq + 8 < seg_kv;
+      uint32_t pb[NGT][2];
+#pragma unroll
+      for (int nt = 0; nt < NGT; ++nt) {
+        float s0 = ok0 ? sc[nt][0] * p.scale_log2 : -INFINITY;
+        float s1 = ok0 ? sc[nt][1] * p.scale_log2 : -INFINITY;
+        float s2 = ok1 ? sc[nt][2] * p.scale_log2 : -INFINITY;
+        float s3 = ok1 ? sc[nt][3] * p.scale_log2 : -INFINITY;
+        float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+        for (int o2 = 4; o2 < 32; o2 <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, o2));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, o2));
+        }
+        const float mn0 = fmaxf(m[nt][0], mx0), mn1 = fmaxf(m[nt][1], mx1);
+        const float base0 = mn0 == -INFINITY ? 0.f : mn0;
+        const float base1 = mn1 == -INFINITY ? 0.f : mn1;
+        const float a0 = fast_exp2(m[nt][0] - base0), a1 = fast_exp2(m[nt][1] - base1);
+        m[nt][0] = mn0;
+        m[nt][1] = mn1;
+        s0 = fast_exp2(s0 - base0);
+        s1 = fast_exp2(s1 - base1);
+        s2 = fast_exp2(s2 - base0);
+        s3 = fast_exp2(s3 - base1);
+        l[nt][0] = l[nt][0] * a0 + s0 + s2;
+        l[nt][1] = l[nt][1] * a1 + s1 + s3;
+#pragma unroll
+        for (int mt = 0; mt < KSTEPS; ++mt) {
+          o[nt][mt][0] *= a0;
+          o[nt][mt][1] *= a1;
+          o[nt][mt][2] *= a0;
+          o[nt][mt][3] *= a1;
+        }
+        pb[nt][0] = movmatrix_trans(pack_bf16x2(s0, s1));  // keys 0-7
+        pb[nt][1] = movmatrix_trans(pack_bf16x2(s2, s3));  // keys 8-15
+      }
+      // ---- O^T += V^T . P^T : 16 d rows x 8 heads per m-tile ----
+      {
+        const int key = (mi >> 1) * 8 + rr;
+#pragma unroll
+        for (int mt = 0; mt < KSTEPS; ++mt) {
+          const int chunk = mt * 2 + (mi & 1);
+          uint32_t a[4];
+          ldmatrix_x4_trans(vbase + (key * D + ((chunk ^ (key & 7)) * 8)) * 2, a[0], a[1], a[2],
+                            a[3]);
+#pragma unroll
+          for (int nt = 0; nt < NGT; ++nt) mma_bf16_16816(o[nt][mt], a, pb[nt][0], pb[nt][1]);
         }
       }
     }
-    __syncthreads();  // the combine area is rewritten by the next item
+
+    // ---- finish this warp's KV head of the segment ----
+#pragma unroll
+    for (int nt = 0; nt < NGT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int o2 = 4; o2 < 32; o2 <<= 1) l[nt][j] += __shfl_xor_sync(FULL, l[nt][j], o2);
+
+    if (n_chunks <= 1) {
+#pragma unroll
+      for (int nt = 0; nt < NGT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int hl = nt * 8 + 2 * tq + j;
+          if (hl < g) {
+            const float inv = l[nt][j] > 0.f ? 1.f / l[nt][j] : 0.f;
+            __nv_bfloat16* orow = p.out + ((size_t)seg_q * p.num_q_heads + head0 + hl) * D;
+#pragma unroll
+            for (int mt = 0; mt < KSTEPS; ++mt) {
+              orow[mt * 16 + gq] = __float2bfloat16_rn(o[nt][mt][j] * inv);
+              orow[mt * 16 + gq + 8] = __float2bfloat16_rn(o[nt][mt][2 + j] * inv);
+            }
+          }
+        }
+    } else {
+      const int pair = (int)c + seq;  // partial slot of (range c, sequence seq)
+#pragma unroll
+      for (int nt = 0; nt < NGT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int hl = nt * 8 + 2 * tq + j;
+          if (hl < g) {
+            const float inv = l[nt][j] > 0.f ? 1.f / l[nt][j] : 0.f;
+            float* dst = part_buf + ((size_t)pair * p.num_q_heads + head0 + hl) * D;
+#pragma unroll
+            for (int mt = 0; mt < KSTEPS; ++mt) {
+              dst[mt * 16 + gq] = o[nt][mt][j] * inv;
+              dst[mt * 16 + gq + 8] = o[nt][mt][2 + j] * inv;
+            }
+            if (gq == 0)
+              lse_buf[(size_t)pair * p.num_q_heads + head0 + hl] =
+                  l[nt][j] > 0.f ? m[nt][j] + log2f(l[nt][j]) : -INFINITY;
+          }
+        }
+      __threadfence();
+      __syncwarp();
+      int old = 0;
+      if (lane == 0) old = atomicAdd(&counters[(size_t)seq * Hkv + kvh], 1);
+      old = __shfl_sync(FULL, old, 0);
+      if (old == n_chunks - 1) {
+        // last chunk of this (sequence, KV head) to finish: merge all of them
+        __threadfence();
+        const int pb0 = pair_base;
+        for (int hl = 0; hl < g; ++hl) {
+          const int head = head0 + hl;
+          float M = -INFINITY;
+          for (int c = lane; c < n_chunks; c += 32)
+            M = fmaxf(M, __ldcg(lse_buf + (size_t)(pb0 + c) * p.num_q_heads + head));
+#pragma unroll
+          for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, o2));
+          if (lane * 4 < D) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            float wsum = 0.f;
+            if (M != -INFINITY) {
+              for (int c = 0; c < n_chunks; ++c) {
+                const float lc = __ldcg(lse_buf + (size_t)(pb0 + c) * p.num_q_heads + head);
+                const float w = (lc == -INFINITY) ? 0.f : fast_exp2(lc - M);
+                wsum += w;
+                const float4 x = __ldcg(reinterpret_cast<const float4*>(
+                    part_buf + ((size_t)(pb0 + c) * p.num_q_heads + head) * D + lane * 4));
+                acc.x += w * x.x;
+                acc.y += w * x.y;
+                acc.z += w * x.z;
+                acc.w += w * x.w;
+              }
+            }
+            const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+            uint2 v;
+            v.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+            v.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+            *reinterpret_cast<uint2*>(p.out + ((size_t)seg_q * p.num_q_heads + head) * D +
+                                      lane * 4) = v;
+          }
+        }
+        if (lane == 0) counters[(size_t)seq * Hkv + kvh] = 0;  // ready for the next call
+      }
+    }
+
+
+    // ---- next sequence with pages ----
+    if (x < b1) {
+      do {
+        ++seq;
+      } while (pfx(seq + 1) <= x);
+    }
   }
   cp_async_wait<0>();
 }
 
-template <int D, int NSTAGE>
-static cudaError_t launch_decode_t(const DecodeParams& p, int grid, cudaStream_t stream) {
-  using Shape = DecodeShape<D, NSTAGE>;
-  const int smem = Shape::smem_bytes(p.group);
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NSTAGE>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+namespace {
+
+// KV heads per CTA: the largest of 8, 4, 2, 1 that divides num_kv_heads.
+int heads_per_cta(int num_kv_heads) {
+  for (int h = 8; h > 1; h >>= 1)
+    if (num_kv_heads % h == 0) return h;
+  return 1;
+}
+
+template <int D, int HPC, int NSTAGE, int NGT>
+cudaError_t launch_t(const DecodeParams& p, int num_sms, cudaStream_t stream) {
+  using Shape = DecodeShape<D, HPC, NSTAGE>;
+  auto kernel = decode_kernel<D, HPC, NSTAGE, NGT>;
+  const int smem = Shape::smem_bytes(p.self_plan != 0);
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  decode_kernel<D, NSTAGE><<<grid, kDecodeWarps * 32, smem, stream>>>(p);
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, HPC * 32, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  // one resident wave; each KV-head group gets the same number of page ranges,
+  // and there are never more ranges per group than the partial slots allow
+  const int groups = p.num_kv_heads / HPC;
+  long long ranges = (long long)per_sm * num_sms / groups;
+  const long long cap = (kDecodeMaxWarps + p.num_kv_heads - 1) / p.num_kv_heads;
+  if (ranges > cap) ranges = cap;
+  if (ranges < 1) ranges = 1;
+  kernel<<<(unsigned)(ranges * groups), HPC * 32, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode(const DecodeParams& p, int head_dim, int grid, cudaStream_t stream) {
-  if (head_dim == 128) return launch_decode_t<128, 2>(p, grid, stream);
-  return launch_decode_t<64, 3>(p, grid, stream);
+template <int D, int NSTAGE, int NGT>
+cudaError_t launch_hpc(const DecodeParams& p, int hpc, int num_sms, cudaStream_t stream) {
+  switch (hpc) {
+    case 8: return launch_t<D, 8, NSTAGE, NGT>(p, num_sms, stream);
+    case 4: return launch_t<D, 4, NSTAGE, NGT>(p, num_sms, stream);
+    case 2: return launch_t<D, 2, NSTAGE, NGT>(p, num_sms, stream);
+    default: return launch_t<D, 1, NSTAGE, NGT>(p, num_sms, stream);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeParams& p, int head_dim, int num_sms, cudaStream_t stream) {
+  const int hpc = heads_per_cta(p.num_kv_heads);
+  if (head_dim == 128) {
+    if (p.group <= 8) return launch_hpc<128, 3, 1>(p, hpc, num_sms, stream);
+    return launch_hpc<128, 3, 2>(p, hpc, num_sms, stream);
+  }
+  if (p.group <= 8) return launch_hpc<64, 6, 1>(p, hpc, num_sms, stream);
+  return launch_hpc<64, 6, 2>(p, hpc, num_sms, stream);
 }
 
 }  // namespace pa

@@ -19,8 +19,7 @@ cudaError_t launch_write_kv(const void* k, const void* v, const int64_t* slot_ma
 void launch_plan(const int32_t* query_start_loc, const int32_t* seq_lens, int num_seqs,
                  long long num_q_tokens, int max_blocks_per_seq, int block_size,
                  int max_query_len, int max_seq_len, int causal, int num_kv_heads,
-                 int target_items, unsigned char* ws, const WorkspaceLayout& L,
-                 cudaStream_t stream);
+                 unsigned char* ws, const WorkspaceLayout& L, cudaStream_t stream);
 
 // ---- split-KV decode -------------------------------------------------------
 struct DecodeParams {
@@ -28,17 +27,25 @@ struct DecodeParams {
   const __nv_bfloat16* k_cache;
   const __nv_bfloat16* v_cache;
   const int32_t* block_tables;
+  const int32_t* query_start_loc;
+  const int32_t* seq_lens;
+  int num_seqs;
+  long long num_q_tokens;
   int max_blocks_per_seq;
+  int max_query_len; // host hint, checked
+  int max_seq_len;   // host hint, checked
   int num_q_heads;
   int num_kv_heads;
   int group;  // num_q_heads / num_kv_heads, <= 16
   long long num_blocks;
   float scale_log2;  // scale * log2(e)
+  int self_plan;     // 1: every CTA plans the decode work itself (num_seqs <= kSelfPlanMaxSeqs)
   __nv_bfloat16* out;
   unsigned char* ws;
   WorkspaceLayout L;
 };
-cudaError_t launch_decode(const DecodeParams& p, int head_dim, int grid, cudaStream_t stream);
+// Persistent launch: one resident wave, num_sms from the device.
+cudaError_t launch_decode(const DecodeParams& p, int head_dim, int num_sms, cudaStream_t stream);
 
 // ---- tcgen05 prefill ------------------------------------------------------
 struct PrefillParams {

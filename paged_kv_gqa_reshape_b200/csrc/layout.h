@@ -10,11 +10,10 @@ namespace pa {
 
 constexpr int kPrefillTileM = 128;      // query rows per prefill tile (tcgen05 M)
 constexpr int kPrefillTileN = 128;      // keys per prefill KV tile (tcgen05 N)
-constexpr int kDecodeWarps = 4;         // warps per decode CTA
 constexpr int kPageKeys = 16;           // block_size this build supports
-constexpr int kDecodeMinChunk = 256;    // smallest split-KV chunk (keys)
-constexpr int kDecodeMaxItems = 4096;   // upper bound on the plan's (seq, chunk, kv-head) target
+constexpr int kDecodeMaxWarps = 4096;   // bound on decode warps in one launch (8 per SM)
 constexpr int kCostBuckets = 4096;      // prefill tiles are sorted by KV-tile count
+constexpr int kSelfPlanMaxSeqs = 1024;  // decode CTAs plan for themselves up to this many sequences
 
 // Sanitised geometry of one sequence, written by the plan kernel.  The
 // attention kernels read lengths only from here, never from the raw inputs.
@@ -22,17 +21,13 @@ struct SeqInfo {
   int32_t q_start;    // first query token of the sequence
   int32_t q_len;      // number of query tokens (0 if the sequence is skipped)
   int32_t kv_len;     // number of keys (clamped to the block table's reach)
-  int32_t n_chunks;   // decode only: split-KV chunks (0 for non-decode sequences)
-  int32_t pair_base;  // decode only: index of the first (seq, chunk) pair
-  int32_t chunk_len;  // decode only: keys per chunk (multiple of 64)
-  int32_t pad0, pad1;
+  int32_t pad;
 };
 
 struct PlanHeader {
-  int32_t num_prefill_tiles;  // entries in the prefill tile list
-  int32_t num_decode_pairs;   // entries in the decode (seq, chunk) list
-  int32_t total_decode_keys;
-  int32_t pad[61];
+  int32_t num_prefill_tiles;   // entries in the prefill tile list
+  int32_t total_decode_pages;  // 16-key pages over all single-query sequences
+  int32_t pad[62];
 };
 
 struct WorkspaceLayout {
@@ -40,13 +35,13 @@ struct WorkspaceLayout {
   size_t header;     // PlanHeader
   size_t seq_info;   // SeqInfo[num_seqs]
   size_t tiles;      // int2[max_tiles]   (seq, first query row of the tile)
-  size_t pairs;      // int2[max_pairs]   (seq, chunk)
+  size_t page_pfx;   // int32[num_seqs + 1]  exclusive prefix of decode pages
   size_t counters;   // int32[num_seqs * num_kv_heads]  split-KV arrival counters
-  size_t lse;        // float[max_pairs * num_q_heads]   log2-sum-exp per partial
-  size_t partial;    // float[max_pairs * num_q_heads * head_dim]
+  size_t lse;        // float[max_slots * num_q_heads]   log2-sum-exp per partial
+  size_t partial;    // float[max_slots * num_q_heads * head_dim]
   size_t total;
   int64_t max_tiles;
-  int64_t max_pairs;
+  int64_t max_slots;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -64,18 +59,17 @@ inline WorkspaceLayout make_layout(int64_t num_seqs, int64_t num_q_tokens, int64
   L.max_tiles = (num_q_tokens + kPrefillTileM - 1) / kPrefillTileM + num_seqs;
   L.tiles = off;
   off = align_up(off + 8 * (size_t)L.max_tiles, 256);
-  // The plan picks chunk >= total_decode_keys * Hkv / target_items with
-  // target_items <= kDecodeMaxItems, so sum_s ceil(L_s / chunk) <=
-  // target_items / Hkv + num_seqs.
-  L.max_pairs = (kDecodeMaxItems + num_kv_heads - 1) / num_kv_heads + num_seqs;
-  L.pairs = off;
-  off = align_up(off + 8 * (size_t)L.max_pairs, 256);
+  // Decode CTA c of a KV-head group covering sequence s writes partial slot
+  // c + s; a launch has at most kDecodeMaxWarps / Hkv page ranges per group.
+  L.max_slots = (kDecodeMaxWarps + num_kv_heads - 1) / num_kv_heads + num_seqs;
+  L.page_pfx = off;
+  off = align_up(off + 4 * (size_t)(num_seqs + 1), 256);
   L.counters = off;
   off = align_up(off + 4 * (size_t)(num_seqs * num_kv_heads), 256);
   L.lse = off;
-  off = align_up(off + 4 * (size_t)(L.max_pairs * num_q_heads), 256);
+  off = align_up(off + 4 * (size_t)(L.max_slots * num_q_heads), 256);
   L.partial = off;
-  off = align_up(off + 4 * (size_t)(L.max_pairs * num_q_heads * head_dim), 256);
+  off = align_up(off + 4 * (size_t)(L.max_slots * num_q_heads * head_dim), 256);
   L.total = off;
   return L;
 }

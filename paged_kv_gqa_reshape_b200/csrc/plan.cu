@@ -4,9 +4,9 @@
 //  - the prefill tile list: one entry per 128-query-row tile of every
 //    sequence with more than one query, ordered by descending KV-tile count
 //    (longest work first, for the persistent prefill grid);
-//  - the decode list: one (seq, chunk) pair per split-KV chunk of every
-//    single-query sequence, with a chunk length chosen from the total decode
-//    key count so that the decode grid gets a few items per CTA;
+//  - the exclusive prefix of 16-key pages over the single-query (decode)
+//    sequences, from which the decode CTAs cut their balanced page ranges
+//    when there are too many sequences for them to plan themselves;
 //  - zeroed split-KV arrival counters.
 // This plays the role of the device-side runtime length reduction of
 // ROCm/TransformerEngine PR #461 (description: the real maximum is found on
@@ -61,25 +61,21 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
     plan_kernel(const int32_t* __restrict__ query_start_loc, const int32_t* __restrict__ seq_lens,
                 int num_seqs, long long num_q_tokens, int max_blocks_per_seq, int block_size,
                 int max_query_len, int max_seq_len, int causal, int num_kv_heads,
-                int target_items, unsigned char* ws, WorkspaceLayout L) {
+                unsigned char* ws, WorkspaceLayout L) {
   uint32_t* err = reinterpret_cast<uint32_t*>(ws + L.err);
   PlanHeader* hdr = reinterpret_cast<PlanHeader*>(ws + L.header);
   SeqInfo* info = reinterpret_cast<SeqInfo*>(ws + L.seq_info);
   int2* tiles = reinterpret_cast<int2*>(ws + L.tiles);
-  int2* pairs = reinterpret_cast<int2*>(ws + L.pairs);
+  int32_t* page_pfx = reinterpret_cast<int32_t*>(ws + L.page_pfx);
   int32_t* counters = reinterpret_cast<int32_t*>(ws + L.counters);
 
   __shared__ int s_warp[32];
-  __shared__ unsigned long long s_dec_keys;
   __shared__ int s_hist[kCostBuckets];
   __shared__ int s_carry;
   __shared__ uint32_t s_err;
 
   const int tid = threadIdx.x;
-  if (tid == 0) {
-    s_dec_keys = 0;
-    s_err = 0;
-  }
+  if (tid == 0) s_err = 0;
   for (int i = tid; i < kCostBuckets; i += blockDim.x) s_hist[i] = 0;
   for (long long i = tid; i < (long long)num_seqs * num_kv_heads; i += blockDim.x)
     counters[i] = 0;
@@ -110,58 +106,37 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
     si.q_start = (int)qs;
     si.q_len = (int)ql;
     si.kv_len = (int)kv;
-    si.n_chunks = 0;
-    si.pair_base = 0;
-    si.chunk_len = 0;
-    si.pad0 = si.pad1 = 0;
+    si.pad = 0;
     info[s] = si;
-    if (ql == 1) atomicAdd(&s_dec_keys, (unsigned long long)kv);
     if (e) atomicOr(&s_err, e);
   }
   __syncthreads();
 
-  // split-KV chunk: enough chunks for ~target_items (seq, chunk, kv-head)
-  // items, never below kDecodeMinChunk keys, always a multiple of 64 keys
-  long long want = ((long long)s_dec_keys * num_kv_heads + target_items - 1) / max(target_items, 1);
-  int chunk = (int)max((long long)kDecodeMinChunk, min(want, (long long)1 << 30));
-  chunk = (chunk + 63) / 64 * 64;
-
-  // ---- pass 2: chunk counts, tile histogram ---------------------------------
+  // ---- pass 2: decode page prefix, tile histogram --------------------------
   if (tid == 0) s_carry = 0;
   __syncthreads();
   for (int base = 0; base < num_seqs; base += blockDim.x) {
-    int s = base + tid;
-    int n_chunks = 0;
-    SeqInfo si;
+    const int s = base + tid;
+    int pages = 0;
     if (s < num_seqs) {
-      si = info[s];
-      if (si.q_len == 1) n_chunks = max(1, (si.kv_len + chunk - 1) / chunk);
+      const SeqInfo si = info[s];
+      if (si.q_len == 1) pages = (si.kv_len + kPageKeys - 1) / kPageKeys;
       if (si.q_len > 1) {
         for (int r = 0; r < si.q_len; r += kPrefillTileM) {
-          int c = tile_cost(si, r, causal);
+          const int c = tile_cost(si, r, causal);
           atomicAdd(&s_hist[kCostBuckets - 1 - min(c, kCostBuckets - 1)], 1);
         }
       }
     }
     int excl;
-    int total = block_exclusive_scan(n_chunks, &excl, s_warp);
-    if (s < num_seqs && n_chunks) {
-      int pb = s_carry + excl;
-      info[s].n_chunks = n_chunks;
-      info[s].pair_base = pb;
-      info[s].chunk_len = chunk;
-      for (int c = 0; c < n_chunks; ++c)
-        if ((long long)(pb + c) < (long long)L.max_pairs) pairs[pb + c] = make_int2(s, c);
-    }
+    const int total = block_exclusive_scan(pages, &excl, s_warp);
+    if (s < num_seqs) page_pfx[s] = s_carry + excl;
     __syncthreads();
     if (tid == 0) s_carry += total;
     __syncthreads();
   }
-  int num_pairs = s_carry;
-  if ((long long)num_pairs > (long long)L.max_pairs) {  // cannot happen for target_items <= kDecodeMaxItems
-    if (tid == 0) atomicOr(&s_err, PA_DEVERR_LENGTHS);
-    num_pairs = (int)L.max_pairs;
-  }
+  if (tid == 0) page_pfx[num_seqs] = s_carry;
+  const int total_pages = s_carry;
 
   // ---- pass 3: counting sort of prefill tiles by descending cost -----------
   // exclusive scan of the histogram (bucket 0 = most expensive)
@@ -200,8 +175,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
     // the last bucket's running cursor ends at the number of tiles
     num_tiles = (int)min((long long)s_hist[kCostBuckets - 1], (long long)L.max_tiles);
     hdr->num_prefill_tiles = num_tiles;
-    hdr->num_decode_pairs = num_pairs;
-    hdr->total_decode_keys = (int)min(s_dec_keys, (unsigned long long)0x7fffffff);
+    hdr->total_decode_pages = total_pages;
     if (s_err) atomicOr(err, s_err);
   }
 }
@@ -209,12 +183,10 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
 void launch_plan(const int32_t* query_start_loc, const int32_t* seq_lens, int num_seqs,
                  long long num_q_tokens, int max_blocks_per_seq, int block_size,
                  int max_query_len, int max_seq_len, int causal, int num_kv_heads,
-                 int target_items, unsigned char* ws, const WorkspaceLayout& L,
-                 cudaStream_t stream) {
+                 unsigned char* ws, const WorkspaceLayout& L, cudaStream_t stream) {
   plan_kernel<<<1, kPlanThreads, 0, stream>>>(query_start_loc, seq_lens, num_seqs, num_q_tokens,
                                               max_blocks_per_seq, block_size, max_query_len,
-                                              max_seq_len, causal, num_kv_heads, target_items,
-                                              ws, L);
+                                              max_seq_len, causal, num_kv_heads, ws, L);
 }
 
 }  // namespace pa

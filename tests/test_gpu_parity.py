@@ -322,3 +322,26 @@ def test_prefill_with_decode_hint_is_reported():
     _, _, _, ws = run_varlen(dev, max_query_len=1)
     st, bits = pa.get_error(ws)
     assert bits & pa.DEVERR_HINT
+
+
+def test_decode_many_sequences_uses_plan_kernel_lists():
+    # more sequences than the decode CTAs plan for themselves
+    rng = np.random.default_rng(77)
+    lens = rng.integers(0, 300, size=1100).tolist()
+    cpu = build(lens, [1 if l > 0 else 0 for l in lens], 8, 2, 128, seed=77)
+    out, _, _, ws = run_varlen(case_to(cpu, "cuda"))
+    assert_attention_close(out, oracle_varlen(cpu), what="decode, 1100 sequences")
+    assert pa.get_error(ws) == (0, 0)
+
+
+def test_decode_repeated_calls_reuse_counters():
+    # split-KV arrival counters return to zero after every call
+    cpu = build([5000, 3000, 17, 4096], [1, 1, 1, 1], 32, 8, 128, seed=13)
+    dev = case_to(cpu, "cuda")
+    ref = oracle_varlen(cpu)
+    ws = pa.varlen_workspace(dev.num_seqs, dev.num_q_tokens, dev.num_q_heads, dev.num_kv_heads,
+                             dev.head_dim)
+    outs = [run_varlen(dev, workspace=ws)[0] for _ in range(3)]
+    for o in outs:
+        assert_attention_close(o, ref, what="repeated decode")
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
