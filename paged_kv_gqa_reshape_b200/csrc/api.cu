@@ -269,7 +269,7 @@ pa_status pa_attention_smallseq(const void* q, const void* k, const void* v,
   p.scale_log2 = scale * 1.4426950408889634f;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.err = static_cast<uint32_t*>(workspace);
-  cudaError_t e = pa::launch_smallseq(p, head_dim, static_cast<cudaStream_t>(stream));
+  cudaError_t e = pa::launch_smallseq(p, head_dim, sm_count(), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

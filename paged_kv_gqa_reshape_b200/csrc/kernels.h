@@ -82,6 +82,7 @@ struct SmallSeqParams {
   __nv_bfloat16* out;
   uint32_t* err;
 };
-cudaError_t launch_smallseq(const SmallSeqParams& p, int head_dim, cudaStream_t stream);
+cudaError_t launch_smallseq(const SmallSeqParams& p, int head_dim, int num_sms,
+                            cudaStream_t stream);
 
 }  // namespace pa
