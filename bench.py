@@ -153,6 +153,24 @@ class ClockSampler:
                 "power_w_max": max(power) if power else None}
 
 
+def shard_seed(rank: int) -> int:
+    """Each rank attends its own, independently drawn decode batch."""
+    return 1002 + rank
+
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """Elapsed time of the whole job: the slowest rank's (MAX all-reduce)."""
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(bytes_per_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Throughput of all ranks together: every rank moves bytes_per_step per step."""
+    return bytes_per_step * steps * world / (max_ms * 1e-3) / 1e9
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -263,7 +281,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     hbm_peak, tc_peak, tc_sust, peak_kind = measured_peaks()
 
-    case = workloads.decode_batch(device=dev, seed=1002 + rank, keep_logical=False)
+    case = workloads.decode_batch(device=dev, seed=shard_seed(rank), keep_logical=False)
     ws = pa.varlen_workspace(case.num_seqs, case.num_q_tokens, case.num_q_heads,
                              case.num_kv_heads, case.head_dim, device=dev)
     out = torch.empty_like(case.q)
@@ -309,21 +327,14 @@ def run_ours(args, rank, world, local_rank):
     if st != 0:
         raise RuntimeError(f"device error word {bits:#x} in the timed region")
 
-    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = max_over_ranks(elapsed_ms, world, dev)
     bytes_step = scatter_bytes(case) + attention_bytes(case)
-    total_bytes = bytes_step * args.steps * world
-    value = total_bytes / (max_ms * 1e-3) / 1e9
+    value = whole_job_gbs(bytes_step, args.steps, world, max_ms)
 
     # end to end through the public API: pinned host inputs in, output back, every step
     e2e = run_e2e(pa, case, args, dev, ws)
-    if world > 1:
-        te = torch.tensor([e2e["ms"]], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
-        e2e["ms"] = float(te.item())
-    e2e_value = bytes_step * args.steps * world / (e2e["ms"] * 1e-3) / 1e9
+    e2e["ms"] = max_over_ranks(e2e["ms"], world, dev)
+    e2e_value = whole_job_gbs(bytes_step, args.steps, world, e2e["ms"])
 
     attn_bytes = attention_bytes(case)
     achieved = attn_bytes / (attn_ms * 1e-3) / 1e9
