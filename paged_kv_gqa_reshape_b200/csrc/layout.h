@@ -9,6 +9,7 @@
 namespace pa {
 
 constexpr int kPrefillTileM = 128;      // query rows per prefill tile (tcgen05 M)
+constexpr int kPrefillItemRows = 256;   // query rows per prefill work item: two tiles
 constexpr int kPrefillTileN = 128;      // keys per prefill KV tile (tcgen05 N)
 constexpr int kPageKeys = 16;           // block_size this build supports
 constexpr int kDecodeMaxWarps = 4096;   // bound on decode warps in one launch (8 per SM)
@@ -34,7 +35,7 @@ struct WorkspaceLayout {
   size_t err;        // uint32 error word (PA_ERROR_WORD_BYTES reserved)
   size_t header;     // PlanHeader
   size_t seq_info;   // SeqInfo[num_seqs]
-  size_t tiles;      // int2[max_tiles]   (seq, first query row of the tile)
+  size_t tiles;      // int2[max_tiles]   (seq, first query row of a 256-row work item)
   size_t page_pfx;   // int32[num_seqs + 1]  exclusive prefix of decode pages
   size_t counters;   // int32[num_seqs * num_kv_heads]  split-KV arrival counters
   size_t lse;        // float[max_slots * num_q_heads]   log2-sum-exp per partial
@@ -56,7 +57,7 @@ inline WorkspaceLayout make_layout(int64_t num_seqs, int64_t num_q_tokens, int64
   off += sizeof(PlanHeader);
   L.seq_info = off;
   off = align_up(off + sizeof(SeqInfo) * (size_t)num_seqs, 256);
-  L.max_tiles = (num_q_tokens + kPrefillTileM - 1) / kPrefillTileM + num_seqs;
+  L.max_tiles = (num_q_tokens + kPrefillItemRows - 1) / kPrefillItemRows + num_seqs;
   L.tiles = off;
   off = align_up(off + 8 * (size_t)L.max_tiles, 256);
   // Decode CTA c of a KV-head group covering sequence s writes partial slot

@@ -1,9 +1,10 @@
 // Work planning on the device (one CTA), so no length ever travels to the host.
 //
 // Reads query_start_loc and seq_lens, sanitises them into SeqInfo, and builds
-//  - the prefill tile list: one entry per 128-query-row tile of every
-//    sequence with more than one query, ordered by descending KV-tile count
-//    (longest work first, for the persistent prefill grid);
+//  - the prefill work list: one entry per 256-query-row item (two 128-row
+//    tiles) of every sequence with more than one query, ordered by
+//    descending KV-tile count (longest work first, for the persistent
+//    prefill grid);
 //  - the exclusive prefix of 16-key pages over the single-query (decode)
 //    sequences, from which the decode CTAs cut their balanced page ranges
 //    when there are too many sequences for them to plan themselves;
@@ -48,11 +49,19 @@ __device__ int block_exclusive_scan(int v, int* out_excl, int* s_warp) {
   return total;
 }
 
-__device__ __forceinline__ int tile_cost(const SeqInfo& si, int row0, int causal) {
-  int last_row = min(si.q_len, row0 + kPrefillTileM) - 1;
+// KV tiles of one 128-row tile whose rows are [row0, row0 + rows)
+__device__ __forceinline__ int kv_tiles(const SeqInfo& si, int row0, int rows, int causal) {
+  if (rows <= 0) return 0;
   int vis = si.kv_len;
-  if (causal) vis = max(0, min(si.kv_len, si.kv_len - si.q_len + last_row + 1));
+  if (causal) vis = max(0, min(si.kv_len, si.kv_len - si.q_len + row0 + rows));
   return (vis + kPrefillTileN - 1) / kPrefillTileN;
+}
+
+// cost of a 256-row work item: the KV tiles of its two 128-row tiles
+__device__ __forceinline__ int tile_cost(const SeqInfo& si, int row0, int causal) {
+  const int rows_a = min(kPrefillTileM, si.q_len - row0);
+  const int rows_b = min(kPrefillTileM, si.q_len - row0 - kPrefillTileM);
+  return kv_tiles(si, row0, rows_a, causal) + kv_tiles(si, row0 + kPrefillTileM, rows_b, causal);
 }
 
 }  // namespace
@@ -122,7 +131,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
       const SeqInfo si = info[s];
       if (si.q_len == 1) pages = (si.kv_len + kPageKeys - 1) / kPageKeys;
       if (si.q_len > 1) {
-        for (int r = 0; r < si.q_len; r += kPrefillTileM) {
+        for (int r = 0; r < si.q_len; r += kPrefillItemRows) {
           const int c = tile_cost(si, r, causal);
           atomicAdd(&s_hist[kCostBuckets - 1 - min(c, kCostBuckets - 1)], 1);
         }
@@ -162,7 +171,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
   for (int s = tid; s < num_seqs; s += blockDim.x) {
     SeqInfo si = info[s];
     if (si.q_len > 1) {
-      for (int r = 0; r < si.q_len; r += kPrefillTileM) {
+      for (int r = 0; r < si.q_len; r += kPrefillItemRows) {
         int c = tile_cost(si, r, causal);
         int pos = atomicAdd(&s_hist[kCostBuckets - 1 - min(c, kCostBuckets - 1)], 1);
         if ((long long)pos < (long long)L.max_tiles) tiles[pos] = make_int2(s, r);  // overlapping query ranges can overflow

@@ -9,24 +9,31 @@
 // diagonal mask, BestLA's CPU tiles) are prior art; this is a flash-style
 // kernel written for sm_100a:
 //
-//  * persistent grid, one CTA per SM, walking the plan's tile list (128 query
-//    rows of one head per work item, most expensive first);
-//  * warp 0 (one lane): TMA producer.  Q tile via a 3-D map over
+//  * persistent grid, one CTA per SM, walking the plan's work list; a work
+//    item is 256 query rows of one head, split into two 128-row tiles A and B
+//    that share every K/V tile;
+//  * warp 0 (one lane): TMA producer.  Q tiles via a 3-D map over
 //    [tokens, Hq, D]; each 128-key K/V tile as eight 16-key pages fetched
 //    through the block table with a 4-D map over [blocks, 16, Hkv, D]
 //    (a page past the sequence end, or a bad block id, is fetched at an
 //    out-of-range coordinate, i.e. as zeros).  128-byte swizzle, no
-//    multicast.  NS-deep K and V rings;
-//  * warp 1 (one lane): tcgen05.mma issuer.  S = Q.K^T into one of two TMEM
-//    buffers (M = 128, N = 128, K = 16 per instruction), O += P.V into a TMEM
-//    accumulator (B = V read MN-major straight from the TMA layout);
-//    completion reported through tcgen05.commit -> mbarrier;
-//  * warps 2-5: softmax, one thread per query row (= TMEM lane).  tcgen05.ld
-//    of the S row, scale folded with log2 e, mask only on tiles that cross
-//    the diagonal or the sequence end, online softmax in fp32 with lazy
-//    rescaling (O in TMEM is rescaled only when the running max grows by
-//    more than 2^8), P rounded to bf16 into a swizzled SMEM tile that is the
-//    A operand of the P.V MMA; final O / l -> bf16 -> global.
+//    multicast.  K and V tiles go through one 3-slot ring in the order
+//    K0 V0 K1 V1 ...;
+//  * warp 1 (one lane): tcgen05.mma issuer.  Per KV tile j it issues
+//    PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): S = Q.K^T into the tile's TMEM
+//    S buffer (M = 128, N = 128, K = 16 per instruction) and O += P.V into
+//    the tile's TMEM accumulator (B = V read MN-major straight from the TMA
+//    layout).  While one tile's softmax runs, the tensor core works on the
+//    other tile; completion is reported through tcgen05.commit -> mbarrier;
+//  * warps 2-5 / 6-9: softmax of tile A / B, one thread per query row
+//    (= TMEM lane).  tcgen05.ld of the S row, mask only on tiles that cross
+//    the diagonal or the sequence end, online softmax in fp32 (scale folded
+//    into the exponent's FFMA, tree reductions) with lazy rescaling (O in
+//    TMEM is rescaled only when the running max grows by more than 2^8),
+//    P rounded to bf16 into the tile's swizzled SMEM buffer, the A operand of
+//    the P.V MMA; final O / l -> bf16 -> global.
+// TMEM: S_A, S_B, O_A, O_B (4 x 128 columns for D = 128).
+// SMEM: Q_A, Q_B, the 3-slot K/V ring and P_A, P_B (224 KB for D = 128).
 // Every mbarrier wait is bounded in time; a CTA that gives up raises
 // PA_DEVERR_TIMEOUT, lets in-flight copies land, frees its TMEM and exits.
 #include <math.h>
@@ -39,33 +46,44 @@ namespace pa {
 
 namespace {
 
-constexpr int kThreads = 192;  // 6 warps
+constexpr int kWarps = 10;  // 0 producer, 1 MMA, 2-5 softmax A, 6-9 softmax B
+constexpr int kThreads = kWarps * 32;
 constexpr int BM = kPrefillTileM;
 constexpr int BN = kPrefillTileN;
+constexpr int kRing = 3;  // K/V slots
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows by > 2^8
 
-template <int D, int NS>
+template <int D>
 struct PrefillSmem {
-  static constexpr int kQBytes = BM * D * 2;
+  static constexpr int kQBytes = BM * D * 2;   // one 128-row Q tile
   static constexpr int kKVBytes = BN * D * 2;  // one K or V tile
-  static constexpr int kPBytes = BM * BN * 2;
-  static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + kQBytes;
-  static constexpr int kVOff = kKOff + NS * kKVBytes;
-  static constexpr int kPOff = kVOff + NS * kKVBytes;
-  static constexpr int kBarOff = kPOff + kPBytes;
-  // barriers: q_full, q_empty, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
-  //           s_full[2], p_full, o_done
-  static constexpr int kNumBars = 2 + 4 * NS + 2 + 2;
+  static constexpr int kPBytes = BM * BN * 2;  // one P tile
+  static constexpr int kQOff = 0;              // Q_A, Q_B
+  static constexpr int kRingOff = kQOff + 2 * kQBytes;
+  static constexpr int kPOff = kRingOff + kRing * kKVBytes;  // P_A, P_B
+  static constexpr int kBarOff = kPOff + 2 * kPBytes;
+  // barriers: q_full, q_empty, slot_full[kRing], slot_empty[kRing], s_full[2],
+  //           p_full[2], o_done[2]
+  static constexpr int kNumBars = 2 + 2 * kRing + 6;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 64;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B
 };
 
 struct Work {
-  int seq, head, row0, rows, q_start, q_len, kv_len, n;
+  int seq, head, row0, q_start, q_len, kv_len;
+  int rows[2];  // query rows of tile A / B in this item (B may have none)
+  int n[2];     // KV tiles tile A / B must visit
+  int nmax;
 };
+
+__device__ __forceinline__ int kv_tiles_for(int kv_len, int q_len, int row0, int rows, int causal) {
+  if (rows <= 0) return 0;
+  int vis = kv_len;
+  if (causal) vis = max(0, min(kv_len, kv_len - q_len + row0 + rows));
+  return (vis + BN - 1) / BN;
+}
 
 __device__ __forceinline__ Work decode_work(int w, const int2* tiles, const SeqInfo* info,
                                             int num_q_heads, int causal) {
@@ -78,21 +96,22 @@ __device__ __forceinline__ Work decode_work(int w, const int2* tiles, const SeqI
   k.q_start = si.q_start;
   k.q_len = si.q_len;
   k.kv_len = si.kv_len;
-  k.rows = min(BM, si.q_len - t.y);
-  int vis = si.kv_len;
-  if (causal) vis = max(0, min(si.kv_len, si.kv_len - si.q_len + t.y + k.rows));
-  k.n = (vis + BN - 1) / BN;
+  k.rows[0] = min(BM, si.q_len - t.y);
+  k.rows[1] = max(0, min(BM, si.q_len - t.y - BM));
+  k.n[0] = kv_tiles_for(si.kv_len, si.q_len, t.y, k.rows[0], causal);
+  k.n[1] = kv_tiles_for(si.kv_len, si.q_len, t.y + BM, k.rows[1], causal);
+  k.nmax = max(k.n[0], k.n[1]);
   return k;
 }
 
 }  // namespace
 
-template <int D, int NS>
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(PrefillParams p, const __grid_constant__ CUtensorMap q_map,
                    const __grid_constant__ CUtensorMap k_map,
                    const __grid_constant__ CUtensorMap v_map) {
-  using SM = PrefillSmem<D, NS>;
+  using SM = PrefillSmem<D>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -103,19 +122,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBarOff);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* k_full = bars + 2;
-  uint64_t* k_empty = k_full + NS;
-  uint64_t* v_full = k_empty + NS;
-  uint64_t* v_empty = v_full + NS;
-  uint64_t* s_full = v_empty + NS;  // [2]
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_done = p_full + 1;
+  uint64_t* slot_full = bars + 2;
+  uint64_t* slot_empty = slot_full + kRing;
+  uint64_t* s_full = slot_empty + kRing;  // [2]: tile A, tile B
+  uint64_t* p_full = s_full + 2;          // [2]
+  uint64_t* o_done = p_full + 2;          // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::kMiscOff + 4);
 
   const uint32_t q_s = smem_u32(smem + SM::kQOff);
-  const uint32_t k_s = smem_u32(smem + SM::kKOff);
-  const uint32_t v_s = smem_u32(smem + SM::kVOff);
+  const uint32_t ring_s = smem_u32(smem + SM::kRingOff);
   const uint32_t p_s = smem_u32(smem + SM::kPOff);
 
   unsigned char* ws = p.ws;
@@ -128,16 +144,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(k_full + i, 1);
-      mbar_init(k_empty + i, 1);
-      mbar_init(v_full + i, 1);
-      mbar_init(v_empty + i, 1);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(slot_full + i, 1);
+      mbar_init(slot_empty + i, 1);
     }
-    mbar_init(s_full + 0, 1);
-    mbar_init(s_full + 1, 1);
-    mbar_init(p_full, 4 * 32);
-    mbar_init(o_done, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(s_full + x, 1);
+      mbar_init(p_full + x, 4 * 32);
+      mbar_init(o_done + x, 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -149,8 +164,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_s0 = tmem;          // S buffers: columns [0, 256)
-  const uint32_t tmem_o = tmem + 2 * BN;  // O: columns [256, 256 + D)
+  // S_A, S_B: columns [0, 128), [128, 256); O_A, O_B: [256, 256 + D), [256 + D, 256 + 2D)
+  auto tmem_s = [&](int x) { return tmem + (uint32_t)(x * BN); };
+  auto tmem_o = [&](int x) { return tmem + (uint32_t)(2 * BN + x * D); };
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
@@ -158,22 +174,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tma_desc(&q_map);
       prefetch_tma_desc(&k_map);
       prefetch_tma_desc(&v_map);
-      int kv_it = 0, tcount = 0;
+      long long ld = 0;  // K/V tiles loaded so far (slot = ld % kRing)
+      int tcount = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < num_work && ok; w += gridDim.x) {
         const Work wk = decode_work(w, tiles, info, p.num_q_heads, p.causal);
-        if (wk.n == 0) continue;
+        if (wk.nmax == 0) continue;
         const int kvh = wk.head / p.group;
         if (tcount > 0) ok = mbar_wait_bounded(q_empty, (tcount - 1) & 1, abort_flag, err);
         if (!ok) break;
-        mbar_arrive_expect_tx(q_full, SM::kQBytes);
+        mbar_arrive_expect_tx(q_full, 2 * SM::kQBytes);
 #pragma unroll
-        for (int dh = 0; dh < D / 64; ++dh)
-          tma_load_3d(q_s + dh * (BM * 128), &q_map, q_full, dh * 64, wk.head,
-                      wk.q_start + wk.row0);
+        for (int x = 0; x < 2; ++x)
+#pragma unroll
+          for (int dh = 0; dh < D / 64; ++dh)
+            tma_load_3d(q_s + x * SM::kQBytes + dh * (BM * 128), &q_map, q_full, dh * 64, wk.head,
+                        wk.q_start + wk.row0 + x * BM);
         const int32_t* table = p.block_tables + (size_t)wk.seq * p.max_blocks_per_seq;
-        for (int j = 0; j < wk.n && ok; ++j, ++kv_it) {
-          const int st = kv_it % NS, round = kv_it / NS;
+        for (int j = 0; j < wk.nmax && ok; ++j) {
           int blk[BN / kPageKeys];
 #pragma unroll
           for (int pg = 0; pg < BN / kPageKeys; ++pg) {
@@ -188,24 +206,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             blk[pg] = b;
           }
-          if (round > 0) ok = mbar_wait_bounded(k_empty + st, (round - 1) & 1, abort_flag, err);
-          if (!ok) break;
-          mbar_arrive_expect_tx(k_full + st, SM::kKVBytes);
 #pragma unroll
-          for (int pg = 0; pg < BN / kPageKeys; ++pg)
+          for (int kv = 0; kv < 2; ++kv, ++ld) {  // K_j, then V_j
+            const int st = (int)(ld % kRing);
+            const long long round = ld / kRing;
+            if (round > 0) ok = mbar_wait_bounded(slot_empty + st, (round - 1) & 1, abort_flag, err);
+            if (!ok) break;
+            mbar_arrive_expect_tx(slot_full + st, SM::kKVBytes);
+            const void* map = kv == 0 ? (const void*)&k_map : (const void*)&v_map;
 #pragma unroll
-            for (int dh = 0; dh < D / 64; ++dh)
-              tma_load_4d(k_s + st * SM::kKVBytes + dh * (BN * 128) + pg * (kPageKeys * 128),
-                          &k_map, k_full + st, dh * 64, kvh, 0, blk[pg]);
-          if (round > 0) ok = mbar_wait_bounded(v_empty + st, (round - 1) & 1, abort_flag, err);
-          if (!ok) break;
-          mbar_arrive_expect_tx(v_full + st, SM::kKVBytes);
+            for (int pg = 0; pg < BN / kPageKeys; ++pg)
 #pragma unroll
-          for (int pg = 0; pg < BN / kPageKeys; ++pg)
-#pragma unroll
-            for (int dh = 0; dh < D / 64; ++dh)
-              tma_load_4d(v_s + st * SM::kKVBytes + dh * (BN * 128) + pg * (kPageKeys * 128),
-                          &v_map, v_full + st, dh * 64, kvh, 0, blk[pg]);
+              for (int dh = 0; dh < D / 64; ++dh)
+                tma_load_4d(ring_s + st * SM::kKVBytes + dh * (BN * 128) + pg * (kPageKeys * 128),
+                            map, slot_full + st, dh * 64, kvh, 0, blk[pg]);
+          }
         }
         ++tcount;
       }
@@ -215,193 +230,231 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = instr_desc_bf16(BM, BN, 0);
       constexpr uint32_t idesc_o = instr_desc_bf16(BM, D, 1);
-      int kv_it = 0, s_it = 0, tcount = 0;
+      long long ld = 0;   // K/V tiles consumed (mirrors the producer)
+      int tcount = 0;
+      int s_it[2] = {0, 0}, pv_it[2] = {0, 0};
       bool ok = true;
-      auto issue_s = [&](int sidx, int stage) {
-        const uint32_t d_tmem = tmem_s0 + (sidx & 1) * BN;
+      auto wait_tile = [&](long long idx) {
+        return mbar_wait_bounded(slot_full + (int)(idx % kRing), (uint32_t)((idx / kRing) & 1),
+                                 abort_flag, err);
+      };
+      auto issue_s = [&](int x, long long kidx) {
+        const uint32_t kb = ring_s + (int)(kidx % kRing) * SM::kKVBytes;
+        const uint32_t qb = q_s + x * SM::kQBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-          const uint64_t a = smem_desc_sw128(q_s + off, 16, 1024);
-          const uint64_t b = smem_desc_sw128(k_s + stage * SM::kKVBytes + off, 16, 1024);
-          tc_mma(d_tmem, a, b, idesc_s, kk > 0 ? 1u : 0u);
+          tc_mma(tmem_s(x), smem_desc_sw128(qb + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
+                 idesc_s, kk > 0 ? 1u : 0u);
         }
+        tc_commit(s_full + x);
+        ++s_it[x];
       };
-      auto issue_o = [&](int stage, bool accumulate) {
+      auto issue_pv = [&](int x, long long vidx, bool accumulate) {
+        const uint32_t vb = ring_s + (int)(vidx % kRing) * SM::kKVBytes;
+        const uint32_t pb = p_s + x * SM::kPBytes;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t a =
-              smem_desc_sw128(p_s + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t b = smem_desc_sw128(v_s + stage * SM::kKVBytes + kk * (16 * 128),
-                                             BN * 128, 1024);
-          tc_mma(tmem_o, a, b, idesc_o, (accumulate || kk > 0) ? 1u : 0u);
+          const uint64_t a = smem_desc_sw128(pb + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t b = smem_desc_sw128(vb + kk * (16 * 128), BN * 128, 1024);
+          tc_mma(tmem_o(x), a, b, idesc_o, (accumulate || kk > 0) ? 1u : 0u);
         }
+        tc_commit(o_done + x);
+        ++pv_it[x];
       };
       for (int w = blockIdx.x; w < num_work && ok; w += gridDim.x) {
         const Work wk = decode_work(w, tiles, info, p.num_q_heads, p.causal);
-        if (wk.n == 0) continue;
+        if (wk.nmax == 0) continue;
         ok = mbar_wait_bounded(q_full, tcount & 1, abort_flag, err);
         if (!ok) break;
         tc_fence_after();
-        {
-          const int st = kv_it % NS;
-          ok = mbar_wait_bounded(k_full + st, (kv_it / NS) & 1, abort_flag, err);
-          if (!ok) break;
-          tc_fence_after();
-          issue_s(s_it, st);
-          tc_commit(s_full + (s_it & 1));
-          tc_commit(k_empty + st);
-          if (wk.n == 1) tc_commit(q_empty);
-        }
-        for (int j = 0; j < wk.n && ok; ++j) {
-          const int cur = s_it + j;
-          if (j + 1 < wk.n) {
-            const int kvn = kv_it + j + 1, st = kvn % NS;
-            ok = mbar_wait_bounded(k_full + st, (kvn / NS) & 1, abort_flag, err);
+        const long long base = ld;  // K_j = base + 2j, V_j = base + 2j + 1
+        ok = wait_tile(base);
+        if (!ok) break;
+        tc_fence_after();
+        if (wk.n[0] > 0) issue_s(0, base);
+        if (wk.n[1] > 0) issue_s(1, base);
+        tc_commit(slot_empty + (int)(base % kRing));  // K_0 read by both S MMAs
+        if (wk.nmax == 1) tc_commit(q_empty);
+        for (int j = 0; j < wk.nmax && ok; ++j) {
+          const long long kn = base + 2 * (j + 1), vj = base + 2 * j + 1;
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            if (j >= wk.n[x]) continue;
+            ok = mbar_wait_bounded(p_full + x, pv_it[x] & 1, abort_flag, err);
+            if (ok) ok = wait_tile(vj);
             if (!ok) break;
             tc_fence_after();
-            issue_s(cur + 1, st);
-            tc_commit(s_full + ((cur + 1) & 1));
-            tc_commit(k_empty + st);
-            if (j + 2 == wk.n) tc_commit(q_empty);  // last S of the tile issued
+            issue_pv(x, vj, j > 0);
+            if (j + 1 < wk.n[x]) {
+              ok = wait_tile(kn);
+              if (!ok) break;
+              tc_fence_after();
+              issue_s(x, kn);
+            }
           }
-          ok = mbar_wait_bounded(p_full, cur & 1, abort_flag, err);
           if (!ok) break;
-          const int kvc = kv_it + j, st = kvc % NS;
-          ok = mbar_wait_bounded(v_full + st, (kvc / NS) & 1, abort_flag, err);
-          if (!ok) break;
-          tc_fence_after();
-          issue_o(st, j > 0);
-          tc_commit(o_done);
-          tc_commit(v_empty + st);
+          tc_commit(slot_empty + (int)(vj % kRing));            // V_j done
+          if (j + 1 < wk.nmax) tc_commit(slot_empty + (int)(kn % kRing));  // K_{j+1} done
+          if (j + 2 == wk.nmax) tc_commit(q_empty);             // last S MMAs issued
         }
-        kv_it += wk.n;
-        s_it += wk.n;
+        ld = base + 2 * wk.nmax;
         ++tcount;
       }
     }
   } else {
-    // ------------------------------ softmax warps -----------------------------
-    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    // ------------------------- softmax warps (tile x) --------------------------
+    const int x = (warp - 2) >> 2;  // 0: tile A (warps 2-5), 1: tile B (warps 6-9)
+    const int quarter = warp & 3;   // TMEM lanes this warp may access
     const int r = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    int s_it = 0;
+    const uint32_t s_col = tmem_s(x) + lane_base;
+    const uint32_t o_col = tmem_o(x) + lane_base;
+    const uint32_t p_tile = p_s + x * SM::kPBytes;
+    int it = 0;  // S tiles of this query tile consumed so far (phase counter)
     bool ok = true;
     for (int w = blockIdx.x; w < num_work && ok; w += gridDim.x) {
       const Work wk = decode_work(w, tiles, info, p.num_q_heads, p.causal);
-      const bool row_ok = r < wk.rows;
-      __nv_bfloat16* orow =
-          p.out + ((size_t)(wk.q_start + wk.row0 + r) * p.num_q_heads + wk.head) * D;
-      if (wk.n == 0) {
+      const int rows = wk.rows[x], n = wk.n[x];
+      const int qrow = wk.row0 + x * BM + r;  // query index within the sequence
+      const bool row_ok = r < rows;
+      if (n == 0) {
         if (row_ok) {
+          __nv_bfloat16* orow =
+              p.out + ((size_t)(wk.q_start + qrow) * p.num_q_heads + wk.head) * D;
 #pragma unroll
-          for (int c = 0; c < D / 8; ++c)
-            reinterpret_cast<uint4*>(orow)[c] = make_uint4(0, 0, 0, 0);
+          for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = make_uint4(0, 0, 0, 0);
         }
         continue;
       }
       // last key this row may see (inclusive); below 0 means none
       int limit = wk.kv_len - 1;
-      if (p.causal) limit = min(limit, wk.kv_len - wk.q_len + wk.row0 + r);
+      if (p.causal) limit = min(limit, wk.kv_len - wk.q_len + qrow);
       float m_use = -INFINITY, l = 0.f;
-      for (int j = 0; j < wk.n; ++j) {
-        const int cur = s_it + j;
-        ok = mbar_wait_bounded(s_full + (cur & 1), (cur >> 1) & 1, abort_flag, err);
+      for (int j = 0; j < n; ++j) {
+        const int cur = it + j;
+        // S_x(j) has landed.  P_x(j-1).V was issued before S_x(j) by the same
+        // thread, so waiting for it here (P buffer free, O stable) costs nothing
+        // and lets P be stored as it is computed.
+        ok = mbar_wait_bounded(s_full + x, cur & 1, abort_flag, err);
+        if (ok && cur > 0) ok = mbar_wait_bounded(o_done + x, (cur - 1) & 1, abort_flag, err);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        uint32_t sv[BN];
-        {
-          const uint32_t base = tmem_s0 + (cur & 1) * BN + lane_base;
-          tmem_ld32(base + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-          tmem_ld32(base + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-          tmem_ld32(base + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
-          tmem_ld32(base + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
-          tmem_ld_wait();
-        }
-        float s[BN];
+        // Pass 1: row max over the raw scores, 64 columns (two TMEM loads) at a
+        // time; masked keys count as -inf.  The scale is applied afterwards
+        // (scale_log2 > 0, so the max commutes with it) and in the exponent's
+        // FFMA.  Reductions use independent partials (short trees, not
+        // 128-long dependency chains).
         const int key0 = j * BN;
-        float m_tile = -INFINITY;
-        if (key0 + BN - 1 > limit) {
+        const bool masked_tile = key0 + BN - 1 > limit;
+        constexpr int NP = 4;
+        float mp[NP];
 #pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            const float v = __uint_as_float(sv[c]) * p.scale_log2;
-            s[c] = (key0 + c <= limit) ? v : -INFINITY;
-            m_tile = fmaxf(m_tile, s[c]);
-          }
-        } else {
+        for (int i = 0; i < NP; ++i) mp[i] = -INFINITY;
+        // Unmasked tiles take a loop with one FMNMX per score (FMNMX runs on
+        // the half-rate ALU pipe, so no per-score index or mask work there);
+        // only tiles crossing the diagonal or the sequence end test each key.
+        const int valid = limit - key0 + 1;  // keys [0, valid) of this tile are visible
 #pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            s[c] = __uint_as_float(sv[c]) * p.scale_log2;
-            m_tile = fmaxf(m_tile, s[c]);
+        for (int h = 0; h < BN; h += 64) {
+          uint32_t sv[64];
+          tmem_ld32(s_col + h, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+          tmem_ld32(s_col + h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+          tmem_ld_wait();
+          if (!masked_tile) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) mp[c % NP] = fmaxf(mp[c % NP], __uint_as_float(sv[c]));
+          } else {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              mp[c % NP] = fmaxf(mp[c % NP], h + c < valid ? __uint_as_float(sv[c]) : -INFINITY);
           }
         }
+#pragma unroll
+        for (int wdt = NP / 2; wdt >= 1; wdt >>= 1)
+#pragma unroll
+          for (int i = 0; i < wdt; ++i) mp[i] = fmaxf(mp[i], mp[i + wdt]);
+        const float m_tile = mp[0] * p.scale_log2;  // scale_log2 > 0: max commutes with it
         const float m_old = m_use;
-        const bool grow = m_tile > m_old + kRescaleThreshold || (m_old == -INFINITY && m_tile > -INFINITY);
+        const bool grow =
+            m_tile > m_old + kRescaleThreshold || (m_old == -INFINITY && m_tile > -INFINITY);
         if (grow) m_use = m_tile;
         const float base = (m_use == -INFINITY) ? 0.f : m_use;
         const bool rescale_o = grow && m_old != -INFINITY && j > 0;
         const float alpha = (grow && m_old != -INFINITY) ? fast_exp2(m_old - m_use) : 1.f;
-        float rowsum = 0.f;
-        uint32_t pk[BN / 2];
-#pragma unroll
-        for (int c = 0; c < BN; c += 2) {
-          const float p0 = fast_exp2(s[c] - base);
-          const float p1 = fast_exp2(s[c + 1] - base);
-          rowsum += p0 + p1;
-          pk[c / 2] = pack_bf16x2(p0, p1);
-        }
-        l = l * alpha + rowsum;
-
-        // P buffer free and O stable once the previous P.V has completed
-        if (cur > 0) {
-          ok = mbar_wait_bounded(o_done, (cur - 1) & 1, abort_flag, err);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          tc_fence_after();
-        }
         if (__any_sync(0xffffffffu, rescale_o)) {
           const float f = rescale_o ? alpha : 1.f;
 #pragma unroll
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t ov[32];
-            tmem_ld32(tmem_o + lane_base + c0, ov);
+            tmem_ld32(o_col + c0, ov);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
-            tmem_st32(tmem_o + lane_base + c0, ov);
+            tmem_st32(o_col + c0, ov);
           }
           tmem_st_wait();
         }
-        // P row -> swizzled K-major SMEM tile (A operand of O += P.V)
-        {
-          const uint32_t row_base = p_s + (r >> 3) * 1024 + (r & 7) * 128;
+        // p = 2^(scale_log2 * s - base), rounded to bf16 and stored chunk by
+        // chunk into the swizzled K-major P tile (A operand of O += P.V)
+        float rs[NP];
 #pragma unroll
-          for (int kc = 0; kc < BN / 8; ++kc) {
+        for (int i = 0; i < NP; ++i) rs[i] = 0.f;
+        const uint32_t row_base = p_tile + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+        for (int h = 0; h < BN; h += 64) {
+          // Pass 2: re-read 64 scores, exponentiate, round to bf16 and store
+          uint32_t sv[64];
+          tmem_ld32(s_col + h, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+          tmem_ld32(s_col + h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+          tmem_ld_wait();
+          if (masked_tile) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (h + c >= valid) sv[c] = __float_as_uint(-INFINITY);
+          }
+#pragma unroll
+          for (int kc = 0; kc < 8; ++kc) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = kc * 8 + 2 * e;
+              const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c]), p.scale_log2, -base));
+              const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), p.scale_log2, -base));
+              rs[e % NP] += p0 + p1;
+              pk[e] = pack_bf16x2(p0, p1);
+            }
+            const int chunk = h / 8 + kc;  // 16-byte chunk (8 keys) within the row
             const uint32_t addr =
-                row_base + (kc >> 3) * (BM * 128) + (((kc & 7) ^ (r & 7)) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                         "r"(pk[kc * 4 + 0]), "r"(pk[kc * 4 + 1]), "r"(pk[kc * 4 + 2]),
-                         "r"(pk[kc * 4 + 3])
+                row_base + (chunk >> 3) * (BM * 128) + (((chunk & 7) ^ (r & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[0]),
+                         "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
                          : "memory");
           }
         }
+#pragma unroll
+        for (int wdt = NP / 2; wdt >= 1; wdt >>= 1)
+#pragma unroll
+          for (int i = 0; i < wdt; ++i) rs[i] += rs[i + wdt];
+        l = l * alpha + rs[0];
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(p_full);
+        mbar_arrive(p_full + x);
       }
       if (!ok) break;
       // epilogue: O / l -> bf16 -> global
-      const int last = s_it + wk.n - 1;
-      ok = mbar_wait_bounded(o_done, last & 1, abort_flag, err);
+      const int last = it + n - 1;
+      ok = mbar_wait_bounded(o_done + x, last & 1, abort_flag, err);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* orow = p.out + ((size_t)(wk.q_start + qrow) * p.num_q_heads + wk.head) * D;
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t ov[32];
-        tmem_ld32(tmem_o + lane_base + c0, ov);
+        tmem_ld32(o_col + c0, ov);
         tmem_ld_wait();
         if (row_ok) {
 #pragma unroll
@@ -416,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      s_it += wk.n;
+      it += n;
     }
   }
 
@@ -433,23 +486,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int NS>
+template <int D>
 static cudaError_t launch_prefill_t(const PrefillParams& p, const CUtensorMap& q_map,
                                     const CUtensorMap& k_map, const CUtensorMap& v_map, int grid,
                                     cudaStream_t stream) {
-  using SM = PrefillSmem<D, NS>;
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, NS>,
+  using SM = PrefillSmem<D>;
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc);
   if (e != cudaSuccess) return e;
-  prefill_kernel<D, NS><<<grid, kThreads, SM::kAlloc, stream>>>(p, q_map, k_map, v_map);
+  prefill_kernel<D><<<grid, kThreads, SM::kAlloc, stream>>>(p, q_map, k_map, v_map);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& q_map,
                            const CUtensorMap& k_map, const CUtensorMap& v_map, int head_dim,
                            int grid, cudaStream_t stream) {
-  if (head_dim == 128) return launch_prefill_t<128, 2>(p, q_map, k_map, v_map, grid, stream);
-  return launch_prefill_t<64, 4>(p, q_map, k_map, v_map, grid, stream);
+  if (head_dim == 128) return launch_prefill_t<128>(p, q_map, k_map, v_map, grid, stream);
+  return launch_prefill_t<64>(p, q_map, k_map, v_map, grid, stream);
 }
 
 }  // namespace pa
