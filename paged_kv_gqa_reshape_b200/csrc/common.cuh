@@ -37,8 +37,69 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // 2^x on the SFU (ex2.approx, flush-to-zero): a hardware instruction.
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
-  asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// ---------------------------------------------------------------------------
+// packed fp32 pairs (one instruction on two lanes of a 64-bit register pair)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  return ((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// max(a, b, c) in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Coefficients of the degree-3 polynomial q(f) that minimises
+// max |q(f) / 2^f - 1| over f in [-1/2, 1/2] (solved as a linear program on a
+// 4001-point grid); the maximum relative error is 7.5e-5, below half an ulp
+// of bf16 (2^-9), the precision the probabilities are rounded to.
+constexpr float kExp2PolyC0 = 0.99992806f;
+constexpr float kExp2PolyC1 = 0.69326097f;
+constexpr float kExp2PolyC2 = 0.24261113f;
+constexpr float kExp2PolyC3 = 0.05517167f;
+
+// 2^x for a pair of arguments on the FMA pipe instead of the SFU, so that
+// both units share the exponentials of a softmax tile.  Range reduction:
+// x = n + f with n = rint(x) and |f| <= 1/2; 2^f from the polynomial above;
+// 2^n built directly as a float by shifting the biased exponent 127 + n into
+// place.  Adding 1.5 * 2^23 + 127 to x leaves 127 + n in the low mantissa bits
+// (round to nearest), so one shift of those bits gives 2^n; x is clamped to
+// -127 first, where the biased exponent 0 makes 2^n exactly +0, so -inf (a
+// masked score) yields exactly 0.  Valid for x < 128.
+__device__ __forceinline__ uint64_t exp2_poly_pair(float x0, float x1) {
+  constexpr float kShift = 12583039.0f;  // 1.5 * 2^23 + 127
+  const uint64_t x = f2_pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+  const uint64_t t = f2_add(x, f2_pack(kShift, kShift));
+  const uint64_t n = f2_add(t, f2_pack(-kShift, -kShift));  // rint(x)
+  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x);
+  uint64_t q = f2_fma(f2_pack(kExp2PolyC3, kExp2PolyC3), f, f2_pack(kExp2PolyC2, kExp2PolyC2));
+  q = f2_fma(q, f, f2_pack(kExp2PolyC1, kExp2PolyC1));
+  q = f2_fma(q, f, f2_pack(kExp2PolyC0, kExp2PolyC0));
+  const uint32_t e_lo = (uint32_t)t << 23, e_hi = (uint32_t)(t >> 32) << 23;
+  const uint64_t two_n = ((uint64_t)e_hi << 32) | e_lo;
+  return f2_mul(q, two_n);
 }
 
 // ---------------------------------------------------------------------------
@@ -234,6 +295,17 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16; A (K-major, M rows in the
+// TMEM lanes, two 16-bit elements per 32-bit column) is read from TMEM.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // 32 consecutive 32-bit columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile(
@@ -257,6 +329,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
       "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
       "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
       "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
       : "memory");
 }
 __device__ __forceinline__ void tmem_ld_wait() {

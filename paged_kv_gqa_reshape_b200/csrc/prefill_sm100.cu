@@ -17,23 +17,26 @@
 //    through the block table with a 4-D map over [blocks, 16, Hkv, D]
 //    (a page past the sequence end, or a bad block id, is fetched at an
 //    out-of-range coordinate, i.e. as zeros).  128-byte swizzle, no
-//    multicast.  K and V tiles go through one 3-slot ring in the order
-//    K0 V0 K1 V1 ...;
+//    multicast.  K and V tiles go through one ring (5 slots for D = 128,
+//    10 for D = 64) in the order K0 V0 K1 V1 ...;
 //  * warp 1 (one lane): tcgen05.mma issuer.  Per KV tile j it issues
 //    PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): S = Q.K^T into the tile's TMEM
 //    S buffer (M = 128, N = 128, K = 16 per instruction) and O += P.V into
-//    the tile's TMEM accumulator (B = V read MN-major straight from the TMA
-//    layout).  While one tile's softmax runs, the tensor core works on the
-//    other tile; completion is reported through tcgen05.commit -> mbarrier;
+//    the tile's TMEM accumulator, with A = P read from TMEM and B = V read
+//    MN-major straight from the TMA layout.  S_x(j+1) overwrites the columns
+//    that hold P_x(j), so it is issued once P_x(j).V has completed.  While one
+//    tile's softmax runs, the tensor core works on the other tile;
+//    completion is reported through tcgen05.commit -> mbarrier;
 //  * warps 2-5 / 6-9: softmax of tile A / B, one thread per query row
-//    (= TMEM lane).  tcgen05.ld of the S row, mask only on tiles that cross
-//    the diagonal or the sequence end, online softmax in fp32 (scale folded
-//    into the exponent's FFMA, tree reductions) with lazy rescaling (O in
-//    TMEM is rescaled only when the running max grows by more than 2^8),
-//    P rounded to bf16 into the tile's swizzled SMEM buffer, the A operand of
-//    the P.V MMA; final O / l -> bf16 -> global.
-// TMEM: S_A, S_B, O_A, O_B (4 x 128 columns for D = 128).
-// SMEM: Q_A, Q_B, the 3-slot K/V ring and P_A, P_B (224 KB for D = 128).
+//    (= TMEM lane).  The 128 scores of the row come into registers once,
+//    the mask is applied only on tiles that cross the diagonal or the
+//    sequence end, online softmax in fp32 (3-input max, scale folded into a
+//    packed-pair FFMA, packed row sums) with lazy rescaling (O in TMEM is
+//    rescaled only when the running max grows by more than 2^8), P rounded
+//    to bf16 and written back over the first 64 columns of S (two keys per
+//    column), the A operand of the P.V MMA; final O / l -> bf16 -> global.
+// TMEM: S_A, S_B, O_A, O_B (4 x 128 columns for D = 128); P_x inside S_x.
+// SMEM: Q_A, Q_B and the K/V ring (224 KB for D = 128).
 // Every mbarrier wait is bounded in time; a CTA that gives up raises
 // PA_DEVERR_TIMEOUT, lets in-flight copies land, frees its TMEM and exits.
 #include <math.h>
@@ -46,11 +49,11 @@ namespace pa {
 
 namespace {
 
+constexpr int kPolyPairs = 0;  // of every 16 exponent pairs, computed on the FMA pipe
 constexpr int kWarps = 10;  // 0 producer, 1 MMA, 2-5 softmax A, 6-9 softmax B
 constexpr int kThreads = kWarps * 32;
 constexpr int BM = kPrefillTileM;
 constexpr int BN = kPrefillTileN;
-constexpr int kRing = 3;  // K/V slots
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows by > 2^8
 
@@ -58,11 +61,10 @@ template <int D>
 struct PrefillSmem {
   static constexpr int kQBytes = BM * D * 2;   // one 128-row Q tile
   static constexpr int kKVBytes = BN * D * 2;  // one K or V tile
-  static constexpr int kPBytes = BM * BN * 2;  // one P tile
+  static constexpr int kRing = D == 128 ? 5 : 10;  // K/V slots (~160 KB)
   static constexpr int kQOff = 0;              // Q_A, Q_B
   static constexpr int kRingOff = kQOff + 2 * kQBytes;
-  static constexpr int kPOff = kRingOff + kRing * kKVBytes;  // P_A, P_B
-  static constexpr int kBarOff = kPOff + 2 * kPBytes;
+  static constexpr int kBarOff = kRingOff + kRing * kKVBytes;
   // barriers: q_full, q_empty, slot_full[kRing], slot_empty[kRing], s_full[2],
   //           p_full[2], o_done[2]
   static constexpr int kNumBars = 2 + 2 * kRing + 6;
@@ -112,6 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap k_map,
                    const __grid_constant__ CUtensorMap v_map) {
   using SM = PrefillSmem<D>;
+  constexpr int kRing = SM::kRing;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -132,7 +135,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const uint32_t q_s = smem_u32(smem + SM::kQOff);
   const uint32_t ring_s = smem_u32(smem + SM::kRingOff);
-  const uint32_t p_s = smem_u32(smem + SM::kPOff);
 
   unsigned char* ws = p.ws;
   uint32_t* err = reinterpret_cast<uint32_t*>(ws + p.L.err);
@@ -164,7 +166,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // S_A, S_B: columns [0, 128), [128, 256); O_A, O_B: [256, 256 + D), [256 + D, 256 + 2D)
+  // S_A, S_B: columns [0, 128), [128, 256); O_A, O_B: [256, 256 + D), [256 + D, 256 + 2D).
+  // P_x (bf16, two keys per 32-bit column) overwrites the first 64 columns of
+  // S_x once the softmax holds those scores in registers.
   auto tmem_s = [&](int x) { return tmem + (uint32_t)(x * BN); };
   auto tmem_o = [&](int x) { return tmem + (uint32_t)(2 * BN + x * D); };
 
@@ -252,12 +256,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto issue_pv = [&](int x, long long vidx, bool accumulate) {
         const uint32_t vb = ring_s + (int)(vidx % kRing) * SM::kKVBytes;
-        const uint32_t pb = p_s + x * SM::kPBytes;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t a = smem_desc_sw128(pb + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024);
+          // A = P from TMEM: keys 16kk..16kk+15 are columns 8kk..8kk+7 of P_x
           const uint64_t b = smem_desc_sw128(vb + kk * (16 * 128), BN * 128, 1024);
-          tc_mma(tmem_o(x), a, b, idesc_o, (accumulate || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tmem_o(x), tmem_s(x) + 8 * kk, b, idesc_o, (accumulate || kk > 0) ? 1u : 0u);
         }
         tc_commit(o_done + x);
         ++pv_it[x];
@@ -287,7 +290,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             issue_pv(x, vj, j > 0);
             if (j + 1 < wk.n[x]) {
-              ok = wait_tile(kn);
+              // S_x(j+1) overwrites the columns P_x(j) occupies: let P_x(j).V finish
+              ok = mbar_wait_bounded(o_done + x, (pv_it[x] - 1) & 1, abort_flag, err);
+              if (ok) ok = wait_tile(kn);
               if (!ok) break;
               tc_fence_after();
               issue_s(x, kn);
@@ -310,7 +315,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t s_col = tmem_s(x) + lane_base;
     const uint32_t o_col = tmem_o(x) + lane_base;
-    const uint32_t p_tile = p_s + x * SM::kPBytes;
     int it = 0;  // S tiles of this query tile consumed so far (phase counter)
     bool ok = true;
     for (int w = blockIdx.x; w < num_work && ok; w += gridDim.x) {
@@ -341,36 +345,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        // Pass 1: row max over the raw scores, 64 columns (two TMEM loads) at a
-        // time; masked keys count as -inf.  The scale is applied afterwards
-        // (scale_log2 > 0, so the max commutes with it) and in the exponent's
-        // FFMA.  Reductions use independent partials (short trees, not
-        // 128-long dependency chains).
+        // The row's 128 raw scores come into registers with four TMEM loads and
+        // one wait; the max and the exponentials both work from those registers.
+        // The scale is applied after the max (scale_log2 > 0, so the max
+        // commutes with it) and in the exponent's FFMA.  Reductions use
+        // independent partials (short trees, not 128-long dependency chains).
         const int key0 = j * BN;
         const bool masked_tile = key0 + BN - 1 > limit;
+        const int valid = limit - key0 + 1;  // keys [0, valid) of this tile are visible
+        uint32_t sv[BN];
+#pragma unroll
+        for (int c = 0; c < BN; c += 32)
+          tmem_ld32(s_col + c, *reinterpret_cast<uint32_t(*)[32]>(&sv[c]));
+        tmem_ld_wait();
+        // Tiles crossing the diagonal or the sequence end set hidden keys to
+        // -inf once; the others skip every per-key test.
+        if (masked_tile) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (c >= valid) sv[c] = __float_as_uint(-INFINITY);
+        }
         constexpr int NP = 4;
         float mp[NP];
 #pragma unroll
         for (int i = 0; i < NP; ++i) mp[i] = -INFINITY;
-        // Unmasked tiles take a loop with one FMNMX per score (FMNMX runs on
-        // the half-rate ALU pipe, so no per-score index or mask work there);
-        // only tiles crossing the diagonal or the sequence end test each key.
-        const int valid = limit - key0 + 1;  // keys [0, valid) of this tile are visible
 #pragma unroll
-        for (int h = 0; h < BN; h += 64) {
-          uint32_t sv[64];
-          tmem_ld32(s_col + h, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-          tmem_ld32(s_col + h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-          tmem_ld_wait();
-          if (!masked_tile) {
-#pragma unroll
-            for (int c = 0; c < 64; ++c) mp[c % NP] = fmaxf(mp[c % NP], __uint_as_float(sv[c]));
-          } else {
-#pragma unroll
-            for (int c = 0; c < 64; ++c)
-              mp[c % NP] = fmaxf(mp[c % NP], h + c < valid ? __uint_as_float(sv[c]) : -INFINITY);
-          }
-        }
+        for (int c = 0; c < BN; c += 2)
+          mp[(c / 2) % NP] = fmax3(mp[(c / 2) % NP], __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
 #pragma unroll
         for (int wdt = NP / 2; wdt >= 1; wdt >>= 1)
 #pragma unroll
@@ -383,6 +384,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float base = (m_use == -INFINITY) ? 0.f : m_use;
         const bool rescale_o = grow && m_old != -INFINITY && j > 0;
         const float alpha = (grow && m_old != -INFINITY) ? fast_exp2(m_old - m_use) : 1.f;
+        // p = 2^(scale_log2 * s - base), rounded to bf16 and written to TMEM as
+        // the A operand of O += P.V.  kPolyPairs of every 16 pairs take the
+        // polynomial 2^x on the FMA pipe, the rest the SFU: the SFU alone would
+        // bound this loop.  Scaling and row sums run on packed fp32 pairs.
+        const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t nbase2 = f2_pack(-base, -base);
+        uint64_t rs2[NP / 2];
+#pragma unroll
+        for (int i = 0; i < NP / 2; ++i) rs2[i] = 0;
+#pragma unroll
+        for (int h = 0; h < BN; h += 32) {
+          // 32 scores -> 16 packed bf16 pairs over S columns [h/2, h/2 + 16),
+          // whose scores are already in registers
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c = h + 2 * e;
+            const uint64_t xx = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
+                                       scale2, nbase2);
+            uint64_t pp;
+            if ((c / 2) % 16 < kPolyPairs)
+              pp = exp2_poly_pair(f2_lo(xx), f2_hi(xx));
+            else
+              pp = f2_pack(fast_exp2(f2_lo(xx)), fast_exp2(f2_hi(xx)));
+            rs2[e % (NP / 2)] = f2_add(rs2[e % (NP / 2)], pp);
+            pk[e] = pack_bf16x2(f2_lo(pp), f2_hi(pp));
+          }
+          tmem_st16(s_col + h / 2, pk);
+        }
+#pragma unroll
+        for (int i = 1; i < NP / 2; ++i) rs2[0] = f2_add(rs2[0], rs2[i]);
+        float rs[1] = {f2_lo(rs2[0]) + f2_hi(rs2[0])};
+        l = l * alpha + rs[0];
+        // O *= alpha where the running max moved (rare: lazy threshold); done
+        // after P so the scores' registers are free.  PV(j-1) has completed.
         if (__any_sync(0xffffffffu, rescale_o)) {
           const float f = rescale_o ? alpha : 1.f;
 #pragma unroll
@@ -394,51 +430,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
             tmem_st32(o_col + c0, ov);
           }
-          tmem_st_wait();
         }
-        // p = 2^(scale_log2 * s - base), rounded to bf16 and stored chunk by
-        // chunk into the swizzled K-major P tile (A operand of O += P.V)
-        float rs[NP];
-#pragma unroll
-        for (int i = 0; i < NP; ++i) rs[i] = 0.f;
-        const uint32_t row_base = p_tile + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-        for (int h = 0; h < BN; h += 64) {
-          // Pass 2: re-read 64 scores, exponentiate, round to bf16 and store
-          uint32_t sv[64];
-          tmem_ld32(s_col + h, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-          tmem_ld32(s_col + h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-          tmem_ld_wait();
-          if (masked_tile) {
-#pragma unroll
-            for (int c = 0; c < 64; ++c)
-              if (h + c >= valid) sv[c] = __float_as_uint(-INFINITY);
-          }
-#pragma unroll
-          for (int kc = 0; kc < 8; ++kc) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = kc * 8 + 2 * e;
-              const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c]), p.scale_log2, -base));
-              const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), p.scale_log2, -base));
-              rs[e % NP] += p0 + p1;
-              pk[e] = pack_bf16x2(p0, p1);
-            }
-            const int chunk = h / 8 + kc;  // 16-byte chunk (8 keys) within the row
-            const uint32_t addr =
-                row_base + (chunk >> 3) * (BM * 128) + (((chunk & 7) ^ (r & 7)) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[0]),
-                         "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
-                         : "memory");
-          }
-        }
-#pragma unroll
-        for (int wdt = NP / 2; wdt >= 1; wdt >>= 1)
-#pragma unroll
-          for (int i = 0; i < wdt; ++i) rs[i] += rs[i + wdt];
-        l = l * alpha + rs[0];
-        fence_proxy_async_smem();
+        tmem_st_wait();
         tc_fence_before();
         mbar_arrive(p_full + x);
       }
