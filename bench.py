@@ -14,6 +14,7 @@ oracle on a bounded sample of the same workload instead.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -35,6 +36,38 @@ METRIC = "paged-attn decode HBM GB/s + prefill TFLOP/s (fraction of B200 rooflin
 WORKLOAD = ("decode_batch: 64 seqs x 1 query token, context U[256,4096], Hq 32 / Hkv 8, "
             "head_dim 128, block 16, bf16, shuffled block tables; step = scatter of the 64 new "
             "K/V rows + split-KV decode attention")
+
+
+# DRAM bytes (read + write) of one decode-kernel launch on the decode batch, from
+# one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), valid only
+# while the decode kernel's sources hash to the recorded value.
+DECODE_TRAFFIC = {"sources_sha256": "8246a080b29f8dacef4a7ed3a166f6fbcd884297e7584ca3ff34dedea2abbd42",
+                  "bytes_per_launch": 604642304}
+DECODE_SOURCES = ("decode.cu", "common.cuh", "layout.h")
+
+
+def decode_sources_sha() -> str:
+    h = hashlib.sha256()
+    for n in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "paged_kv_gqa_reshape_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic():
+    if DECODE_TRAFFIC["sources_sha256"] and DECODE_TRAFFIC["sources_sha256"] == decode_sources_sha():
+        return DECODE_TRAFFIC["bytes_per_launch"]
+    return None
+
+
+def launches_per_step(case) -> int:
+    """Kernels the step launches: write_kv, the plan (only when the batch has a
+    multi-token query or more sequences than the decode kernel plans for
+    itself), the prefill kernel if there is a multi-token query, and the
+    decode kernel (always)."""
+    prefill = case.max_query_len > 1
+    plan = prefill or case.num_seqs > 1024
+    return 1 + int(plan) + int(prefill) + 1
 
 
 # ---------------------------------------------------------------------------
@@ -199,14 +232,14 @@ def time_varlen_component(pa, case, iters=20, warmup=3, with_scatter=False):
     ws = pa.varlen_workspace(case.num_seqs, case.num_q_tokens, case.num_q_heads,
                              case.num_kv_heads, case.head_dim)
     out = torch.empty_like(case.q)
+    mql, msl = case.max_query_len, case.max_seq_len
 
     def run():
         if with_scatter:
             pa.write_kv(case.k_new, case.v_new, case.slot_mapping, case.k_cache, case.v_cache)
         pa.attention_varlen(case.q, case.k_cache, case.v_cache, case.block_tables, case.seq_lens,
                             case.query_start_loc, case.num_kv_heads, case.scale, case.causal, out,
-                            max_query_len=case.max_query_len, max_seq_len=case.max_seq_len,
-                            workspace=ws)
+                            max_query_len=mql, max_seq_len=msl, workspace=ws)
 
     if not with_scatter:
         pa.write_kv(case.k_new, case.v_new, case.slot_mapping, case.k_cache, case.v_cache)
@@ -350,11 +383,12 @@ def run_ours(args, rank, world, local_rank):
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                      "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
-                     "traffic": args.traffic,
-                     "kernel": "pa_attention_varlen (plan + split-KV decode), per-call events",
+                     "traffic": args.traffic if args.traffic is not None else recorded_traffic(),
+                     "kernel": "decode_kernel (split-KV decode; the call launches only it), "
+                               "CUDA events around each call",
                      "peak_kind": peak_kind},
         "clocks": clk,
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": launches_per_step(case) * args.steps,
     }
     return result, case
 
@@ -386,15 +420,16 @@ def run_single_workload(args):
         ws = pa.varlen_workspace(case.num_seqs, case.num_q_tokens, case.num_q_heads,
                                  case.num_kv_heads, case.head_dim, device=dev)
         out = torch.empty_like(case.q)
+        mql, msl = case.max_query_len, case.max_seq_len
 
         def step():
             pa.write_kv(case.k_new, case.v_new, case.slot_mapping, case.k_cache, case.v_cache,
                         workspace=ws)
             pa.attention_varlen(case.q, case.k_cache, case.v_cache, case.block_tables,
                                 case.seq_lens, case.query_start_loc, case.num_kv_heads,
-                                case.scale, case.causal, out, max_query_len=case.max_query_len,
-                                max_seq_len=case.max_seq_len, workspace=ws)
-        if case.max_query_len > 1:
+                                case.scale, case.causal, out, max_query_len=mql,
+                                max_seq_len=msl, workspace=ws)
+        if mql > 1:
             work, unit, scale_div, peak = attention_flops(case), "TFLOP/s", 1e12, tc_peak
         else:
             work = scatter_bytes(case) + attention_bytes(case)
@@ -425,6 +460,7 @@ def run_e2e(pa, case, args, dev, ws):
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_h.numel() * out_h.element_size()
     steps = max(1, min(args.steps, 500))
+    mql, msl = case.max_query_len, case.max_seq_len  # host-side metadata, known before the step
 
     def step():
         for n in names:
@@ -433,8 +469,8 @@ def run_e2e(pa, case, args, dev, ws):
                     case.v_cache, workspace=ws)
         pa.attention_varlen(devt["q"], case.k_cache, case.v_cache, devt["block_tables"],
                             devt["seq_lens"], devt["query_start_loc"], case.num_kv_heads,
-                            case.scale, case.causal, out_d, max_query_len=case.max_query_len,
-                            max_seq_len=case.max_seq_len, workspace=ws)
+                            case.scale, case.causal, out_d, max_query_len=mql,
+                            max_seq_len=msl, workspace=ws)
         out_h.copy_(out_d, non_blocking=True)
 
     for _ in range(3):
@@ -481,7 +517,7 @@ def cpu_baseline(budget_s=12.0):
     nbytes = scatter_bytes(case) + attention_bytes(case)
     times = []
     t_begin = time.perf_counter()
-    while not times or (time.perf_counter() - t_begin < budget_s and len(times) < 20):
+    while not times or (time.perf_counter() - t_begin < budget_s and len(times) < 500):
         times.append(time_oracle_step(case))
     gbs = nbytes * len(times) / sum(times) / 1e9
     return {"value": round(gbs, 4), "unit": "GB/s", "cores": oracle.num_threads(),
