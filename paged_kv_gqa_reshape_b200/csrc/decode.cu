@@ -406,39 +406,124 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
       if (lane == 0) old = atomicAdd(&counters[(size_t)seq * Hkv + kvh], 1);
       old = __shfl_sync(FULL, old, 0);
       if (old == n_chunks - 1) {
-        // last chunk of this (sequence, KV head) to finish: merge all of them
+        // last chunk of this (sequence, KV head) to finish: merge all of them.
+        // out = sum_c 2^(lse_c - M) O_c / sum_c 2^(lse_c - M), M = max_c lse_c.
+        // Loads are issued in batches so that a merge costs a few dependent
+        // global round trips rather than two per chunk and head.
         __threadfence();
         const int pb0 = pair_base;
-        for (int hl = 0; hl < g; ++hl) {
-          const int head = head0 + hl;
-          float M = -INFINITY;
-          for (int c = lane; c < n_chunks; c += 32)
-            M = fmaxf(M, __ldcg(lse_buf + (size_t)(pb0 + c) * p.num_q_heads + head));
+        const int nhc = g * n_chunks;  // (head, chunk) pairs, head-major
+        constexpr int kFast = 24;
+        if (nhc <= kFast) {
+          // One round of loads: lane i holds pair i's log-sum-exp, and every
+          // lane this lane's 4 d-values of every pair's partial.
+          float lse_mine = -INFINITY;
+          if (lane < nhc)
+            lse_mine = __ldcg(lse_buf + (size_t)(pb0 + lane % n_chunks) * p.num_q_heads + head0 +
+                              lane / n_chunks);
+          float4 xv[kFast];
 #pragma unroll
-          for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, o2));
-          if (lane * 4 < D) {
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            float wsum = 0.f;
-            if (M != -INFINITY) {
-              for (int c = 0; c < n_chunks; ++c) {
-                const float lc = __ldcg(lse_buf + (size_t)(pb0 + c) * p.num_q_heads + head);
-                const float w = (lc == -INFINITY) ? 0.f : fast_exp2(lc - M);
-                wsum += w;
-                const float4 x = __ldcg(reinterpret_cast<const float4*>(
-                    part_buf + ((size_t)(pb0 + c) * p.num_q_heads + head) * D + lane * 4));
-                acc.x += w * x.x;
-                acc.y += w * x.y;
-                acc.z += w * x.z;
-                acc.w += w * x.w;
+          for (int i = 0; i < kFast; ++i) {
+            xv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i < nhc && lane * 4 < D)
+              xv[i] = __ldcg(reinterpret_cast<const float4*>(
+                  part_buf + ((size_t)(pb0 + i % n_chunks) * p.num_q_heads + head0 + i / n_chunks) * D +
+                  lane * 4));
+          }
+          // per-head max and weight sum over the head's lanes [h*nc, h*nc + nc)
+          const int seg0 = (lane / n_chunks) * n_chunks;
+          float M = -INFINITY;
+          for (int j = 0; j < n_chunks; ++j)
+            M = fmaxf(M, __shfl_sync(FULL, lse_mine, (seg0 + j) & 31));
+          const float w_mine =
+              (lane < nhc && lse_mine != -INFINITY && M != -INFINITY) ? fast_exp2(lse_mine - M) : 0.f;
+          float wsum = 0.f;
+          for (int j = 0; j < n_chunks; ++j) wsum += __shfl_sync(FULL, w_mine, (seg0 + j) & 31);
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int i = 0; i < kFast; ++i) {
+            if (i < nhc) {
+              const float w = __shfl_sync(FULL, w_mine, i);
+              const float ws = __shfl_sync(FULL, wsum, i);
+              acc.x += w * xv[i].x;
+              acc.y += w * xv[i].y;
+              acc.z += w * xv[i].z;
+              acc.w += w * xv[i].w;
+              if (i % n_chunks == n_chunks - 1) {  // the head's last chunk: write it
+                if (lane * 4 < D) {
+                  const float inv = ws > 0.f ? 1.f / ws : 0.f;
+                  uint2 v;
+                  v.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+                  v.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+                  *reinterpret_cast<uint2*>(
+                      p.out + ((size_t)seg_q * p.num_q_heads + head0 + i / n_chunks) * D + lane * 4) = v;
+                }
+                acc = make_float4(0.f, 0.f, 0.f, 0.f);
               }
             }
+          }
+        } else {
+        // larger merges: per head, loads batched four chunks at a time
+        const bool one_pass = g * n_chunks <= 32;
+        float lse_mine = -INFINITY;
+        if (one_pass && lane < g * n_chunks)
+          lse_mine = __ldcg(lse_buf + (size_t)(pb0 + lane % n_chunks) * p.num_q_heads + head0 +
+                            lane / n_chunks);
+        for (int hl = 0; hl < g; ++hl) {
+          const int head = head0 + hl;
+          // lane c (c < n_chunks, per pass of 32) holds chunk c's weight
+          float M = -INFINITY;
+          for (int c0 = 0; c0 < n_chunks; c0 += 32) {
+            const float lc = one_pass ? __shfl_sync(FULL, lse_mine, (hl * n_chunks + lane) & 31)
+                             : (c0 + lane < n_chunks
+                                    ? __ldcg(lse_buf + (size_t)(pb0 + c0 + lane) * p.num_q_heads + head)
+                                    : -INFINITY);
+            M = fmaxf(M, lane < n_chunks - c0 ? lc : -INFINITY);
+          }
+#pragma unroll
+          for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, o2));
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          float wsum = 0.f;
+          if (M != -INFINITY) {
+            for (int c0 = 0; c0 < n_chunks; c0 += 32) {
+              float lc = one_pass ? __shfl_sync(FULL, lse_mine, (hl * n_chunks + lane) & 31)
+                         : (c0 + lane < n_chunks
+                                ? __ldcg(lse_buf + (size_t)(pb0 + c0 + lane) * p.num_q_heads + head)
+                                : -INFINITY);
+              if (lane >= n_chunks - c0) lc = -INFINITY;
+              const float w_mine = (lc == -INFINITY) ? 0.f : fast_exp2(lc - M);
+              const int nc = min(32, n_chunks - c0);
+              for (int cb = 0; cb < nc; cb += 4) {
+                float4 xv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  xv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                  if (cb + u < nc && lane * 4 < D)
+                    xv[u] = __ldcg(reinterpret_cast<const float4*>(
+                        part_buf + ((size_t)(pb0 + c0 + cb + u) * p.num_q_heads + head) * D + lane * 4));
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  const float w = __shfl_sync(FULL, w_mine, (cb + u) & 31);
+                  if (cb + u < nc) {
+                    wsum += w;
+                    acc.x += w * xv[u].x;
+                    acc.y += w * xv[u].y;
+                    acc.z += w * xv[u].z;
+                    acc.w += w * xv[u].w;
+                  }
+                }
+              }
+            }
+          }
+          if (lane * 4 < D) {
             const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
             uint2 v;
             v.x = pack_bf16x2(acc.x * inv, acc.y * inv);
             v.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-            *reinterpret_cast<uint2*>(p.out + ((size_t)seg_q * p.num_q_heads + head) * D +
-                                      lane * 4) = v;
+            *reinterpret_cast<uint2*>(p.out + ((size_t)seg_q * p.num_q_heads + head) * D + lane * 4) = v;
           }
+        }
         }
         if (lane == 0) counters[(size_t)seq * Hkv + kvh] = 0;  // ready for the next call
       }
