@@ -71,37 +71,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// Coefficients of the degree-3 polynomial q(f) that minimises
-// max |q(f) / 2^f - 1| over f in [-1/2, 1/2] (solved as a linear program on a
-// 4001-point grid); the maximum relative error is 7.5e-5, below half an ulp
-// of bf16 (2^-9), the precision the probabilities are rounded to.
-constexpr float kExp2PolyC0 = 0.99992806f;
-constexpr float kExp2PolyC1 = 0.69326097f;
-constexpr float kExp2PolyC2 = 0.24261113f;
-constexpr float kExp2PolyC3 = 0.05517167f;
-
-// 2^x for a pair of arguments on the FMA pipe instead of the SFU, so that
-// both units share the exponentials of a softmax tile.  Range reduction:
-// x = n + f with n = rint(x) and |f| <= 1/2; 2^f from the polynomial above;
-// 2^n built directly as a float by shifting the biased exponent 127 + n into
-// place.  Adding 1.5 * 2^23 + 127 to x leaves 127 + n in the low mantissa bits
-// (round to nearest), so one shift of those bits gives 2^n; x is clamped to
-// -127 first, where the biased exponent 0 makes 2^n exactly +0, so -inf (a
-// masked score) yields exactly 0.  Valid for x < 128.
-__device__ __forceinline__ uint64_t exp2_poly_pair(float x0, float x1) {
-  constexpr float kShift = 12583039.0f;  // 1.5 * 2^23 + 127
-  const uint64_t x = f2_pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
-  const uint64_t t = f2_add(x, f2_pack(kShift, kShift));
-  const uint64_t n = f2_add(t, f2_pack(-kShift, -kShift));  // rint(x)
-  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x);
-  uint64_t q = f2_fma(f2_pack(kExp2PolyC3, kExp2PolyC3), f, f2_pack(kExp2PolyC2, kExp2PolyC2));
-  q = f2_fma(q, f, f2_pack(kExp2PolyC1, kExp2PolyC1));
-  q = f2_fma(q, f, f2_pack(kExp2PolyC0, kExp2PolyC0));
-  const uint32_t e_lo = (uint32_t)t << 23, e_hi = (uint32_t)(t >> 32) << 23;
-  const uint64_t two_n = ((uint64_t)e_hi << 32) | e_lo;
-  return f2_mul(q, two_n);
-}
-
 // ---------------------------------------------------------------------------
 // shared-memory addresses
 // ---------------------------------------------------------------------------
