@@ -10,10 +10,13 @@
 // key blocks, and no time goes to retiring and launching short-lived CTAs.
 // Each item's K and V rows (16-byte loads, up to 16 keys) are all issued
 // before any arithmetic, and the next item's cu_seqlens bounds are loaded
-// while the current item computes.  Passes past the entry's key count are
-// skipped (warp-uniform), so a 2-key entry costs 2 keys of math, not 16.
-// (Holding a second item's rows in registers instead halves the resident
-// warps and measured at half the bandwidth.)
+// while the current item computes.  The math runs over the smallest power of
+// two of key passes covering the entry, as straight-line code, so the shuffle
+// trees of all passes overlap (a branch per pass serialised them: 76 % -> 85 %
+// of the copy bandwidth).  (Holding a second item's rows in registers instead
+// halves the resident warps and measured at half the bandwidth; staging whole
+// entries through a shared-memory ring with bulk copies left the per-entry
+// math of 16 warps per SM as the bound.)
 //
 // Within an item a key row of head_dim bf16 is covered by D/8 lanes holding
 // 16 bytes each (32/(D/8) keys per pass: 2 for D = 128).  Dot products reduce
@@ -21,6 +24,8 @@
 // stays in registers (log2 domain, scale folded with log2 e); an empty entry
 // writes zeros.  The work is pure bandwidth: 2 FLOP per byte.
 #include <math.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -112,41 +117,58 @@ __global__ void __launch_bounds__(256, 3) smallseq_kernel(SmallSeqParams p) {
         qf[2 * i + 1] = bf16hi(w[i]) * p.scale_log2;
       }
     }
-    float s[PASSES];
-    float m = -INFINITY;
-#pragma unroll
-    for (int pp = 0; pp < PASSES; ++pp) {
-      s[pp] = -INFINITY;
-      if (pp * KPP >= cur.n) continue;  // warp-uniform: no key of this pass exists
-      const uint32_t w[4] = {cur.k[pp].x, cur.k[pp].y, cur.k[pp].z, cur.k[pp].w};
-      float dot = 0.f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        dot = fmaf(qf[2 * i], bf16lo(w[i]), dot);
-        dot = fmaf(qf[2 * i + 1], bf16hi(w[i]), dot);
-      }
-#pragma unroll
-      for (int o = LPK / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-      s[pp] = (pp * KPP + sub < cur.n) ? dot : -INFINITY;
-      m = fmaxf(m, s[pp]);
-    }
-#pragma unroll
-    for (int o = LPK; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    // NP passes of KPP keys, straight-line (the shuffle trees of all passes
+    // overlap); NP is the smallest power of two covering the entry's keys
     float sum = 0.f, acc[8];
+    auto attend = [&](auto np_tag) {
+      constexpr int NP = decltype(np_tag)::value;
+      float sc[NP];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      for (int pp = 0; pp < NP; ++pp) {
+        const uint32_t w[4] = {cur.k[pp].x, cur.k[pp].y, cur.k[pp].z, cur.k[pp].w};
+        float dot = 0.f;
 #pragma unroll
-    for (int pp = 0; pp < PASSES; ++pp) {
-      if (pp * KPP >= cur.n) continue;
-      const float pw = (s[pp] == -INFINITY) ? 0.f : fast_exp2(s[pp] - m);
-      sum += pw;
-      const uint32_t w[4] = {cur.v[pp].x, cur.v[pp].y, cur.v[pp].z, cur.v[pp].w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        acc[2 * i] = fmaf(pw, bf16lo(w[i]), acc[2 * i]);
-        acc[2 * i + 1] = fmaf(pw, bf16hi(w[i]), acc[2 * i + 1]);
+        for (int i = 0; i < 4; ++i) {
+          dot = fmaf(qf[2 * i], bf16lo(w[i]), dot);
+          dot = fmaf(qf[2 * i + 1], bf16hi(w[i]), dot);
+        }
+        sc[pp] = dot;
       }
-    }
+#pragma unroll
+      for (int o = LPK / 2; o >= 1; o >>= 1)
+#pragma unroll
+        for (int pp = 0; pp < NP; ++pp) sc[pp] += __shfl_xor_sync(0xffffffffu, sc[pp], o);
+      float m = -INFINITY;
+#pragma unroll
+      for (int pp = 0; pp < NP; ++pp) {
+        if (pp * KPP + sub >= cur.n) sc[pp] = -INFINITY;
+        m = fmaxf(m, sc[pp]);
+      }
+#pragma unroll
+      for (int o = LPK; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int pp = 0; pp < NP; ++pp) {
+        const float pw = (sc[pp] == -INFINITY) ? 0.f : fast_exp2(sc[pp] - m);
+        sum += pw;
+        const uint32_t w[4] = {cur.v[pp].x, cur.v[pp].y, cur.v[pp].z, cur.v[pp].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[2 * i] = fmaf(pw, bf16lo(w[i]), acc[2 * i]);
+          acc[2 * i + 1] = fmaf(pw, bf16hi(w[i]), acc[2 * i + 1]);
+        }
+      }
+    };
+    const int npass = (cur.n + KPP - 1) / KPP;
+    if (npass <= 1)
+      attend(std::integral_constant<int, 1>{});
+    else if (npass <= 2)
+      attend(std::integral_constant<int, 2>{});
+    else if (PASSES <= 4 || npass <= 4)
+      attend(std::integral_constant<int, (PASSES < 4 ? PASSES : 4)>{});
+    else
+      attend(std::integral_constant<int, PASSES>{});
 #pragma unroll
     for (int o = LPK; o < 32; o <<= 1) {
       sum += __shfl_xor_sync(0xffffffffu, sum, o);

@@ -180,12 +180,24 @@ def test_tiny_config():
 
 @pytest.mark.parametrize("d", [128, 64])
 @pytest.mark.parametrize("causal", [True, False])
-@pytest.mark.parametrize("g,hkv", [(4, 2), (1, 3), (8, 1)])
+@pytest.mark.parametrize("g,hkv", [(4, 2), (1, 3), (8, 1), (16, 1)])
 def test_prefill_small(d, causal, g, hkv):
     lens = [2, 15, 16, 17, 127, 128, 129, 300, 513]
     cpu = build(lens, lens, g * hkv, hkv, d, causal=causal, seed=d + g + causal)
     out, _, _, ws = run_varlen(case_to(cpu, "cuda"))
     assert_attention_close(out, oracle_varlen(cpu), what=f"prefill d={d} causal={causal} g={g}")
+    assert pa.get_error(ws) == (0, 0)
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_prefill_exact_tile_multiples(d):
+    # query counts on 128-row tile / 256-row work-item boundaries, key counts on
+    # 128-key KV-tile boundaries, and one work item whose second tile is empty
+    seq_lens = [256, 384, 1024, 128, 512, 640]
+    qlens = [256, 384, 128, 128, 256, 128]
+    cpu = build(seq_lens, qlens, 8, 2, d, causal=True, seed=40 + d)
+    out, _, _, ws = run_varlen(case_to(cpu, "cuda"))
+    assert_attention_close(out, oracle_varlen(cpu), what=f"tile multiples d={d}")
     assert pa.get_error(ws) == (0, 0)
 
 
