@@ -55,6 +55,9 @@ def _load():
         lib.oracle_attention_varlen.restype = i32
         lib.oracle_attention_varlen.argtypes = [
             p, p, p, p, p, p, i32, i32, i32, i32, f64, i32, p, i64, p]
+        lib.oracle_attention_varlen_spans.restype = i32
+        lib.oracle_attention_varlen_spans.argtypes = [
+            p, p, p, p, p, p, i32, i32, i32, i32, f64, p, p, p, i64, p]
         lib.oracle_attention_varlen_paged.restype = i32
         lib.oracle_attention_varlen_paged.argtypes = [
             p, p, p, p, i32, p, p, i32, i32, i32, i32, i32, i64, f64, i32, p, i64, p]
@@ -115,6 +118,31 @@ def attention_varlen(q, k_seq, v_seq, kv_offsets, seq_lens, query_start_loc,
         _ptr(rows_a), 0 if rows_a is None else len(rows_a), _ptr(out))
     if rc != 0:
         raise ValueError(f"oracle_attention_varlen failed ({rc})")
+    return out
+
+
+def attention_varlen_spans(q, k_seq, v_seq, kv_offsets, seq_lens, query_start_loc,
+                           num_kv_heads, scale, span_offsets, spans, rows=None):
+    """Piecewise block-causal attention (full segments + causal rest), logical
+    form; span_offsets [S+1] int32, spans [N, 2] int32 (start, end) key
+    positions.  Returns float64 [T, Hq, D]."""
+    q = _arr(q, np.uint16)
+    k_seq, v_seq = _arr(k_seq, np.uint16), _arr(v_seq, np.uint16)
+    kv_offsets = _arr(kv_offsets, np.int64)
+    seq_lens = _arr(seq_lens, np.int32)
+    qsl = _arr(query_start_loc, np.int32)
+    so = _arr(span_offsets, np.int32)
+    sp = _arr(np.asarray(spans).reshape(-1, 2) if np.asarray(spans).size else
+              np.zeros((1, 2), np.int32), np.int32)
+    t, hq, d = q.shape
+    out = np.zeros((t, hq, d), dtype=np.float64)
+    rows_a = None if rows is None else _arr(rows, np.int64)
+    rc = _load().oracle_attention_varlen_spans(
+        _ptr(q), _ptr(k_seq), _ptr(v_seq), _ptr(kv_offsets), _ptr(seq_lens), _ptr(qsl),
+        len(seq_lens), hq, num_kv_heads, d, float(scale), _ptr(so), _ptr(sp),
+        _ptr(rows_a), 0 if rows_a is None else len(rows_a), _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_attention_varlen_spans failed ({rc})")
     return out
 
 

@@ -35,6 +35,17 @@
  *      reads them through a block table from a cache this file wrote, which
  *      lets a test pin page addressing against the logical form.
  *
+ *  oracle_attention_varlen_spans
+ *      The piecewise block-causal attention of vllm-omni PR #9244 "Support
+ *      piecewise block-causal attention for full_attn_spans" (description:
+ *      the shared segment plan).  A sequence's key positions are split into
+ *      full segments (the spans, [start, end)) and causal segments (the
+ *      rest).  A query at key position p inside a full segment [start, end)
+ *      attends bidirectionally to the truncated prefix, keys j < end; any
+ *      other query sees keys j <= p, as with plain causal attention.  With
+ *      queries and keys aligned this is the description's dense reference,
+ *      "key at or before the query, or in the same full block".
+ *
  *  oracle_attention_smallseq
  *      ROCm/TransformerEngine PR #461 "CK varlen cross attention for
  *      small-seq", description: one query per batch entry (s_q = 1), keys and
@@ -147,6 +158,27 @@ static int64_t visible_keys(int64_t i, int64_t len_q, int64_t len_kv, int causal
     return n;
 }
 
+/* Keys a query at key position p may see when full segments are given:
+   sp[0..2*nsp) holds the sequence's spans as (start, end) pairs.  A span is
+   used only if 0 <= start < end <= len_kv and start >= the previous pair's
+   end; the others are ignored.  Inside a used span [start, end): keys
+   0 .. end-1; otherwise keys 0 .. p (causal).  Returns a count clamped to
+   [0, len_kv]. */
+static int64_t visible_keys_spans(int64_t p, int64_t len_kv, const int32_t *sp,
+                                  int64_t nsp) {
+    int64_t n = p + 1;
+    int64_t prev_end = 0;
+    for (int64_t k = 0; k < nsp; ++k) {
+        int64_t a = sp[2 * k], b = sp[2 * k + 1];
+        int ok = a >= 0 && a < b && b <= len_kv && a >= prev_end;
+        prev_end = b;
+        if (ok && p >= a && p < b && b > n) n = b;
+    }
+    if (n < 0) n = 0;
+    if (n > len_kv) n = len_kv;
+    return n;
+}
+
 /*
  * out[d] = sum_j w_j v_j[d],  w_j = exp(s_j) / sum_i exp(s_i),
  * s_j = scale * <q, k_j>, over keys j < n_vis.  n_vis == 0 gives zeros.
@@ -201,6 +233,7 @@ static int varlen_driver(const uint16_t *q, const uint16_t *k_base,
                          const int32_t *seq_lens, const int32_t *query_start_loc,
                          int num_seqs, int num_q_heads, int num_kv_heads,
                          int head_dim, double scale, int causal,
+                         const int32_t *span_offsets, const int32_t *spans,
                          const int64_t *rows, int64_t num_rows, double *out) {
     if (num_kv_heads <= 0 || num_q_heads <= 0 || num_q_heads % num_kv_heads != 0)
         return -1;
@@ -225,6 +258,11 @@ static int varlen_driver(const uint16_t *q, const uint16_t *k_base,
             int64_t len_kv = seq_lens[s];
             int64_t i = t - query_start_loc[s];
             int64_t n_vis = visible_keys(i, len_q, len_kv, causal);
+            if (span_offsets) {
+                int64_t a = span_offsets[s], b = span_offsets[s + 1];
+                n_vis = visible_keys_spans((len_kv - len_q) + i, len_kv,
+                                           spans + 2 * a, b > a ? b - a : 0);
+            }
             for (int h = 0; h < num_q_heads; ++h) {
                 kv_view kview = {0}, vview = {0};
                 kview.num_kv_heads = vview.num_kv_heads = num_kv_heads;
@@ -274,7 +312,27 @@ int oracle_attention_varlen(const uint16_t *q, const uint16_t *k_seq,
                             int64_t num_rows, double *out) {
     return varlen_driver(q, k_seq, v_seq, kv_offsets, NULL, 0, 1, 0, seq_lens,
                          query_start_loc, num_seqs, num_q_heads, num_kv_heads,
-                         head_dim, scale, causal, rows, num_rows, out);
+                         head_dim, scale, causal, NULL, NULL, rows, num_rows, out);
+}
+
+/*
+ * Logical form with full segments (see visible_keys_spans): span_offsets
+ * [num_seqs + 1] indexes spans [*, 2] int32 (start, end) key positions;
+ * sequence s owns pairs span_offsets[s] .. span_offsets[s+1]-1.  Queries
+ * outside every full segment are causal.
+ */
+int oracle_attention_varlen_spans(const uint16_t *q, const uint16_t *k_seq,
+                                  const uint16_t *v_seq, const int64_t *kv_offsets,
+                                  const int32_t *seq_lens,
+                                  const int32_t *query_start_loc, int num_seqs,
+                                  int num_q_heads, int num_kv_heads, int head_dim,
+                                  double scale, const int32_t *span_offsets,
+                                  const int32_t *spans, const int64_t *rows,
+                                  int64_t num_rows, double *out) {
+    if (!span_offsets || !spans) return -1;
+    return varlen_driver(q, k_seq, v_seq, kv_offsets, NULL, 0, 1, 0, seq_lens,
+                         query_start_loc, num_seqs, num_q_heads, num_kv_heads,
+                         head_dim, scale, 1, span_offsets, spans, rows, num_rows, out);
 }
 
 /*
@@ -294,7 +352,7 @@ int oracle_attention_varlen_paged(const uint16_t *q, const uint16_t *k_cache,
     return varlen_driver(q, k_cache, v_cache, NULL, block_tables,
                          max_blocks_per_seq, block_size, num_blocks, seq_lens,
                          query_start_loc, num_seqs, num_q_heads, num_kv_heads,
-                         head_dim, scale, causal, rows, num_rows, out);
+                         head_dim, scale, causal, NULL, NULL, rows, num_rows, out);
 }
 
 /*
