@@ -259,6 +259,36 @@ def time_varlen_component(pa, case, iters=20, warmup=3, with_scatter=False):
     return statistics.mean(a.elapsed_time(b) for a, b in evs)
 
 
+def time_spans_component(pa, case, span_offsets, spans, iters=20, warmup=3):
+    """Average device time (ms) of one attention_varlen_spans call."""
+    ws = pa.varlen_workspace(case.num_seqs, case.num_q_tokens, case.num_q_heads,
+                             case.num_kv_heads, case.head_dim)
+    out = torch.empty_like(case.q)
+    mql, msl = case.max_query_len, case.max_seq_len
+    pa.write_kv(case.k_new, case.v_new, case.slot_mapping, case.k_cache, case.v_cache)
+
+    def run():
+        pa.attention_varlen_spans(case.q, case.k_cache, case.v_cache, case.block_tables,
+                                  case.seq_lens, case.query_start_loc, case.num_kv_heads,
+                                  case.scale, span_offsets, spans, out, max_query_len=mql,
+                                  max_seq_len=msl, workspace=ws)
+
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(iters)]
+    for a, b in evs:
+        a.record()
+        run()
+        b.record()
+    torch.cuda.synchronize()
+    st, bits = pa.get_error(ws)
+    if st != 0:
+        raise RuntimeError(f"device error word {bits:#x}")
+    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+
 def components(pa, hbm_peak, tc_peak, peak_kind):
     """Secondary single-GPU measurements on the other workloads (device time per call)."""
     res = {}
@@ -287,6 +317,15 @@ def components(pa, hbm_peak, tc_peak, peak_kind):
     res["smallseq_batch"] = {"ms": round(ms, 4), "gbs": round(gbs, 1),
                              "frac": round(gbs / hbm_peak, 3), "unit": "GB/s", "of": peak_kind}
     del ss, out
+    sc, so, sp = workloads.spans_prefill(device=dev, keep_logical=False)
+    ms = time_spans_component(pa, sc, so, sp)
+    pairs = workloads.spans_visible_pairs(sc.seq_lens.tolist(), sc.query_lens.tolist(),
+                                          so.tolist(), sp.tolist())
+    tf = 4 * sc.head_dim * sc.num_q_heads * pairs / (ms * 1e-3) / 1e12
+    res["spans_prefill"] = {"ms": round(ms, 4), "tflops": round(tf, 1),
+                            "frac": round(tf / tc_peak, 3), "peak": tc_peak,
+                            "unit": "TFLOP/s", "of": peak_kind}
+    del sc, so, sp
     mx = workloads.mixed_step(device=dev, keep_logical=False)
     ms = time_varlen_component(pa, mx, iters=10)
     nbytes = attention_bytes(mx)
@@ -406,6 +445,15 @@ def run_single_workload(args):
     torch.cuda.set_device(dev)
     hbm_peak, tc_peak, _, peak_kind = measured_peaks()
     name = args.workload
+    if name == "spans_prefill":
+        sc, so, sp = workloads.spans_prefill(device=dev, keep_logical=False)
+        ms = time_spans_component(pa, sc, so, sp, iters=args.steps, warmup=args.warmup)
+        pairs = workloads.spans_visible_pairs(sc.seq_lens.tolist(), sc.query_lens.tolist(),
+                                              so.tolist(), sp.tolist())
+        v = 4 * sc.head_dim * sc.num_q_heads * pairs / (ms * 1e-3) / 1e12
+        return {"workload": name, "value": round(v, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 5),
+                "steps": args.steps, "warmup": args.warmup, "frac": round(v / tc_peak, 4),
+                "peak": tc_peak, "peak_kind": peak_kind}
     if name == "smallseq_batch":
         ss = workloads.smallseq_batch(device=dev)
         out = torch.empty_like(ss.q)
@@ -571,7 +619,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-components", action="store_true")
-    ap.add_argument("--workload", default="decode_batch", choices=sorted(workloads.NAMED),
+    ap.add_argument("--workload", default="decode_batch",
+                    choices=sorted(list(workloads.NAMED) + ["spans_prefill"]),
                     help="decode_batch is the headline; the others time one workload alone")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per dominant-kernel launch from an ncu capture, if current")

@@ -68,6 +68,7 @@ typedef enum {
 #define PA_DEVERR_QLEN      0x8u  /* a sequence has more queries than keys       */
 #define PA_DEVERR_HINT      0x10u /* a length exceeded max_query_len/max_seq_len */
 #define PA_DEVERR_TIMEOUT   0x20u /* a bounded wait inside a kernel gave up      */
+#define PA_DEVERR_SPANS     0x40u /* a full-attention span was malformed (unused) */
 
 /* Bytes at the start of every workspace reserved for the error word. */
 #define PA_ERROR_WORD_BYTES 256
@@ -156,6 +157,43 @@ pa_status pa_attention_varlen(const void* q, const void* k_cache, const void* v_
                               int32_t max_query_len, int32_t max_seq_len, float scale,
                               int32_t causal, void* out, void* workspace,
                               size_t workspace_bytes, void* stream);
+
+/*
+ * pa_attention_varlen_spans — pa_attention_varlen with piecewise block-causal
+ * masking (full-attention blocks inside causal sequences).
+ *
+ * Defined by vllm-omni PR #9244 "Support piecewise block-causal attention for
+ * full_attn_spans" (description: the shared segment plan).  A sequence's key
+ * positions are split into full segments, listed as spans, and causal
+ * segments (everything else).  With Lq queries and Lkv keys, query i sits at
+ * key position p = (Lkv - Lq) + i.  If p lies in a span [start, end) the
+ * query attends bidirectionally to keys 0 .. end-1 (the truncated prefix);
+ * otherwise it attends to keys 0 .. p, as with causal == 1.  Single-query
+ * (decode) sequences are unaffected: their one query sees every key either
+ * way when spans end at or before Lkv.
+ *
+ *  span_offsets  [num_seqs + 1] int32: sequence s owns spans
+ *                span_offsets[s] .. span_offsets[s+1]-1
+ *  spans         [num_spans, 2] int32 (start, end) key positions, in
+ *                increasing order per sequence; may be NULL if num_spans == 0
+ *  num_spans     total spans
+ * Every other argument is pa_attention_varlen's (there is no causal flag:
+ * positions outside spans are causal).  A span that is empty, outside
+ * [0, Lkv], or starts before the previous span of its sequence ends is
+ * ignored and raises PA_DEVERR_SPANS; span_offsets that decrease or leave
+ * [0, num_spans] make that sequence span-free and raise PA_DEVERR_SPANS.
+ * The workspace is the same as pa_attention_varlen's.
+ */
+pa_status pa_attention_varlen_spans(const void* q, const void* k_cache, const void* v_cache,
+                                    const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                    const int32_t* seq_lens, const int32_t* query_start_loc,
+                                    int32_t num_seqs, int64_t num_q_tokens,
+                                    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                    int32_t block_size, int64_t num_blocks,
+                                    int32_t max_query_len, int32_t max_seq_len, float scale,
+                                    const int32_t* span_offsets, const int32_t* spans,
+                                    int32_t num_spans, void* out, void* workspace,
+                                    size_t workspace_bytes, void* stream);
 
 /*
  * pa_attention_varlen_static — pa_attention_varlen for callers that cannot

@@ -25,24 +25,25 @@ import torch
 
 __all__ = [
     "PaError", "library_path", "load", "write_kv", "attention_varlen", "attention_smallseq",
-    "attention_varlen_static", "STATIC_SCRATCH_BYTES",
+    "attention_varlen_static", "attention_varlen_spans", "STATIC_SCRATCH_BYTES",
     "varlen_workspace_size", "varlen_workspace", "error_workspace", "get_error",
     "status_string", "version", "EXPORTED_SYMBOLS",
     "DEVERR_SLOT", "DEVERR_BLOCK", "DEVERR_LENGTHS", "DEVERR_QLEN", "DEVERR_HINT",
-    "DEVERR_TIMEOUT", "ERROR_WORD_BYTES",
+    "DEVERR_TIMEOUT", "DEVERR_SPANS", "ERROR_WORD_BYTES",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 PA_OK = 0
 DEVERR_SLOT, DEVERR_BLOCK, DEVERR_LENGTHS = 0x1, 0x2, 0x4
 DEVERR_QLEN, DEVERR_HINT, DEVERR_TIMEOUT = 0x8, 0x10, 0x20
+DEVERR_SPANS = 0x40
 ERROR_WORD_BYTES = 256
 STATIC_SCRATCH_BYTES = 32 << 20  # PA_STATIC_SCRATCH_BYTES
 
 EXPORTED_SYMBOLS = (
     "pa_write_kv", "pa_attention_varlen_workspace_size", "pa_attention_varlen",
     "pa_attention_smallseq", "pa_get_error", "pa_status_string", "pa_version",
-    "pa_attention_varlen_static",
+    "pa_attention_varlen_static", "pa_attention_varlen_spans",
 )
 
 _lib = None
@@ -91,6 +92,10 @@ def load(build_if_missing: bool = True):
         lib.pa_attention_varlen_static.argtypes = [
             p, p, p, p, i32, p, p, i32, i64, i32, i32, i32, i32, i64, i32, i32,
             ctypes.c_float, i32, p, p]
+        lib.pa_attention_varlen_spans.restype = ctypes.c_int
+        lib.pa_attention_varlen_spans.argtypes = [
+            p, p, p, p, i32, p, p, i32, i64, i32, i32, i32, i32, i64, i32, i32,
+            ctypes.c_float, p, p, i32, p, p, ctypes.c_size_t, p]
         lib.pa_attention_smallseq.restype = ctypes.c_int
         lib.pa_attention_smallseq.argtypes = [p, p, p, p, i32, i32, i32, i32, i32,
                                               ctypes.c_float, p, p, p]
@@ -210,6 +215,52 @@ def attention_varlen(q, k_cache, v_cache, block_tables, seq_lens, query_start_lo
         float(scale), int(bool(causal)), out.data_ptr(), workspace.data_ptr(),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _raise(st, "pa_attention_varlen")
+    return out
+
+
+def attention_varlen_spans(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc,
+                           num_kv_heads, scale, span_offsets, spans, out, max_query_len=None,
+                           max_seq_len=None, workspace=None, stream=None):
+    """Paged varlen attention with full-attention spans inside causal sequences.
+
+    span_offsets: int32 [S+1] (sequence s owns spans span_offsets[s] ..
+    span_offsets[s+1]-1); spans: int32 [N, 2] (start, end) key positions.
+    A query whose key position lies in a span [start, end) sees keys
+    0 .. end-1; every other query is causal.  Writes out [T, Hq, D] (bf16).
+    """
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k_cache, "k_cache", torch.bfloat16, 4)
+    _check(v_cache, "v_cache", torch.bfloat16, 4)
+    _check(block_tables, "block_tables", torch.int32, 2)
+    _check(seq_lens, "seq_lens", torch.int32, 1)
+    _check(query_start_loc, "query_start_loc", torch.int32, 1)
+    _check(span_offsets, "span_offsets", torch.int32, 1)
+    _check(spans, "spans", torch.int32, 2)
+    _check(out, "out", torch.bfloat16, 3)
+    t, hq, d = q.shape
+    nb, bs, hkv, d_c = k_cache.shape
+    if hkv != num_kv_heads or d_c != d or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shape does not match q / num_kv_heads")
+    if out.shape != q.shape:
+        raise ValueError("out must have q's shape")
+    s = seq_lens.shape[0]
+    if query_start_loc.shape[0] != s + 1 or block_tables.shape[0] != s:
+        raise ValueError("seq_lens, query_start_loc and block_tables disagree on num_seqs")
+    if span_offsets.shape[0] != s + 1 or (spans.numel() and spans.shape[1] != 2):
+        raise ValueError("span_offsets must be [S+1] and spans [N, 2]")
+    mb = block_tables.shape[1]
+    mql = t if max_query_len is None else int(max_query_len)
+    msl = mb * bs if max_seq_len is None else int(max_seq_len)
+    if workspace is None:
+        workspace = varlen_workspace(s, t, hq, hkv, d, device=q.device)
+    n_spans = spans.shape[0] if spans.numel() else 0
+    st = load().pa_attention_varlen_spans(
+        q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(), mb,
+        seq_lens.data_ptr(), query_start_loc.data_ptr(), s, t, hq, hkv, d, bs, nb, mql, msl,
+        float(scale), span_offsets.data_ptr(), spans.data_ptr() if n_spans else None, n_spans,
+        out.data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    _raise(st, "pa_attention_varlen_spans")
     return out
 
 

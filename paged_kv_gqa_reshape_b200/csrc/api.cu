@@ -132,14 +132,18 @@ size_t pa_attention_varlen_workspace_size(int32_t num_seqs, int64_t num_q_tokens
   return pa::make_layout(num_seqs, num_q_tokens, num_q_heads, num_kv_heads, head_dim).total;
 }
 
-pa_status pa_attention_varlen(const void* q, const void* k_cache, const void* v_cache,
-                              const int32_t* block_tables, int32_t max_blocks_per_seq,
-                              const int32_t* seq_lens, const int32_t* query_start_loc,
-                              int32_t num_seqs, int64_t num_q_tokens, int32_t num_q_heads,
-                              int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
-                              int64_t num_blocks, int32_t max_query_len, int32_t max_seq_len,
-                              float scale, int32_t causal, void* out, void* workspace,
-                              size_t workspace_bytes, void* stream) {
+namespace {
+
+// pa_attention_varlen and pa_attention_varlen_spans (span_offsets non-null)
+pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* v_cache,
+                                const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                const int32_t* seq_lens, const int32_t* query_start_loc,
+                                int32_t num_seqs, int64_t num_q_tokens, int32_t num_q_heads,
+                                int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                int64_t num_blocks, int32_t max_query_len, int32_t max_seq_len,
+                                float scale, int32_t causal, const int32_t* span_offsets,
+                                const int32_t* spans, int32_t num_spans, void* out,
+                                void* workspace, size_t workspace_bytes, void* stream) {
   // ---- host-visible checks (nothing launched yet) ----
   if (num_seqs < 0 || num_q_tokens < 0 || num_q_tokens > 0x7fffffffll || num_q_heads <= 0 ||
       num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || max_blocks_per_seq <= 0 ||
@@ -153,6 +157,10 @@ pa_status pa_attention_varlen(const void* q, const void* k_cache, const void* v_
   if (num_seqs == 0 || num_q_tokens == 0) return PA_OK;
   if (!q || !k_cache || !v_cache || !block_tables || !seq_lens || !query_start_loc || !out ||
       !workspace)
+    return PA_ERR_INVALID_ARG;
+  if (span_offsets && (num_spans < 0 || (num_spans > 0 && !spans) ||
+                       (reinterpret_cast<uintptr_t>(span_offsets) & 3u) ||
+                       (reinterpret_cast<uintptr_t>(spans) & 3u)))
     return PA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
       !aligned16(workspace) || (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
@@ -191,7 +199,8 @@ pa_status pa_attention_varlen(const void* q, const void* k_cache, const void* v_
   cudaError_t e = cudaSuccess;
   if (run_prefill || !self_plan) {
     pa::launch_plan(query_start_loc, seq_lens, num_seqs, num_q_tokens, max_blocks_per_seq,
-                    block_size, max_query_len, max_seq_len, causal, num_kv_heads, ws, L, st);
+                    block_size, max_query_len, max_seq_len, causal, num_kv_heads, span_offsets,
+                    spans, num_spans, ws, L, st);
     e = cudaGetLastError();
     if (e != cudaSuccess) return PA_ERR_CUDA;
   }
@@ -207,6 +216,9 @@ pa_status pa_attention_varlen(const void* q, const void* k_cache, const void* v_
     pp.num_q_tokens = num_q_tokens;
     pp.scale_log2 = scale_log2;
     pp.causal = causal;
+    pp.span_offsets = span_offsets;
+    pp.spans = spans;
+    pp.num_spans = num_spans;
     pp.out = static_cast<__nv_bfloat16*>(out);
     pp.ws = ws;
     pp.L = L;
@@ -240,6 +252,39 @@ pa_status pa_attention_varlen(const void* q, const void* k_cache, const void* v_
     fprintf(stderr, "[pa] varlen S=%d T=%lld Hq=%d Hkv=%d D=%d prefill=%d sms=%d\n", num_seqs,
             (long long)num_q_tokens, num_q_heads, num_kv_heads, head_dim, (int)run_prefill, nsm);
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // namespace
+
+pa_status pa_attention_varlen(const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* block_tables, int32_t max_blocks_per_seq,
+                              const int32_t* seq_lens, const int32_t* query_start_loc,
+                              int32_t num_seqs, int64_t num_q_tokens, int32_t num_q_heads,
+                              int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                              int64_t num_blocks, int32_t max_query_len, int32_t max_seq_len,
+                              float scale, int32_t causal, void* out, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  return attention_varlen_impl(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                               query_start_loc, num_seqs, num_q_tokens, num_q_heads, num_kv_heads,
+                               head_dim, block_size, num_blocks, max_query_len, max_seq_len, scale,
+                               causal, nullptr, nullptr, 0, out, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_attention_varlen_spans(const void* q, const void* k_cache, const void* v_cache,
+                                    const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                    const int32_t* seq_lens, const int32_t* query_start_loc,
+                                    int32_t num_seqs, int64_t num_q_tokens, int32_t num_q_heads,
+                                    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                    int64_t num_blocks, int32_t max_query_len, int32_t max_seq_len,
+                                    float scale, const int32_t* span_offsets, const int32_t* spans,
+                                    int32_t num_spans, void* out, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  if (!span_offsets && num_seqs > 0) return PA_ERR_INVALID_ARG;
+  return attention_varlen_impl(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                               query_start_loc, num_seqs, num_q_tokens, num_q_heads, num_kv_heads,
+                               head_dim, block_size, num_blocks, max_query_len, max_seq_len, scale,
+                               1, span_offsets, spans, num_spans, out, workspace, workspace_bytes,
+                               stream);
 }
 
 pa_status pa_attention_smallseq(const void* q, const void* k, const void* v,

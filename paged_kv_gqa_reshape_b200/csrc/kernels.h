@@ -19,6 +19,7 @@ cudaError_t launch_write_kv(const void* k, const void* v, const int64_t* slot_ma
 void launch_plan(const int32_t* query_start_loc, const int32_t* seq_lens, int num_seqs,
                  long long num_q_tokens, int max_blocks_per_seq, int block_size,
                  int max_query_len, int max_seq_len, int causal, int num_kv_heads,
+                 const int32_t* span_offsets, const int32_t* spans, int num_spans,
                  unsigned char* ws, const WorkspaceLayout& L, cudaStream_t stream);
 
 // ---- split-KV decode -------------------------------------------------------
@@ -58,6 +59,9 @@ struct PrefillParams {
   long long num_q_tokens;
   float scale_log2;
   int causal;
+  const int32_t* span_offsets;  // full-attention spans (null: none)
+  const int32_t* spans;
+  int num_spans;
   __nv_bfloat16* out;
   unsigned char* ws;
   WorkspaceLayout L;

@@ -36,6 +36,7 @@ struct WorkspaceLayout {
   size_t header;     // PlanHeader
   size_t seq_info;   // SeqInfo[num_seqs]
   size_t tiles;      // int2[max_tiles]   (seq, first query row of a 256-row work item)
+  size_t tile_n;     // int2[max_tiles]   KV tiles its two 128-row query tiles visit
   size_t page_pfx;   // int32[num_seqs + 1]  exclusive prefix of decode pages
   size_t counters;   // int32[num_seqs * num_kv_heads]  split-KV arrival counters
   size_t lse;        // float[max_slots * num_q_heads]   log2-sum-exp per partial
@@ -59,6 +60,8 @@ inline WorkspaceLayout make_layout(int64_t num_seqs, int64_t num_q_tokens, int64
   off = align_up(off + sizeof(SeqInfo) * (size_t)num_seqs, 256);
   L.max_tiles = (num_q_tokens + kPrefillItemRows - 1) / kPrefillItemRows + num_seqs;
   L.tiles = off;
+  off = align_up(off + 8 * (size_t)L.max_tiles, 256);
+  L.tile_n = off;
   off = align_up(off + 8 * (size_t)L.max_tiles, 256);
   // Decode CTA c of a KV-head group covering sequence s writes partial slot
   // c + s; a launch has at most kDecodeMaxWarps / Hkv page ranges per group.

@@ -2,8 +2,9 @@
 //
 // Reads query_start_loc and seq_lens, sanitises them into SeqInfo, and builds
 //  - the prefill work list: one entry per 256-query-row item (two 128-row
-//    tiles) of every sequence with more than one query, ordered by
-//    descending KV-tile count (longest work first, for the persistent
+//    tiles) of every sequence with more than one query, with the KV tiles
+//    each tile visits (causal, full-attention spans, or all keys), ordered
+//    by descending KV-tile count (longest work first, for the persistent
 //    prefill grid);
 //  - the exclusive prefix of 16-key pages over the single-query (decode)
 //    sequences, from which the decode CTAs cut their balanced page ranges
@@ -14,6 +15,7 @@
 // the device before routing), without any host synchronisation.
 #include "common.cuh"
 #include "layout.h"
+#include "spans.cuh"
 
 namespace pa {
 
@@ -49,19 +51,30 @@ __device__ int block_exclusive_scan(int v, int* out_excl, int* s_warp) {
   return total;
 }
 
-// KV tiles of one 128-row tile whose rows are [row0, row0 + rows)
-__device__ __forceinline__ int kv_tiles(const SeqInfo& si, int row0, int rows, int causal) {
+// KV tiles of one 128-row tile whose rows are [row0, row0 + rows): enough
+// for the most keys any of its rows sees (causal, spans or neither)
+__device__ __forceinline__ int kv_tiles(const SeqInfo& si, int row0, int rows, int causal,
+                                        const SpanList& sl, bool* malformed) {
   if (rows <= 0) return 0;
   int vis = si.kv_len;
-  if (causal) vis = max(0, min(si.kv_len, si.kv_len - si.q_len + row0 + rows));
+  const int p0 = si.kv_len - si.q_len + row0;  // key positions of the tile's rows
+  if (sl.pairs || !sl.offsets_ok)
+    vis = span_visible(sl, p0, p0 + rows - 1, malformed);
+  else if (causal)
+    vis = max(0, min(si.kv_len, p0 + rows));
   return (vis + kPrefillTileN - 1) / kPrefillTileN;
 }
 
-// cost of a 256-row work item: the KV tiles of its two 128-row tiles
-__device__ __forceinline__ int tile_cost(const SeqInfo& si, int row0, int causal) {
+// KV tiles of a 256-row work item's two 128-row tiles
+__device__ __forceinline__ int2 item_tiles(const SeqInfo& si, int row0, int causal,
+                                           const SpanList& sl, bool* malformed) {
   const int rows_a = min(kPrefillTileM, si.q_len - row0);
   const int rows_b = min(kPrefillTileM, si.q_len - row0 - kPrefillTileM);
-  return kv_tiles(si, row0, rows_a, causal) + kv_tiles(si, row0 + kPrefillTileM, rows_b, causal);
+  bool bad_a = false, bad_b = false;
+  const int2 n = make_int2(kv_tiles(si, row0, rows_a, causal, sl, &bad_a),
+                           kv_tiles(si, row0 + kPrefillTileM, rows_b, causal, sl, &bad_b));
+  if (malformed) *malformed = bad_a || bad_b;
+  return n;
 }
 
 }  // namespace
@@ -70,11 +83,13 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
     plan_kernel(const int32_t* __restrict__ query_start_loc, const int32_t* __restrict__ seq_lens,
                 int num_seqs, long long num_q_tokens, int max_blocks_per_seq, int block_size,
                 int max_query_len, int max_seq_len, int causal, int num_kv_heads,
-                unsigned char* ws, WorkspaceLayout L) {
+                const int32_t* __restrict__ span_offsets, const int32_t* __restrict__ spans,
+                int num_spans, unsigned char* ws, WorkspaceLayout L) {
   uint32_t* err = reinterpret_cast<uint32_t*>(ws + L.err);
   PlanHeader* hdr = reinterpret_cast<PlanHeader*>(ws + L.header);
   SeqInfo* info = reinterpret_cast<SeqInfo*>(ws + L.seq_info);
   int2* tiles = reinterpret_cast<int2*>(ws + L.tiles);
+  int2* tile_n = reinterpret_cast<int2*>(ws + L.tile_n);
   int32_t* page_pfx = reinterpret_cast<int32_t*>(ws + L.page_pfx);
   int32_t* counters = reinterpret_cast<int32_t*>(ws + L.counters);
 
@@ -131,10 +146,16 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
       const SeqInfo si = info[s];
       if (si.q_len == 1) pages = (si.kv_len + kPageKeys - 1) / kPageKeys;
       if (si.q_len > 1) {
+        const SpanList sl = span_list(span_offsets, spans, num_spans, s, si.kv_len);
+        bool bad = false;
         for (int r = 0; r < si.q_len; r += kPrefillItemRows) {
-          const int c = tile_cost(si, r, causal);
+          bool bad_r = false;
+          const int2 n = item_tiles(si, r, causal, sl, &bad_r);
+          bad |= bad_r;
+          const int c = n.x + n.y;
           atomicAdd(&s_hist[kCostBuckets - 1 - min(c, kCostBuckets - 1)], 1);
         }
+        if (bad) atomicOr(&s_err, PA_DEVERR_SPANS);
       }
     }
     int excl;
@@ -171,11 +192,17 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
   for (int s = tid; s < num_seqs; s += blockDim.x) {
     SeqInfo si = info[s];
     if (si.q_len > 1) {
+      const SpanList sl = span_list(span_offsets, spans, num_spans, s, si.kv_len);
       for (int r = 0; r < si.q_len; r += kPrefillItemRows) {
-        int c = tile_cost(si, r, causal);
+        const int2 n = item_tiles(si, r, causal, sl, nullptr);
+        const int c = n.x + n.y;
         int pos = atomicAdd(&s_hist[kCostBuckets - 1 - min(c, kCostBuckets - 1)], 1);
-        if ((long long)pos < (long long)L.max_tiles) tiles[pos] = make_int2(s, r);  // overlapping query ranges can overflow
-        else atomicOr(&s_err, PA_DEVERR_LENGTHS);
+        if ((long long)pos < (long long)L.max_tiles) {  // overlapping query ranges can overflow
+          tiles[pos] = make_int2(s, r);
+          tile_n[pos] = n;
+        } else {
+          atomicOr(&s_err, PA_DEVERR_LENGTHS);
+        }
       }
     }
   }
@@ -192,10 +219,12 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
 void launch_plan(const int32_t* query_start_loc, const int32_t* seq_lens, int num_seqs,
                  long long num_q_tokens, int max_blocks_per_seq, int block_size,
                  int max_query_len, int max_seq_len, int causal, int num_kv_heads,
+                 const int32_t* span_offsets, const int32_t* spans, int num_spans,
                  unsigned char* ws, const WorkspaceLayout& L, cudaStream_t stream) {
   plan_kernel<<<1, kPlanThreads, 0, stream>>>(query_start_loc, seq_lens, num_seqs, num_q_tokens,
                                               max_blocks_per_seq, block_size, max_query_len,
-                                              max_seq_len, causal, num_kv_heads, ws, L);
+                                              max_seq_len, causal, num_kv_heads, span_offsets,
+                                              spans, num_spans, ws, L);
 }
 
 }  // namespace pa

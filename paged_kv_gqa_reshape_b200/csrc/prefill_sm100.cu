@@ -44,6 +44,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "layout.h"
+#include "spans.cuh"
 
 namespace pa {
 
@@ -79,17 +80,13 @@ struct Work {
   int nmax;
 };
 
-__device__ __forceinline__ int kv_tiles_for(int kv_len, int q_len, int row0, int rows, int causal) {
-  if (rows <= 0) return 0;
-  int vis = kv_len;
-  if (causal) vis = max(0, min(kv_len, kv_len - q_len + row0 + rows));
-  return (vis + BN - 1) / BN;
-}
-
-__device__ __forceinline__ Work decode_work(int w, const int2* tiles, const SeqInfo* info,
-                                            int num_q_heads, int causal) {
+// work item w: sequence, rows, and the KV tiles of its two 128-row tiles (as
+// the plan kernel counted them: causal, full-attention spans or all keys)
+__device__ __forceinline__ Work decode_work(int w, const int2* tiles, const int2* tile_n,
+                                            const SeqInfo* info, int num_q_heads) {
   Work k;
   const int2 t = tiles[w / num_q_heads];
+  const int2 tn = tile_n[w / num_q_heads];
   k.head = w % num_q_heads;
   k.seq = t.x;
   k.row0 = t.y;
@@ -99,8 +96,8 @@ __device__ __forceinline__ Work decode_work(int w, const int2* tiles, const SeqI
   k.kv_len = si.kv_len;
   k.rows[0] = min(BM, si.q_len - t.y);
   k.rows[1] = max(0, min(BM, si.q_len - t.y - BM));
-  k.n[0] = kv_tiles_for(si.kv_len, si.q_len, t.y, k.rows[0], causal);
-  k.n[1] = kv_tiles_for(si.kv_len, si.q_len, t.y + BM, k.rows[1], causal);
+  k.n[0] = tn.x;
+  k.n[1] = tn.y;
   k.nmax = max(k.n[0], k.n[1]);
   return k;
 }
@@ -140,6 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(ws + p.L.header);
   const SeqInfo* info = reinterpret_cast<const SeqInfo*>(ws + p.L.seq_info);
   const int2* tiles = reinterpret_cast<const int2*>(ws + p.L.tiles);
+  const int2* tile_n = reinterpret_cast<const int2*>(ws + p.L.tile_n);
   const int num_work = hdr->num_prefill_tiles * p.num_q_heads;
 
   if (threadIdx.x == 0) {
@@ -181,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int tcount = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < num_work && ok; w += gridDim.x) {
-        const Work wk = decode_work(w, tiles, info, p.num_q_heads, p.causal);
+        const Work wk = decode_work(w, tiles, tile_n, info, p.num_q_heads);
         if (wk.nmax == 0) continue;
         const int kvh = wk.head / p.group;
         if (tcount > 0) ok = mbar_wait_bounded(q_empty, (tcount - 1) & 1, abort_flag, err);
@@ -265,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++pv_it[x];
       };
       for (int w = blockIdx.x; w < num_work && ok; w += gridDim.x) {
-        const Work wk = decode_work(w, tiles, info, p.num_q_heads, p.causal);
+        const Work wk = decode_work(w, tiles, tile_n, info, p.num_q_heads);
         if (wk.nmax == 0) continue;
         ok = mbar_wait_bounded(q_full, tcount & 1, abort_flag, err);
         if (!ok) break;
@@ -317,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;  // S tiles of this query tile consumed so far (phase counter)
     bool ok = true;
     for (int w = blockIdx.x; w < num_work && ok; w += gridDim.x) {
-      const Work wk = decode_work(w, tiles, info, p.num_q_heads, p.causal);
+      const Work wk = decode_work(w, tiles, tile_n, info, p.num_q_heads);
       const int rows = wk.rows[x], n = wk.n[x];
       const int qrow = wk.row0 + x * BM + r;  // query index within the sequence
       const bool row_ok = r < rows;
@@ -332,7 +330,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // last key this row may see (inclusive); below 0 means none
       int limit = wk.kv_len - 1;
-      if (p.causal) limit = min(limit, wk.kv_len - wk.q_len + qrow);
+      const int pos = wk.kv_len - wk.q_len + qrow;  // the row's key position
+      if (p.span_offsets) {
+        const SpanList sl = span_list(p.span_offsets, p.spans, p.num_spans, wk.seq, wk.kv_len);
+        limit = span_visible(sl, pos, pos, nullptr) - 1;
+      } else if (p.causal) {
+        limit = min(limit, pos);
+      }
       float m_use = -INFINITY, l = 0.f;
       for (int j = 0; j < n; ++j) {
         const int cur = it + j;

@@ -76,6 +76,31 @@ def test_varlen_empty_batch_is_a_no_op():
     assert _varlen(pa.load(), T=0) == 0
 
 
+def _spans(lib, **over):
+    args = dict(q=1 << 12, kc=1 << 12, vc=1 << 12, bt=1 << 12, mb=4, sl=1 << 12, qsl=1 << 12,
+                S=2, T=4, Hq=4, Hkv=2, D=64, BS=16, NB=8, mql=4, msl=64, scale=0.125,
+                so=1 << 12, sp=1 << 12, nsp=2, out=1 << 12, ws=1 << 12, wsb=1 << 30, stream=None)
+    args.update(over)
+    return lib.pa_attention_varlen_spans(*args.values())
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(so=0), 1),                  # span offsets are required
+    (dict(sp=0), 1),                  # spans required when there are some
+    (dict(nsp=-1), 1),
+    (dict(so=(1 << 12) + 2), 1),      # misaligned int32
+    (dict(D=96), 2),
+    (dict(wsb=16), 1),
+])
+def test_varlen_spans_rejects_before_launch(over, expect):
+    assert _spans(pa.load(), **over) == expect
+
+
+def test_varlen_spans_empty_batch_is_a_no_op():
+    assert _spans(pa.load(), S=0, so=0) == 0
+    assert _spans(pa.load(), T=0) == 0
+
+
 def test_write_kv_rejects_before_launch():
     lib = pa.load()
     ok = dict(k=1 << 12, v=1 << 12, sm=1 << 12, T=3, Hkv=2, D=64, kc=1 << 12, vc=1 << 12,

@@ -264,6 +264,47 @@ def varlen_prefill(device="cpu", seed=1003, lens=(2048, 3000, 4096, 8192),
                              keep_logical=keep_logical)
 
 
+def spans_prefill(device="cpu", seed=1006, num_seqs=4, text=512, cond=1536, target=2048,
+                  num_q_heads=32, num_kv_heads=8, head_dim=128, keep_logical=True):
+    """Piecewise block-causal prefill: each sequence is a causal text run
+    followed by two image blocks with full attention (condition, target),
+    4 x (512 + 1536 + 2048) = 16 384 tokens, Hq 32 / Hkv 8, D 128.
+    Returns (case, span_offsets int32 [S+1], spans int32 [2S, 2])."""
+    n = text + cond + target
+    case = build_varlen_case("spans_prefill", [n] * num_seqs, [n] * num_seqs, num_q_heads,
+                             num_kv_heads, head_dim, True, seed, device=device,
+                             keep_logical=keep_logical)
+    spans = []
+    for _ in range(num_seqs):
+        spans += [(text, text + cond), (text + cond, n)]
+    span_offsets = torch.arange(0, 2 * num_seqs + 1, 2, dtype=torch.int32, device=device)
+    return case, span_offsets, torch.tensor(spans, dtype=torch.int32, device=device)
+
+
+def spans_visible_pairs(seq_lens, query_lens, span_offsets, spans) -> int:
+    """Visible (query, key) pairs under the span rule (per head)."""
+    total = 0
+    so = [int(x) for x in span_offsets]
+    sp = [(int(a), int(b)) for a, b in spans]
+    for s, (lkv, lq) in enumerate(zip(seq_lens, query_lens)):
+        lkv, lq = int(lkv), int(lq)
+        if lq <= 1:
+            total += lkv * lq
+            continue
+        ends = {}
+        prev = 0
+        for a, b in sp[so[s]:so[s + 1]]:
+            if 0 <= a < b <= lkv and a >= prev:
+                for pos in range(a, b):
+                    ends[pos] = b
+            prev = b
+        off = lkv - lq
+        for i in range(lq):
+            pos = off + i
+            total += max(0, min(lkv, ends.get(pos, pos + 1)))
+    return total
+
+
 def smallseq_batch(device="cpu", seed=1004, batch=30720, heads=16, head_dim=128,
                    choices=(2, 4, 6, 8, 12, 16)) -> SmallSeqCase:
     """batch 30720, s_q = 1, s_kv uniform over {2,4,6,8,12,16}, 16 heads,
