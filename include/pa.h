@@ -196,6 +196,51 @@ pa_status pa_attention_varlen_spans(const void* q, const void* k_cache, const vo
                                     size_t workspace_bytes, void* stream);
 
 /*
+ * Element type of q, k, v, the caches and out in the _ex entry points.
+ */
+typedef enum { PA_DTYPE_BF16 = 0, PA_DTYPE_FP16 = 1 } pa_dtype;
+
+/*
+ * pa_write_kv_ex — pa_write_kv with an explicit cache block stride and dtype.
+ *
+ * The cache layouts of vllm-spyre PR #853 "Pytorch Native Attention on
+ * Spyre" (its code moves from separate K and V caches to one tensor shaped
+ * (num_blocks, 2, block_size, Hkv, D)) differ only in the distance between
+ * consecutive blocks: slot s of block b is row s of
+ *     k_cache + b * block_stride   (and v_cache + b * block_stride),
+ * each row [Hkv, D] contiguous.  Separate caches: block_stride =
+ * block_size * Hkv * D (or 0, which means that).  One combined tensor KV:
+ * k_cache = &KV[0][0], v_cache = &KV[0][1], block_stride = 2 * block_size *
+ * Hkv * D.
+ *  block_stride  elements; 0, or >= block_size * Hkv * D and a multiple of 8
+ *  dtype         PA_DTYPE_BF16 or PA_DTYPE_FP16 (a bit copy either way)
+ * Other arguments and errors as pa_write_kv.
+ */
+pa_status pa_write_kv_ex(const void* k, const void* v, const int64_t* slot_mapping,
+                         int64_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                         void* k_cache, void* v_cache, int64_t num_blocks, int32_t block_size,
+                         int64_t block_stride, int32_t dtype, void* workspace, void* stream);
+
+/*
+ * pa_attention_varlen_ex — the general varlen entry point: cache block stride
+ * (see pa_write_kv_ex), element type, and optional full-attention spans
+ * (span_offsets NULL: none, and causal applies; otherwise as
+ * pa_attention_varlen_spans, and causal is ignored).  pa_attention_varlen and
+ * pa_attention_varlen_spans are this call with block_stride 0, bf16.
+ * Returns PA_ERR_UNSUPPORTED for a dtype the build does not run.
+ */
+pa_status pa_attention_varlen_ex(const void* q, const void* k_cache, const void* v_cache,
+                                 const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                 const int32_t* seq_lens, const int32_t* query_start_loc,
+                                 int32_t num_seqs, int64_t num_q_tokens,
+                                 int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                 int32_t block_size, int64_t num_blocks, int64_t block_stride,
+                                 int32_t dtype, int32_t max_query_len, int32_t max_seq_len,
+                                 float scale, int32_t causal, const int32_t* span_offsets,
+                                 const int32_t* spans, int32_t num_spans, void* out,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * pa_attention_varlen_static — pa_attention_varlen for callers that cannot
  * allocate device memory.  This is an addition of this library: the pages it
  * follows have no counterpart.

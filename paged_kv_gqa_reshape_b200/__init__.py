@@ -29,7 +29,7 @@ __all__ = [
     "varlen_workspace_size", "varlen_workspace", "error_workspace", "get_error",
     "status_string", "version", "EXPORTED_SYMBOLS",
     "DEVERR_SLOT", "DEVERR_BLOCK", "DEVERR_LENGTHS", "DEVERR_QLEN", "DEVERR_HINT",
-    "DEVERR_TIMEOUT", "DEVERR_SPANS", "ERROR_WORD_BYTES",
+    "DEVERR_TIMEOUT", "DEVERR_SPANS", "ERROR_WORD_BYTES", "DTYPE_BF16", "DTYPE_FP16",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -43,8 +43,10 @@ STATIC_SCRATCH_BYTES = 32 << 20  # PA_STATIC_SCRATCH_BYTES
 EXPORTED_SYMBOLS = (
     "pa_write_kv", "pa_attention_varlen_workspace_size", "pa_attention_varlen",
     "pa_attention_smallseq", "pa_get_error", "pa_status_string", "pa_version",
-    "pa_attention_varlen_static", "pa_attention_varlen_spans",
+    "pa_attention_varlen_static", "pa_attention_varlen_spans", "pa_write_kv_ex",
+    "pa_attention_varlen_ex",
 )
+DTYPE_BF16, DTYPE_FP16 = 0, 1
 
 _lib = None
 _lock = threading.Lock()
@@ -92,6 +94,12 @@ def load(build_if_missing: bool = True):
         lib.pa_attention_varlen_static.argtypes = [
             p, p, p, p, i32, p, p, i32, i64, i32, i32, i32, i32, i64, i32, i32,
             ctypes.c_float, i32, p, p]
+        lib.pa_write_kv_ex.restype = ctypes.c_int
+        lib.pa_write_kv_ex.argtypes = [p, p, p, i64, i32, i32, p, p, i64, i32, i64, i32, p, p]
+        lib.pa_attention_varlen_ex.restype = ctypes.c_int
+        lib.pa_attention_varlen_ex.argtypes = [
+            p, p, p, p, i32, p, p, i32, i64, i32, i32, i32, i32, i64, i64, i32, i32, i32,
+            ctypes.c_float, i32, p, p, i32, p, p, ctypes.c_size_t, p]
         lib.pa_attention_varlen_spans.restype = ctypes.c_int
         lib.pa_attention_varlen_spans.argtypes = [
             p, p, p, p, i32, p, p, i32, i64, i32, i32, i32, i32, i64, i32, i32,
@@ -160,62 +168,115 @@ def varlen_workspace(num_seqs, num_q_tokens, num_q_heads, num_kv_heads, head_dim
     return torch.zeros(max(n, ERROR_WORD_BYTES), dtype=torch.uint8, device=device or "cuda")
 
 
+_DTYPES = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_FP16}
+
+
+def _element_dtype(t, name):
+    if t.dtype not in _DTYPES:
+        raise TypeError(f"{name} must be bfloat16 or float16, got {t.dtype}")
+    return t.dtype
+
+
+def _check_caches(k_cache, v_cache, dtype):
+    """Caches [NB, BS, Hkv, D] whose rows are contiguous and whose blocks are
+    block_stride elements apart (views of one [NB, 2, BS, Hkv, D] tensor are
+    fine).  Returns block_stride."""
+    for t, name in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        if not isinstance(t, torch.Tensor) or t.dtype != dtype:
+            raise TypeError(f"{name} must be a {dtype} tensor")
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if t.dim() != 4:
+            raise ValueError(f"{name} must have 4 dims [NB, BS, Hkv, D]")
+        nb, bs, hkv, d = t.shape
+        if t.stride(3) != 1 or t.stride(2) != d or t.stride(1) != hkv * d or t.stride(0) < bs * hkv * d:
+            raise ValueError(f"{name}: rows must be contiguous [BS, Hkv, D] blocks")
+    if v_cache.shape != k_cache.shape or v_cache.stride() != k_cache.stride():
+        raise ValueError("k_cache and v_cache must have the same shape and strides")
+    return k_cache.stride(0)
+
+
 def write_kv(k, v, slot_mapping, k_cache, v_cache, workspace=None, stream=None):
-    """Scatter k/v [T, Hkv, D] into the paged caches at slot_mapping (int64 [T])."""
-    _check(k, "k", torch.bfloat16, 3)
-    _check(v, "v", torch.bfloat16, 3)
+    """Scatter k/v [T, Hkv, D] into the paged caches at slot_mapping (int64 [T]).
+
+    k_cache / v_cache: [NB, BS, Hkv, D], bf16 or fp16 like k and v; separate
+    tensors, or the two halves kv[:, 0] / kv[:, 1] of one [NB, 2, BS, Hkv, D]
+    cache.
+    """
+    dt = _element_dtype(k, "k")
+    _check(k, "k", dt, 3)
+    _check(v, "v", dt, 3)
     _check(slot_mapping, "slot_mapping", torch.int64, 1)
-    _check(k_cache, "k_cache", torch.bfloat16, 4)
-    _check(v_cache, "v_cache", torch.bfloat16, 4)
+    stride = _check_caches(k_cache, v_cache, dt)
     t, hkv, d = k.shape
     if v.shape != k.shape or slot_mapping.shape[0] != t:
         raise ValueError("k, v and slot_mapping disagree on the token count / shape")
     nb, bs, hkv_c, d_c = k_cache.shape
-    if v_cache.shape != k_cache.shape or hkv_c != hkv or d_c != d:
+    if hkv_c != hkv or d_c != d:
         raise ValueError("cache shape does not match k/v")
     ws = workspace.data_ptr() if workspace is not None else None
-    st = load().pa_write_kv(k.data_ptr(), v.data_ptr(), slot_mapping.data_ptr(), t, hkv, d,
-                            k_cache.data_ptr(), v_cache.data_ptr(), nb, bs, ws, _stream(stream))
-    _raise(st, "pa_write_kv")
+    st = load().pa_write_kv_ex(k.data_ptr(), v.data_ptr(), slot_mapping.data_ptr(), t, hkv, d,
+                               k_cache.data_ptr(), v_cache.data_ptr(), nb, bs, stride,
+                               _DTYPES[dt], ws, _stream(stream))
+    _raise(st, "pa_write_kv_ex")
 
 
-def attention_varlen(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc,
-                     num_kv_heads, scale, causal, out, max_query_len=None, max_seq_len=None,
-                     workspace=None, stream=None):
-    """Paged varlen attention; writes out [T, Hq, D] (bf16).
-
-    max_query_len / max_seq_len are host-side hints (the metadata builder's
-    maxima); when omitted the safe bounds (all tokens / the block table's
-    reach) are used, which never forces a device synchronisation.
-    """
-    _check(q, "q", torch.bfloat16, 3)
-    _check(k_cache, "k_cache", torch.bfloat16, 4)
-    _check(v_cache, "v_cache", torch.bfloat16, 4)
+def _varlen_ex(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc, num_kv_heads,
+               scale, causal, span_offsets, spans, out, max_query_len, max_seq_len, workspace,
+               stream, what):
+    dt = _element_dtype(q, "q")
+    _check(q, "q", dt, 3)
+    stride = _check_caches(k_cache, v_cache, dt)
     _check(block_tables, "block_tables", torch.int32, 2)
     _check(seq_lens, "seq_lens", torch.int32, 1)
     _check(query_start_loc, "query_start_loc", torch.int32, 1)
-    _check(out, "out", torch.bfloat16, 3)
+    _check(out, "out", dt, 3)
     t, hq, d = q.shape
     nb, bs, hkv, d_c = k_cache.shape
-    if hkv != num_kv_heads or d_c != d or v_cache.shape != k_cache.shape:
+    if hkv != num_kv_heads or d_c != d:
         raise ValueError("cache shape does not match q / num_kv_heads")
     if out.shape != q.shape:
         raise ValueError("out must have q's shape")
     s = seq_lens.shape[0]
     if query_start_loc.shape[0] != s + 1 or block_tables.shape[0] != s:
         raise ValueError("seq_lens, query_start_loc and block_tables disagree on num_seqs")
+    so_ptr, sp_ptr, n_spans = None, None, 0
+    if span_offsets is not None:
+        _check(span_offsets, "span_offsets", torch.int32, 1)
+        _check(spans, "spans", torch.int32, 2)
+        if span_offsets.shape[0] != s + 1 or (spans.numel() and spans.shape[1] != 2):
+            raise ValueError("span_offsets must be [S+1] and spans [N, 2]")
+        n_spans = spans.shape[0] if spans.numel() else 0
+        so_ptr = span_offsets.data_ptr()
+        sp_ptr = spans.data_ptr() if n_spans else None
     mb = block_tables.shape[1]
     mql = t if max_query_len is None else int(max_query_len)
     msl = mb * bs if max_seq_len is None else int(max_seq_len)
     if workspace is None:
         workspace = varlen_workspace(s, t, hq, hkv, d, device=q.device)
-    st = load().pa_attention_varlen(
+    st = load().pa_attention_varlen_ex(
         q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(), mb,
-        seq_lens.data_ptr(), query_start_loc.data_ptr(), s, t, hq, hkv, d, bs, nb, mql, msl,
-        float(scale), int(bool(causal)), out.data_ptr(), workspace.data_ptr(),
-        workspace.numel() * workspace.element_size(), _stream(stream))
-    _raise(st, "pa_attention_varlen")
+        seq_lens.data_ptr(), query_start_loc.data_ptr(), s, t, hq, hkv, d, bs, nb, stride,
+        _DTYPES[dt], mql, msl, float(scale), int(bool(causal)), so_ptr, sp_ptr, n_spans,
+        out.data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    _raise(st, what)
     return out
+
+
+def attention_varlen(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc,
+                     num_kv_heads, scale, causal, out, max_query_len=None, max_seq_len=None,
+                     workspace=None, stream=None):
+    """Paged varlen attention; writes out [T, Hq, D] (q's dtype).
+
+    max_query_len / max_seq_len are host-side hints (the metadata builder's
+    maxima); when omitted the safe bounds (all tokens / the block table's
+    reach) are used, which never forces a device synchronisation.  The caches
+    may be separate tensors or the halves of one [NB, 2, BS, Hkv, D] cache.
+    """
+    return _varlen_ex(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc,
+                      num_kv_heads, scale, causal, None, None, out, max_query_len, max_seq_len,
+                      workspace, stream, "pa_attention_varlen_ex")
 
 
 def attention_varlen_spans(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc,
@@ -226,42 +287,13 @@ def attention_varlen_spans(q, k_cache, v_cache, block_tables, seq_lens, query_st
     span_offsets: int32 [S+1] (sequence s owns spans span_offsets[s] ..
     span_offsets[s+1]-1); spans: int32 [N, 2] (start, end) key positions.
     A query whose key position lies in a span [start, end) sees keys
-    0 .. end-1; every other query is causal.  Writes out [T, Hq, D] (bf16).
+    0 .. end-1; every other query is causal.  Writes out [T, Hq, D].
     """
-    _check(q, "q", torch.bfloat16, 3)
-    _check(k_cache, "k_cache", torch.bfloat16, 4)
-    _check(v_cache, "v_cache", torch.bfloat16, 4)
-    _check(block_tables, "block_tables", torch.int32, 2)
-    _check(seq_lens, "seq_lens", torch.int32, 1)
-    _check(query_start_loc, "query_start_loc", torch.int32, 1)
-    _check(span_offsets, "span_offsets", torch.int32, 1)
-    _check(spans, "spans", torch.int32, 2)
-    _check(out, "out", torch.bfloat16, 3)
-    t, hq, d = q.shape
-    nb, bs, hkv, d_c = k_cache.shape
-    if hkv != num_kv_heads or d_c != d or v_cache.shape != k_cache.shape:
-        raise ValueError("cache shape does not match q / num_kv_heads")
-    if out.shape != q.shape:
-        raise ValueError("out must have q's shape")
-    s = seq_lens.shape[0]
-    if query_start_loc.shape[0] != s + 1 or block_tables.shape[0] != s:
-        raise ValueError("seq_lens, query_start_loc and block_tables disagree on num_seqs")
-    if span_offsets.shape[0] != s + 1 or (spans.numel() and spans.shape[1] != 2):
-        raise ValueError("span_offsets must be [S+1] and spans [N, 2]")
-    mb = block_tables.shape[1]
-    mql = t if max_query_len is None else int(max_query_len)
-    msl = mb * bs if max_seq_len is None else int(max_seq_len)
-    if workspace is None:
-        workspace = varlen_workspace(s, t, hq, hkv, d, device=q.device)
-    n_spans = spans.shape[0] if spans.numel() else 0
-    st = load().pa_attention_varlen_spans(
-        q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(), mb,
-        seq_lens.data_ptr(), query_start_loc.data_ptr(), s, t, hq, hkv, d, bs, nb, mql, msl,
-        float(scale), span_offsets.data_ptr(), spans.data_ptr() if n_spans else None, n_spans,
-        out.data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-        _stream(stream))
-    _raise(st, "pa_attention_varlen_spans")
-    return out
+    if span_offsets is None or spans is None:
+        raise ValueError("span_offsets and spans are required")
+    return _varlen_ex(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc,
+                      num_kv_heads, scale, True, span_offsets, spans, out, max_query_len,
+                      max_seq_len, workspace, stream, "pa_attention_varlen_ex")
 
 
 def attention_varlen_static(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc,

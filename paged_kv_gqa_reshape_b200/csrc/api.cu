@@ -108,9 +108,21 @@ pa_status pa_write_kv(const void* k, const void* v, const int64_t* slot_mapping,
                       int64_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
                       void* k_cache, void* v_cache, int64_t num_blocks, int32_t block_size,
                       void* workspace, void* stream) {
+  return pa_write_kv_ex(k, v, slot_mapping, num_tokens, num_kv_heads, head_dim, k_cache, v_cache,
+                        num_blocks, block_size, 0, PA_DTYPE_BF16, workspace, stream);
+}
+
+pa_status pa_write_kv_ex(const void* k, const void* v, const int64_t* slot_mapping,
+                         int64_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                         void* k_cache, void* v_cache, int64_t num_blocks, int32_t block_size,
+                         int64_t block_stride, int32_t dtype, void* workspace, void* stream) {
   if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || head_dim % 8 != 0 ||
       num_blocks <= 0 || block_size <= 0)
     return PA_ERR_INVALID_ARG;
+  if (dtype != PA_DTYPE_BF16 && dtype != PA_DTYPE_FP16) return PA_ERR_INVALID_ARG;
+  const int64_t block_elems = (int64_t)block_size * num_kv_heads * head_dim;
+  if (block_stride == 0) block_stride = block_elems;
+  if (block_stride < block_elems || block_stride % 8 != 0) return PA_ERR_INVALID_ARG;
   if (num_tokens == 0) return PA_OK;
   if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PA_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
@@ -119,7 +131,8 @@ pa_status pa_write_kv(const void* k, const void* v, const int64_t* slot_mapping,
   const int row_vecs = num_kv_heads * head_dim / 8;
   uint32_t* err = workspace ? static_cast<uint32_t*>(workspace) : nullptr;
   cudaError_t e = pa::launch_write_kv(k, v, slot_mapping, num_tokens, row_vecs, k_cache, v_cache,
-                                      num_blocks * (int64_t)block_size, err, sm_count(),
+                                      num_blocks * (int64_t)block_size, block_size,
+                                      block_stride / 8, err, sm_count(),
                                       static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
@@ -140,11 +153,14 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
                                 const int32_t* seq_lens, const int32_t* query_start_loc,
                                 int32_t num_seqs, int64_t num_q_tokens, int32_t num_q_heads,
                                 int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
-                                int64_t num_blocks, int32_t max_query_len, int32_t max_seq_len,
+                                int64_t num_blocks, int64_t block_stride, int32_t dtype,
+                                int32_t max_query_len, int32_t max_seq_len,
                                 float scale, int32_t causal, const int32_t* span_offsets,
                                 const int32_t* spans, int32_t num_spans, void* out,
                                 void* workspace, size_t workspace_bytes, void* stream) {
   // ---- host-visible checks (nothing launched yet) ----
+  if (dtype != PA_DTYPE_BF16 && dtype != PA_DTYPE_FP16) return PA_ERR_INVALID_ARG;
+  if (dtype != PA_DTYPE_BF16) return PA_ERR_UNSUPPORTED;
   if (num_seqs < 0 || num_q_tokens < 0 || num_q_tokens > 0x7fffffffll || num_q_heads <= 0 ||
       num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || max_blocks_per_seq <= 0 ||
       num_blocks <= 0 || num_blocks > 0x7fffffffll || max_query_len < 0 || max_seq_len < 0 ||
@@ -167,6 +183,9 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
       (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
       (reinterpret_cast<uintptr_t>(query_start_loc) & 3u))
     return PA_ERR_INVALID_ARG;
+  const int64_t block_elems = (int64_t)block_size * num_kv_heads * head_dim;
+  if (block_stride == 0) block_stride = block_elems;
+  if (block_stride < block_elems || block_stride % 8 != 0) return PA_ERR_INVALID_ARG;
   const WorkspaceLayout L =
       pa::make_layout(num_seqs, num_q_tokens, num_q_heads, num_kv_heads, head_dim);
   if (workspace_bytes < L.total) return PA_ERR_INVALID_ARG;
@@ -187,7 +206,7 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
     const cuuint64_t dkv[4] = {(cuuint64_t)head_dim, (cuuint64_t)num_kv_heads,
                                (cuuint64_t)block_size, (cuuint64_t)num_blocks};
     const cuuint64_t skv[3] = {(cuuint64_t)head_dim * 2, (cuuint64_t)num_kv_heads * head_dim * 2,
-                               (cuuint64_t)block_size * num_kv_heads * head_dim * 2};
+                               (cuuint64_t)block_stride * 2};
     if (!make_map(&q_map, q, 3, dq, sq, box_q) || !make_map(&k_map, k_cache, 4, dkv, skv, box_kv) ||
         !make_map(&v_map, v_cache, 4, dkv, skv, box_kv))
       return PA_ERR_CUDA;
@@ -243,6 +262,7 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
   dp.num_kv_heads = num_kv_heads;
   dp.group = group;
   dp.num_blocks = num_blocks;
+  dp.block_stride = block_stride;
   dp.scale_log2 = scale_log2;
   dp.out = static_cast<__nv_bfloat16*>(out);
   dp.ws = ws;
@@ -266,8 +286,9 @@ pa_status pa_attention_varlen(const void* q, const void* k_cache, const void* v_
                               size_t workspace_bytes, void* stream) {
   return attention_varlen_impl(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
                                query_start_loc, num_seqs, num_q_tokens, num_q_heads, num_kv_heads,
-                               head_dim, block_size, num_blocks, max_query_len, max_seq_len, scale,
-                               causal, nullptr, nullptr, 0, out, workspace, workspace_bytes, stream);
+                               head_dim, block_size, num_blocks, 0, PA_DTYPE_BF16, max_query_len,
+                               max_seq_len, scale, causal, nullptr, nullptr, 0, out, workspace,
+                               workspace_bytes, stream);
 }
 
 pa_status pa_attention_varlen_spans(const void* q, const void* k_cache, const void* v_cache,
@@ -282,9 +303,26 @@ pa_status pa_attention_varlen_spans(const void* q, const void* k_cache, const vo
   if (!span_offsets && num_seqs > 0) return PA_ERR_INVALID_ARG;
   return attention_varlen_impl(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
                                query_start_loc, num_seqs, num_q_tokens, num_q_heads, num_kv_heads,
-                               head_dim, block_size, num_blocks, max_query_len, max_seq_len, scale,
-                               1, span_offsets, spans, num_spans, out, workspace, workspace_bytes,
-                               stream);
+                               head_dim, block_size, num_blocks, 0, PA_DTYPE_BF16, max_query_len,
+                               max_seq_len, scale, 1, span_offsets, spans, num_spans, out, workspace,
+                               workspace_bytes, stream);
+}
+
+pa_status pa_attention_varlen_ex(const void* q, const void* k_cache, const void* v_cache,
+                                 const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                 const int32_t* seq_lens, const int32_t* query_start_loc,
+                                 int32_t num_seqs, int64_t num_q_tokens, int32_t num_q_heads,
+                                 int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                 int64_t num_blocks, int64_t block_stride, int32_t dtype,
+                                 int32_t max_query_len, int32_t max_seq_len, float scale,
+                                 int32_t causal, const int32_t* span_offsets, const int32_t* spans,
+                                 int32_t num_spans, void* out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  return attention_varlen_impl(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                               query_start_loc, num_seqs, num_q_tokens, num_q_heads, num_kv_heads,
+                               head_dim, block_size, num_blocks, block_stride, dtype, max_query_len,
+                               max_seq_len, scale, span_offsets ? 1 : causal, span_offsets, spans,
+                               num_spans, out, workspace, workspace_bytes, stream);
 }
 
 pa_status pa_attention_smallseq(const void* q, const void* k, const void* v,

@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
         p.block_tables[(size_t)seq_p * p.max_blocks_per_seq + (x_p - p_first)];
     const bool block_ok = block >= 0 && block < p.num_blocks;
     if (!block_ok && tid == 0) raise_error(err, PA_DEVERR_BLOCK);
-    const size_t base = ((size_t)(block_ok ? block : 0) * kPageKeys * Hkv + (size_t)hg * HPC) * D;
+    const size_t base = (size_t)(block_ok ? block : 0) * p.block_stride + (size_t)hg * HPC * D;
     __nv_bfloat16* kdst = ring + (size_t)stage * 2 * Shape::kTensorStage;
     __nv_bfloat16* vdst = kdst + Shape::kTensorStage;
 #pragma unroll

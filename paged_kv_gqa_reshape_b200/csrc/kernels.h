@@ -13,7 +13,8 @@ namespace pa {
 // ---- KV scatter ------------------------------------------------------------
 cudaError_t launch_write_kv(const void* k, const void* v, const int64_t* slot_mapping,
                             int64_t num_tokens, int row_vecs, void* k_cache, void* v_cache,
-                            int64_t num_slots, uint32_t* err, int num_sms, cudaStream_t stream);
+                            int64_t num_slots, int block_size, int64_t block_vecs, uint32_t* err,
+                            int num_sms, cudaStream_t stream);
 
 // ---- plan ------------------------------------------------------------------
 void launch_plan(const int32_t* query_start_loc, const int32_t* seq_lens, int num_seqs,
@@ -39,6 +40,7 @@ struct DecodeParams {
   int num_kv_heads;
   int group;  // num_q_heads / num_kv_heads, <= 16
   long long num_blocks;
+  long long block_stride;  // elements between consecutive cache blocks
   float scale_log2;  // scale * log2(e)
   int self_plan;     // 1: every CTA plans the decode work itself (num_seqs <= kSelfPlanMaxSeqs)
   __nv_bfloat16* out;

@@ -18,7 +18,8 @@ __global__ void __launch_bounds__(256) write_kv_kernel(const uint4* __restrict__
                                                        long long num_tokens, int row_vecs,
                                                        uint4* __restrict__ k_cache,
                                                        uint4* __restrict__ v_cache,
-                                                       long long num_slots, uint32_t* err) {
+                                                       long long num_slots, int block_size,
+                                                       long long block_vecs, uint32_t* err) {
   const int lane = threadIdx.x & 31;
   const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
   for (long long t = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -31,8 +32,10 @@ __global__ void __launch_bounds__(256) write_kv_kernel(const uint4* __restrict__
     }
     const uint4* ks = k + t * row_vecs;
     const uint4* vs = v + t * row_vecs;
-    uint4* kd = k_cache + slot * row_vecs;
-    uint4* vd = v_cache + slot * row_vecs;
+    // block slot / block_size, row slot % block_size (blocks block_vecs apart)
+    const long long at = (slot / block_size) * block_vecs + (slot % block_size) * row_vecs;
+    uint4* kd = k_cache + at;
+    uint4* vd = v_cache + at;
     // issue all loads of this lane before its stores (row_vecs <= 32 * 8 here)
     constexpr int kMaxPerLane = 8;
     uint4 kr[kMaxPerLane], vr[kMaxPerLane];
@@ -62,7 +65,8 @@ __global__ void __launch_bounds__(256) write_kv_kernel(const uint4* __restrict__
 
 cudaError_t launch_write_kv(const void* k, const void* v, const int64_t* slot_mapping,
                             int64_t num_tokens, int row_vecs, void* k_cache, void* v_cache,
-                            int64_t num_slots, uint32_t* err, int num_sms, cudaStream_t stream) {
+                            int64_t num_slots, int block_size, int64_t block_vecs, uint32_t* err,
+                            int num_sms, cudaStream_t stream) {
   if (num_tokens <= 0) return cudaSuccess;
   const int threads = 256;
   const long long warps_needed = num_tokens;
@@ -71,7 +75,8 @@ cudaError_t launch_write_kv(const void* k, const void* v, const int64_t* slot_ma
   if (blocks > cap) blocks = cap;
   write_kv_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
       static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping, num_tokens,
-      row_vecs, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), num_slots, err);
+      row_vecs, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), num_slots, block_size,
+      block_vecs, err);
   return cudaGetLastError();
 }
 

@@ -101,6 +101,33 @@ def test_varlen_spans_empty_batch_is_a_no_op():
     assert _spans(pa.load(), T=0) == 0
 
 
+def test_ex_entry_points_check_stride_and_dtype():
+    lib = pa.load()
+    base = dict(k=1 << 12, v=1 << 12, sm=1 << 12, T=4, Hkv=2, D=64, kc=1 << 12, vc=1 << 12,
+                NB=8, BS=16, stride=0, dtype=0, ws=None, stream=None)
+
+    def wkv(**over):
+        a = dict(base)
+        a.update(over)
+        return lib.pa_write_kv_ex(*a.values())
+    assert wkv(stride=16 * 2 * 64 - 8) == 1        # smaller than one block
+    assert wkv(stride=2 * 16 * 2 * 64 + 4) == 1    # not a multiple of 8 elements
+    assert wkv(dtype=7) == 1
+    assert wkv(T=0) == 0
+    args = dict(q=1 << 12, kc=1 << 12, vc=1 << 12, bt=1 << 12, mb=4, sl=1 << 12, qsl=1 << 12,
+                S=2, T=4, Hq=4, Hkv=2, D=64, BS=16, NB=8, stride=0, dtype=0, mql=4, msl=64,
+                scale=0.125, causal=1, so=None, sp=None, nsp=0, out=1 << 12, ws=1 << 12,
+                wsb=1 << 30, stream=None)
+
+    def var(**over):
+        a = dict(args)
+        a.update(over)
+        return lib.pa_attention_varlen_ex(*a.values())
+    assert var(stride=100) == 1
+    assert var(dtype=5) == 1
+    assert var(S=0) == 0
+
+
 def test_write_kv_rejects_before_launch():
     lib = pa.load()
     ok = dict(k=1 << 12, v=1 << 12, sm=1 << 12, T=3, Hkv=2, D=64, kc=1 << 12, vc=1 << 12,
