@@ -64,6 +64,13 @@ def _load():
         lib.oracle_attention_weights.restype = i64
         lib.oracle_attention_weights.argtypes = [
             p, p, p, p, p, p, i32, i32, i32, i32, f64, i32, i64, i32, p]
+        lib.oracle_attention_varlen_dtype.restype = i32
+        lib.oracle_attention_varlen_dtype.argtypes = [
+            p, p, p, p, p, p, i32, i32, i32, i32, f64, i32, i32, p, i64, p]
+        lib.oracle_attention_smallseq_dtype.restype = i32
+        lib.oracle_attention_smallseq_dtype.argtypes = [p, p, p, p, i32, i32, i32, i32, f64, i32, p]
+        lib.oracle_widen.restype = f64
+        lib.oracle_widen.argtypes = [ctypes.c_uint16, i32]
         lib.oracle_attention_smallseq.restype = i32
         lib.oracle_attention_smallseq.argtypes = [p, p, p, p, i32, i32, i32, i32, f64, p]
         _lib = lib
@@ -119,6 +126,45 @@ def attention_varlen(q, k_seq, v_seq, kv_offsets, seq_lens, query_start_loc,
     if rc != 0:
         raise ValueError(f"oracle_attention_varlen failed ({rc})")
     return out
+
+
+def attention_varlen_dtype(q, k_seq, v_seq, kv_offsets, seq_lens, query_start_loc,
+                           num_kv_heads, scale, causal, dtype, rows=None):
+    """attention_varlen for dtype 0 (bf16 bits) or 1 (fp16 bits)."""
+    q = _arr(q, np.uint16)
+    k_seq, v_seq = _arr(k_seq, np.uint16), _arr(v_seq, np.uint16)
+    kv_offsets = _arr(kv_offsets, np.int64)
+    seq_lens = _arr(seq_lens, np.int32)
+    qsl = _arr(query_start_loc, np.int32)
+    t, hq, d = q.shape
+    out = np.zeros((t, hq, d), dtype=np.float64)
+    rows_a = None if rows is None else _arr(rows, np.int64)
+    rc = _load().oracle_attention_varlen_dtype(
+        _ptr(q), _ptr(k_seq), _ptr(v_seq), _ptr(kv_offsets), _ptr(seq_lens), _ptr(qsl),
+        len(seq_lens), hq, num_kv_heads, d, float(scale), int(bool(causal)), int(dtype),
+        _ptr(rows_a), 0 if rows_a is None else len(rows_a), _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_attention_varlen_dtype failed ({rc})")
+    return out
+
+
+def smallseq_dtype(q, k, v, cu_seqlens_kv, num_kv_heads, scale, dtype):
+    """attention_smallseq for dtype 0 (bf16 bits) or 1 (fp16 bits)."""
+    q, k, v = _arr(q, np.uint16), _arr(k, np.uint16), _arr(v, np.uint16)
+    cu = _arr(cu_seqlens_kv, np.int32)
+    b, hq, d = q.shape
+    out = np.zeros((b, hq, d), dtype=np.float64)
+    rc = _load().oracle_attention_smallseq_dtype(_ptr(q), _ptr(k), _ptr(v), _ptr(cu), b, hq,
+                                                 num_kv_heads, d, float(scale), int(dtype),
+                                                 _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_attention_smallseq_dtype failed ({rc})")
+    return out
+
+
+def widen(bits: int, dtype: int) -> float:
+    """One 16-bit pattern widened to float (0 = bf16, 1 = fp16)."""
+    return _load().oracle_widen(int(bits), int(dtype))
 
 
 def attention_varlen_spans(q, k_seq, v_seq, kv_offsets, seq_lens, query_start_loc,

@@ -51,6 +51,11 @@
  *      small-seq", description: one query per batch entry (s_q = 1), keys and
  *      values packed in THD layout with cu_seqlens_kv, no causal mask.
  *
+ *  Element types: inputs are bfloat16 bit patterns, or IEEE binary16 (fp16)
+ *      bit patterns in the _dtype variants (vllm-spyre PR #853 runs its path
+ *      in fp16; ROCm/TransformerEngine PR #461's small-seq path takes BF16
+ *      and FP16).  Both widen exactly to double.
+ *
  *  oracle_attention_weights
  *      The softmax weights of one (token, head) row, so that a test can check
  *      that they sum to one and that masked keys get none.
@@ -62,6 +67,21 @@
 #ifdef _OPENMP
 #include <omp.h>
 #endif
+
+/* IEEE binary16 (fp16): 1 sign, 5 exponent (bias 15), 10 fraction bits.
+   Every value is exact in double: subnormals are f * 2^-24, normals
+   (1024 + f) * 2^(e - 25); e == 31 is infinity or NaN. */
+static double half_to_double(uint16_t h) {
+    int sign = h >> 15, e = (h >> 10) & 0x1f, f = h & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -24);
+    else if (e == 31)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + f), e - 25);
+    return sign ? -v : v;
+}
 
 /* bfloat16 is the upper half of an IEEE binary32: widening is exact. */
 static double bf16_to_double(uint16_t bits) {
@@ -131,6 +151,7 @@ typedef struct {
     int kv_head;
     int num_kv_heads;
     int head_dim;
+    double (*widen)(uint16_t);  /* element type: bf16_to_double or half_to_double */
 } kv_view;
 
 /* Pointer to the head_dim values of key/value j, or NULL if its block id is
@@ -197,7 +218,7 @@ static int attention_row(const uint16_t *q, const kv_view *keys,
         if (!kr) return -1;
         double dot = 0.0;
         for (int d = 0; d < head_dim; ++d)
-            dot += bf16_to_double(q[d]) * bf16_to_double(kr[d]);
+            dot += keys->widen(q[d]) * keys->widen(kr[d]);
         s[j] = scale * dot;
         if (s[j] > m) m = s[j];
     }
@@ -211,7 +232,7 @@ static int attention_row(const uint16_t *q, const kv_view *keys,
         if (!vr) return -1;
         double w = s[j] / denom;
         if (weights) weights[j] = w;
-        for (int d = 0; d < head_dim; ++d) out[d] += w * bf16_to_double(vr[d]);
+        for (int d = 0; d < head_dim; ++d) out[d] += w * values->widen(vr[d]);
     }
     return 0;
 }
@@ -233,8 +254,9 @@ static int varlen_driver(const uint16_t *q, const uint16_t *k_base,
                          const int32_t *seq_lens, const int32_t *query_start_loc,
                          int num_seqs, int num_q_heads, int num_kv_heads,
                          int head_dim, double scale, int causal,
-                         const int32_t *span_offsets, const int32_t *spans,
+                         const int32_t *span_offsets, const int32_t *spans, int dtype,
                          const int64_t *rows, int64_t num_rows, double *out) {
+    double (*widen)(uint16_t) = dtype == 1 ? half_to_double : bf16_to_double;
     if (num_kv_heads <= 0 || num_q_heads <= 0 || num_q_heads % num_kv_heads != 0)
         return -1;
     int group = num_q_heads / num_kv_heads;
@@ -268,6 +290,7 @@ static int varlen_driver(const uint16_t *q, const uint16_t *k_base,
                 kview.num_kv_heads = vview.num_kv_heads = num_kv_heads;
                 kview.head_dim = vview.head_dim = head_dim;
                 kview.kv_head = vview.kv_head = h / group;
+                kview.widen = vview.widen = widen;
                 kview.base = k_base;
                 vview.base = v_base;
                 if (block_tables) {
@@ -312,7 +335,24 @@ int oracle_attention_varlen(const uint16_t *q, const uint16_t *k_seq,
                             int64_t num_rows, double *out) {
     return varlen_driver(q, k_seq, v_seq, kv_offsets, NULL, 0, 1, 0, seq_lens,
                          query_start_loc, num_seqs, num_q_heads, num_kv_heads,
-                         head_dim, scale, causal, NULL, NULL, rows, num_rows, out);
+                         head_dim, scale, causal, NULL, NULL, 0, rows, num_rows, out);
+}
+
+/*
+ * Logical form with an element type: dtype 0 = bf16, 1 = fp16 (every input
+ * is that type's bit pattern); otherwise as oracle_attention_varlen.
+ */
+int oracle_attention_varlen_dtype(const uint16_t *q, const uint16_t *k_seq,
+                                  const uint16_t *v_seq, const int64_t *kv_offsets,
+                                  const int32_t *seq_lens,
+                                  const int32_t *query_start_loc, int num_seqs,
+                                  int num_q_heads, int num_kv_heads, int head_dim,
+                                  double scale, int causal, int dtype, const int64_t *rows,
+                                  int64_t num_rows, double *out) {
+    if (dtype != 0 && dtype != 1) return -1;
+    return varlen_driver(q, k_seq, v_seq, kv_offsets, NULL, 0, 1, 0, seq_lens,
+                         query_start_loc, num_seqs, num_q_heads, num_kv_heads,
+                         head_dim, scale, causal, NULL, NULL, dtype, rows, num_rows, out);
 }
 
 /*
@@ -332,7 +372,7 @@ int oracle_attention_varlen_spans(const uint16_t *q, const uint16_t *k_seq,
     if (!span_offsets || !spans) return -1;
     return varlen_driver(q, k_seq, v_seq, kv_offsets, NULL, 0, 1, 0, seq_lens,
                          query_start_loc, num_seqs, num_q_heads, num_kv_heads,
-                         head_dim, scale, 1, span_offsets, spans, rows, num_rows, out);
+                         head_dim, scale, 1, span_offsets, spans, 0, rows, num_rows, out);
 }
 
 /*
@@ -352,7 +392,7 @@ int oracle_attention_varlen_paged(const uint16_t *q, const uint16_t *k_cache,
     return varlen_driver(q, k_cache, v_cache, NULL, block_tables,
                          max_blocks_per_seq, block_size, num_blocks, seq_lens,
                          query_start_loc, num_seqs, num_q_heads, num_kv_heads,
-                         head_dim, scale, causal, NULL, NULL, rows, num_rows, out);
+                         head_dim, scale, causal, NULL, NULL, 0, rows, num_rows, out);
 }
 
 /*
@@ -375,6 +415,7 @@ int64_t oracle_attention_weights(const uint16_t *q, const uint16_t *k_seq,
     int64_t len_kv = seq_lens[s];
     int64_t n_vis = visible_keys(t - query_start_loc[s], len_q, len_kv, causal);
     kv_view kview = {0}, vview = {0};
+    kview.widen = vview.widen = bf16_to_double;
     kview.base = k_seq;
     vview.base = v_seq;
     kview.first_row = vview.first_row = kv_offsets[s];
@@ -403,11 +444,12 @@ int64_t oracle_attention_weights(const uint16_t *q, const uint16_t *k_seq,
  * No causal mask: every key of the entry is visible; an empty entry gives
  * zeros.  Returns 0, or -1 on bad head counts.
  */
-int oracle_attention_smallseq(const uint16_t *q, const uint16_t *k,
-                              const uint16_t *v, const int32_t *cu_seqlens_kv,
-                              int batch, int num_q_heads, int num_kv_heads,
-                              int head_dim, double scale, double *out) {
+static int smallseq_driver(const uint16_t *q, const uint16_t *k,
+                           const uint16_t *v, const int32_t *cu_seqlens_kv,
+                           int batch, int num_q_heads, int num_kv_heads,
+                           int head_dim, double scale, int dtype, double *out) {
     if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return -1;
+    double (*widen)(uint16_t) = dtype == 1 ? half_to_double : bf16_to_double;
     int group = num_q_heads / num_kv_heads;
     int64_t max_len = 1;
     for (int b = 0; b < batch; ++b) {
@@ -428,6 +470,7 @@ int oracle_attention_smallseq(const uint16_t *q, const uint16_t *k,
                 kview.kv_head = vview.kv_head = h / group;
                 kview.num_kv_heads = vview.num_kv_heads = num_kv_heads;
                 kview.head_dim = vview.head_dim = head_dim;
+                kview.widen = vview.widen = widen;
                 const uint16_t *qr = q + ((int64_t)b * num_q_heads + h) * head_dim;
                 double *o = out + ((int64_t)b * num_q_heads + h) * head_dim;
                 attention_row(qr, &kview, &vview, n, head_dim, scale, o, NULL,
@@ -437,4 +480,27 @@ int oracle_attention_smallseq(const uint16_t *q, const uint16_t *k,
         free(scratch);
     }
     return 0;
+}
+
+int oracle_attention_smallseq(const uint16_t *q, const uint16_t *k,
+                              const uint16_t *v, const int32_t *cu_seqlens_kv,
+                              int batch, int num_q_heads, int num_kv_heads,
+                              int head_dim, double scale, double *out) {
+    return smallseq_driver(q, k, v, cu_seqlens_kv, batch, num_q_heads, num_kv_heads,
+                           head_dim, scale, 0, out);
+}
+
+/* The same with an element type: dtype 0 = bf16, 1 = fp16. */
+int oracle_attention_smallseq_dtype(const uint16_t *q, const uint16_t *k,
+                                    const uint16_t *v, const int32_t *cu_seqlens_kv,
+                                    int batch, int num_q_heads, int num_kv_heads,
+                                    int head_dim, double scale, int dtype, double *out) {
+    if (dtype != 0 && dtype != 1) return -1;
+    return smallseq_driver(q, k, v, cu_seqlens_kv, batch, num_q_heads, num_kv_heads,
+                           head_dim, scale, dtype, out);
+}
+
+/* One element widened exactly (dtype 0 = bf16, 1 = fp16), for tests. */
+double oracle_widen(uint16_t bits, int dtype) {
+    return dtype == 1 ? half_to_double(bits) : bf16_to_double(bits);
 }

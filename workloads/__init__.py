@@ -107,14 +107,16 @@ def _gen(seed: int, device) -> torch.Generator:
     return g
 
 
-def _randn_bf16(shape, gen, device, chunk_rows: int = 1 << 20) -> torch.Tensor:
-    """N(0,1) fp32 rounded to bf16, drawn in row chunks to bound fp32 temporaries."""
-    out = torch.empty(shape, dtype=torch.bfloat16, device=device)
+def _randn_bf16(shape, gen, device, chunk_rows: int = 1 << 20,
+                dtype=torch.bfloat16) -> torch.Tensor:
+    """N(0,1) fp32 rounded to `dtype` (bf16 or fp16), drawn in row chunks to
+    bound fp32 temporaries."""
+    out = torch.empty(shape, dtype=dtype, device=device)
     flat = out.view(shape[0], -1) if len(shape) > 1 else out.view(-1, 1)
     for r0 in range(0, flat.shape[0], chunk_rows):
         r1 = min(flat.shape[0], r0 + chunk_rows)
         flat[r0:r1] = torch.randn((r1 - r0, flat.shape[1]), generator=gen,
-                                  device=device, dtype=torch.float32).to(torch.bfloat16)
+                                  device=device, dtype=torch.float32).to(dtype)
     return out
 
 
@@ -122,7 +124,7 @@ def build_varlen_case(name: str, seq_lens, query_lens, num_q_heads: int, num_kv_
                       head_dim: int, causal: bool, seed: int, device="cpu",
                       block_size: int = BLOCK_SIZE, pool_blocks: Optional[int] = None,
                       scale: Optional[float] = None, keep_logical: bool = True,
-                      spare_table_cols: int = 1) -> VarlenCase:
+                      spare_table_cols: int = 1, dtype=torch.bfloat16) -> VarlenCase:
     """Lay out one paged varlen batch.
 
     seq_lens[s] keys per sequence, of which the last query_lens[s] are this
@@ -156,9 +158,11 @@ def build_varlen_case(name: str, seq_lens, query_lens, num_q_heads: int, num_kv_
     total_kv = kv_offsets[-1]
 
     gen = _gen(seed + 7919, device)
-    k_log = _randn_bf16((max(total_kv, 1), num_kv_heads, head_dim), gen, device)[:total_kv]
-    v_log = _randn_bf16((max(total_kv, 1), num_kv_heads, head_dim), gen, device)[:total_kv]
-    q = _randn_bf16((max(T, 1), num_q_heads, head_dim), gen, device)[:T]
+    k_log = _randn_bf16((max(total_kv, 1), num_kv_heads, head_dim), gen, device,
+                        dtype=dtype)[:total_kv]
+    v_log = _randn_bf16((max(total_kv, 1), num_kv_heads, head_dim), gen, device,
+                        dtype=dtype)[:total_kv]
+    q = _randn_bf16((max(T, 1), num_q_heads, head_dim), gen, device, dtype=dtype)[:T]
 
     # logical row of every key, its slot, and whether it is this step's token
     table_dev = table.to(device)
@@ -172,9 +176,9 @@ def build_varlen_case(name: str, seq_lens, query_lens, num_q_heads: int, num_kv_
     is_new = pos_of_row >= new_from[seq_of_row]
 
     k_cache = torch.full((pool, block_size, num_kv_heads, head_dim), K_SENTINEL,
-                         dtype=torch.bfloat16, device=device)
+                         dtype=dtype, device=device)
     v_cache = torch.full((pool, block_size, num_kv_heads, head_dim), V_SENTINEL,
-                         dtype=torch.bfloat16, device=device)
+                         dtype=dtype, device=device)
     prior = ~is_new
     k_cache.view(-1, num_kv_heads, head_dim)[slot_of_row[prior]] = k_log[prior]
     v_cache.view(-1, num_kv_heads, head_dim)[slot_of_row[prior]] = v_log[prior]
@@ -209,7 +213,7 @@ def build_varlen_case(name: str, seq_lens, query_lens, num_q_heads: int, num_kv_
 
 def build_smallseq_case(name: str, kv_lens, num_q_heads: int, num_kv_heads: int,
                         head_dim: int, seed: int, device="cpu",
-                        scale: Optional[float] = None) -> SmallSeqCase:
+                        scale: Optional[float] = None, dtype=torch.bfloat16) -> SmallSeqCase:
     device = torch.device(device)
     kv_lens = [int(x) for x in kv_lens]
     cu = [0]
@@ -217,9 +221,9 @@ def build_smallseq_case(name: str, kv_lens, num_q_heads: int, num_kv_heads: int,
         cu.append(cu[-1] + L)
     B = len(kv_lens)
     gen = _gen(seed + 7919, device)
-    q = _randn_bf16((max(B, 1), num_q_heads, head_dim), gen, device)[:B]
-    k = _randn_bf16((max(cu[-1], 1), num_kv_heads, head_dim), gen, device)[: cu[-1]]
-    v = _randn_bf16((max(cu[-1], 1), num_kv_heads, head_dim), gen, device)[: cu[-1]]
+    q = _randn_bf16((max(B, 1), num_q_heads, head_dim), gen, device, dtype=dtype)[:B]
+    k = _randn_bf16((max(cu[-1], 1), num_kv_heads, head_dim), gen, device, dtype=dtype)[: cu[-1]]
+    v = _randn_bf16((max(cu[-1], 1), num_kv_heads, head_dim), gen, device, dtype=dtype)[: cu[-1]]
     return SmallSeqCase(
         name=name, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads, head_dim=head_dim,
         scale=float(scale if scale is not None else 1.0 / math.sqrt(head_dim)),
@@ -341,6 +345,6 @@ NAMED = {
 
 
 def bf16_bits(t: torch.Tensor):
-    """A bf16 tensor's bit patterns as a host numpy uint16 array."""
+    """A 16-bit (bf16 or fp16) tensor's bit patterns as a host numpy uint16 array."""
     import numpy as np
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
