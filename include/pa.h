@@ -227,7 +227,8 @@ pa_status pa_write_kv_ex(const void* k, const void* v, const int64_t* slot_mappi
  * (span_offsets NULL: none, and causal applies; otherwise as
  * pa_attention_varlen_spans, and causal is ignored).  pa_attention_varlen and
  * pa_attention_varlen_spans are this call with block_stride 0, bf16.
- * Returns PA_ERR_UNSUPPORTED for a dtype the build does not run.
+ * The computation is the same in either element type: fp32 scores and
+ * softmax, P rounded to the element type for P.V, out rounded to it.
  */
 pa_status pa_attention_varlen_ex(const void* q, const void* k_cache, const void* v_cache,
                                  const int32_t* block_tables, int32_t max_blocks_per_seq,
@@ -296,6 +297,18 @@ pa_status pa_attention_smallseq(const void* q, const void* k, const void* v,
                                 int32_t num_q_heads, int32_t num_kv_heads,
                                 int32_t head_dim, int32_t max_seqlen_kv, float scale,
                                 void* out, void* workspace, void* stream);
+
+/*
+ * pa_attention_smallseq_ex — pa_attention_smallseq with an element type
+ * (PA_DTYPE_BF16 or PA_DTYPE_FP16 for q, k, v and out; the small-seq path of
+ * ROCm/TransformerEngine PR #461 takes both).  Other arguments as
+ * pa_attention_smallseq.
+ */
+pa_status pa_attention_smallseq_ex(const void* q, const void* k, const void* v,
+                                   const int32_t* cu_seqlens_kv, int32_t batch,
+                                   int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                   int32_t max_seqlen_kv, float scale, int32_t dtype, void* out,
+                                   void* workspace, void* stream);
 
 /*
  * pa_get_error — synchronise `stream`, read the workspace's error word into

@@ -44,7 +44,7 @@ EXPORTED_SYMBOLS = (
     "pa_write_kv", "pa_attention_varlen_workspace_size", "pa_attention_varlen",
     "pa_attention_smallseq", "pa_get_error", "pa_status_string", "pa_version",
     "pa_attention_varlen_static", "pa_attention_varlen_spans", "pa_write_kv_ex",
-    "pa_attention_varlen_ex",
+    "pa_attention_varlen_ex", "pa_attention_smallseq_ex",
 )
 DTYPE_BF16, DTYPE_FP16 = 0, 1
 
@@ -104,6 +104,9 @@ def load(build_if_missing: bool = True):
         lib.pa_attention_varlen_spans.argtypes = [
             p, p, p, p, i32, p, p, i32, i64, i32, i32, i32, i32, i64, i32, i32,
             ctypes.c_float, p, p, i32, p, p, ctypes.c_size_t, p]
+        lib.pa_attention_smallseq_ex.restype = ctypes.c_int
+        lib.pa_attention_smallseq_ex.argtypes = [p, p, p, p, i32, i32, i32, i32, i32,
+                                                 ctypes.c_float, i32, p, p, p]
         lib.pa_attention_smallseq.restype = ctypes.c_int
         lib.pa_attention_smallseq.argtypes = [p, p, p, p, i32, i32, i32, i32, i32,
                                               ctypes.c_float, p, p, p]
@@ -337,22 +340,24 @@ def attention_varlen_static(q, k_cache, v_cache, block_tables, seq_lens, query_s
 
 def attention_smallseq(q, k, v, cu_seqlens_kv, scale, out, max_seqlen_kv=16, workspace=None,
                        stream=None):
-    """s_q = 1 attention over <= 16 contiguous keys per entry; writes out [B, Hq, D]."""
-    _check(q, "q", torch.bfloat16, 3)
-    _check(k, "k", torch.bfloat16, 3)
-    _check(v, "v", torch.bfloat16, 3)
+    """s_q = 1 attention over <= 16 contiguous keys per entry; writes out [B, Hq, D]
+    (bf16 or fp16, like q)."""
+    dt = _element_dtype(q, "q")
+    _check(q, "q", dt, 3)
+    _check(k, "k", dt, 3)
+    _check(v, "v", dt, 3)
     _check(cu_seqlens_kv, "cu_seqlens_kv", torch.int32, 1)
-    _check(out, "out", torch.bfloat16, 3)
+    _check(out, "out", dt, 3)
     b, hq, d = q.shape
     _, hkv, d_k = k.shape
     if d_k != d or v.shape != k.shape or out.shape != q.shape or cu_seqlens_kv.shape[0] != b + 1:
         raise ValueError("inconsistent small-seq shapes")
     ws = workspace.data_ptr() if workspace is not None else None
-    st = load().pa_attention_smallseq(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                      cu_seqlens_kv.data_ptr(), b, hq, hkv, d,
-                                      int(max_seqlen_kv), float(scale), out.data_ptr(), ws,
-                                      _stream(stream))
-    _raise(st, "pa_attention_smallseq")
+    st = load().pa_attention_smallseq_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                         cu_seqlens_kv.data_ptr(), b, hq, hkv, d,
+                                         int(max_seqlen_kv), float(scale), _DTYPES[dt],
+                                         out.data_ptr(), ws, _stream(stream))
+    _raise(st, "pa_attention_smallseq_ex")
     return out
 
 

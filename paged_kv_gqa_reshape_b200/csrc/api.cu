@@ -73,13 +73,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor map with a 128-byte swizzle; dims/strides innermost first.
+// bf16 or fp16 tensor map with a 128-byte swizzle; dims/strides innermost first.
 bool make_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
-              const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+              const cuuint64_t* strides_bytes, const cuuint32_t* box, bool fp16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint32_t estride[5] = {1, 1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+  CUresult r = fn(map, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                  (cuuint32_t)rank, const_cast<void*>(base),
                   dims, strides_bytes, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -160,7 +161,7 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
                                 void* workspace, size_t workspace_bytes, void* stream) {
   // ---- host-visible checks (nothing launched yet) ----
   if (dtype != PA_DTYPE_BF16 && dtype != PA_DTYPE_FP16) return PA_ERR_INVALID_ARG;
-  if (dtype != PA_DTYPE_BF16) return PA_ERR_UNSUPPORTED;
+  const bool fp16 = dtype == PA_DTYPE_FP16;
   if (num_seqs < 0 || num_q_tokens < 0 || num_q_tokens > 0x7fffffffll || num_q_heads <= 0 ||
       num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || max_blocks_per_seq <= 0 ||
       num_blocks <= 0 || num_blocks > 0x7fffffffll || max_query_len < 0 || max_seq_len < 0 ||
@@ -207,8 +208,9 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
                                (cuuint64_t)block_size, (cuuint64_t)num_blocks};
     const cuuint64_t skv[3] = {(cuuint64_t)head_dim * 2, (cuuint64_t)num_kv_heads * head_dim * 2,
                                (cuuint64_t)block_stride * 2};
-    if (!make_map(&q_map, q, 3, dq, sq, box_q) || !make_map(&k_map, k_cache, 4, dkv, skv, box_kv) ||
-        !make_map(&v_map, v_cache, 4, dkv, skv, box_kv))
+    if (!make_map(&q_map, q, 3, dq, sq, box_q, fp16) ||
+        !make_map(&k_map, k_cache, 4, dkv, skv, box_kv, fp16) ||
+        !make_map(&v_map, v_cache, 4, dkv, skv, box_kv, fp16))
       return PA_ERR_CUDA;
   }
 
@@ -238,10 +240,10 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
     pp.span_offsets = span_offsets;
     pp.spans = spans;
     pp.num_spans = num_spans;
-    pp.out = static_cast<__nv_bfloat16*>(out);
+    pp.out = static_cast<uint16_t*>(out);
     pp.ws = ws;
     pp.L = L;
-    e = pa::launch_prefill(pp, q_map, k_map, v_map, head_dim, nsm, st);
+    e = pa::launch_prefill(pp, q_map, k_map, v_map, head_dim, fp16, nsm, st);
     if (e != cudaSuccess) return PA_ERR_CUDA;
   }
 
@@ -264,10 +266,10 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
   dp.num_blocks = num_blocks;
   dp.block_stride = block_stride;
   dp.scale_log2 = scale_log2;
-  dp.out = static_cast<__nv_bfloat16*>(out);
+  dp.out = static_cast<uint16_t*>(out);
   dp.ws = ws;
   dp.L = L;
-  e = pa::launch_decode(dp, head_dim, nsm, st);
+  e = pa::launch_decode(dp, head_dim, fp16, nsm, st);
   if (log_enabled())
     fprintf(stderr, "[pa] varlen S=%d T=%lld Hq=%d Hkv=%d D=%d prefill=%d sms=%d\n", num_seqs,
             (long long)num_q_tokens, num_q_heads, num_kv_heads, head_dim, (int)run_prefill, nsm);
@@ -329,6 +331,17 @@ pa_status pa_attention_smallseq(const void* q, const void* k, const void* v,
                                 const int32_t* cu_seqlens_kv, int32_t batch, int32_t num_q_heads,
                                 int32_t num_kv_heads, int32_t head_dim, int32_t max_seqlen_kv,
                                 float scale, void* out, void* workspace, void* stream) {
+  return pa_attention_smallseq_ex(q, k, v, cu_seqlens_kv, batch, num_q_heads, num_kv_heads,
+                                  head_dim, max_seqlen_kv, scale, PA_DTYPE_BF16, out, workspace,
+                                  stream);
+}
+
+pa_status pa_attention_smallseq_ex(const void* q, const void* k, const void* v,
+                                   const int32_t* cu_seqlens_kv, int32_t batch,
+                                   int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                   int32_t max_seqlen_kv, float scale, int32_t dtype, void* out,
+                                   void* workspace, void* stream) {
+  if (dtype != PA_DTYPE_BF16 && dtype != PA_DTYPE_FP16) return PA_ERR_INVALID_ARG;
   if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
       max_seqlen_kv < 0 || !isfinite(scale))
     return PA_ERR_INVALID_ARG;
@@ -350,9 +363,10 @@ pa_status pa_attention_smallseq(const void* q, const void* k, const void* v,
   p.group = num_q_heads / num_kv_heads;
   p.max_seqlen_kv = max_seqlen_kv;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.out = static_cast<__nv_bfloat16*>(out);
+  p.out = static_cast<uint16_t*>(out);
   p.err = static_cast<uint32_t*>(workspace);
-  cudaError_t e = pa::launch_smallseq(p, head_dim, sm_count(), static_cast<cudaStream_t>(stream));
+  cudaError_t e = pa::launch_smallseq(p, head_dim, dtype == PA_DTYPE_FP16, sm_count(),
+                                      static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

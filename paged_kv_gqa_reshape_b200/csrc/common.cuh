@@ -9,6 +9,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -32,6 +33,37 @@ __device__ __forceinline__ float bf16hi(uint32_t x) { return __uint_as_float(x &
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ---------------------------------------------------------------------------
+// element type of a kernel instantiation: bf16 (H = false) or fp16 (H = true);
+// two elements per 32-bit word, the lower-indexed one in the low half
+// ---------------------------------------------------------------------------
+template <bool H>
+__device__ __forceinline__ float elo(uint32_t x) {
+  if constexpr (H) return __half2float(__ushort_as_half((unsigned short)(x & 0xffffu)));
+  else return bf16lo(x);
+}
+template <bool H>
+__device__ __forceinline__ float ehi(uint32_t x) {
+  if constexpr (H) return __half2float(__ushort_as_half((unsigned short)(x >> 16)));
+  else return bf16hi(x);
+}
+// round-to-nearest-even pack of two floats
+template <bool H>
+__device__ __forceinline__ uint32_t epack(float lo, float hi) {
+  if constexpr (H) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  } else {
+    return pack_bf16x2(lo, hi);
+  }
+}
+// one element, round-to-nearest-even, as its 16-bit pattern
+template <bool H>
+__device__ __forceinline__ unsigned short ebits(float x) {
+  if constexpr (H) return __half_as_ushort(__float2half_rn(x));
+  else return __bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
 
 // 2^x on the SFU (ex2.approx, flush-to-zero): a hardware instruction.
@@ -130,6 +162,20 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_f16_16816(float (&c)[4], const uint32_t (&a)[4],
+                                              uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+template <bool H>
+__device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+  if constexpr (H) mma_f16_16816(c, a, b0, b1);
+  else mma_bf16_16816(c, a, b0, b1);
 }
 
 // ---------------------------------------------------------------------------
@@ -330,11 +376,16 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo_
   return d;
 }
 
-// Instruction descriptor, kind::f16: f32 accumulator, bf16 A and B,
-// A K-major, B K-major (b_mn_major = 0) or MN-major (1), shape M x N.
+// Instruction descriptor, kind::f16: f32 accumulator, A and B both bf16
+// (format 1) or both fp16 (format 0), A K-major, B K-major (b_mn_major = 0)
+// or MN-major (1), shape M x N.
+__host__ __device__ constexpr uint32_t instr_desc_f16kind(int M, int N, int b_mn_major,
+                                                          bool fp16) {
+  return (1u << 4) | ((fp16 ? 0u : 1u) << 7) | ((fp16 ? 0u : 1u) << 10) |
+         ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
 __host__ __device__ constexpr uint32_t instr_desc_bf16(int M, int N, int b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn_major << 16) |
-         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+  return instr_desc_f16kind(M, N, b_mn_major, false);
 }
 
 }  // namespace pa

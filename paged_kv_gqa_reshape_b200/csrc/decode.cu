@@ -68,7 +68,7 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
 
 }  // namespace
 
-template <int D, int HPC, int NSTAGE, int NGT>
+template <int D, int HPC, int NSTAGE, int NGT, bool H>
 __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams p) {
   using Shape = DecodeShape<D, HPC, NSTAGE>;
   constexpr int CH = Shape::kChunks;
@@ -170,8 +170,8 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
   // single-query sequences with no key: zero output rows (spread over the ranges)
   for (long long s = c; s < S; s += G) {
     if (is_decode((int)s) && seq_kv((int)s) == 0) {
-      __nv_bfloat16* o0 = p.out + ((size_t)seq_q((int)s) * p.num_q_heads + head0) * D;
-      for (int i = lane; i < g * D; i += 32) o0[i] = __float2bfloat16_rn(0.f);
+      uint16_t* o0 = p.out + ((size_t)seq_q((int)s) * p.num_q_heads + head0) * D;
+      for (int i = lane; i < g * D; i += 32) o0[i] = 0;  // +0 in both element types
     }
   }
   if (P == 0) return;
@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
           uint32_t a[4];
           ldmatrix_x4(kbase + (key * D + ((chunk ^ (key & 7)) * 8)) * 2, a[0], a[1], a[2], a[3]);
 #pragma unroll
-          for (int nt = 0; nt < NGT; ++nt) mma_bf16_16816(sc[nt], a, qb[nt][ks][0], qb[nt][ks][1]);
+          for (int nt = 0; nt < NGT; ++nt) mma_16816<H>(sc[nt], a, qb[nt][ks][0], qb[nt][ks][1]);
         }
       }
       // ---- mask, online softmax per head column ----
@@ -338,8 +338,8 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
           o[nt][mt][2] *= a0;
           o[nt][mt][3] *= a1;
         }
-        pb[nt][0] = movmatrix_trans(pack_bf16x2(s0, s1));  // keys 0-7
-        pb[nt][1] = movmatrix_trans(pack_bf16x2(s2, s3));  // keys 8-15
+        pb[nt][0] = movmatrix_trans(epack<H>(s0, s1));  // keys 0-7
+        pb[nt][1] = movmatrix_trans(epack<H>(s2, s3));  // keys 8-15
       }
       // ---- O^T += V^T . P^T : 16 d rows x 8 heads per m-tile ----
       {
@@ -351,7 +351,7 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
           ldmatrix_x4_trans(vbase + (key * D + ((chunk ^ (key & 7)) * 8)) * 2, a[0], a[1], a[2],
                             a[3]);
 #pragma unroll
-          for (int nt = 0; nt < NGT; ++nt) mma_bf16_16816(o[nt][mt], a, pb[nt][0], pb[nt][1]);
+          for (int nt = 0; nt < NGT; ++nt) mma_16816<H>(o[nt][mt], a, pb[nt][0], pb[nt][1]);
         }
       }
     }
@@ -372,11 +372,11 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
           const int hl = nt * 8 + 2 * tq + j;
           if (hl < g) {
             const float inv = l[nt][j] > 0.f ? 1.f / l[nt][j] : 0.f;
-            __nv_bfloat16* orow = p.out + ((size_t)seg_q * p.num_q_heads + head0 + hl) * D;
+            uint16_t* orow = p.out + ((size_t)seg_q * p.num_q_heads + head0 + hl) * D;
 #pragma unroll
             for (int mt = 0; mt < KSTEPS; ++mt) {
-              orow[mt * 16 + gq] = __float2bfloat16_rn(o[nt][mt][j] * inv);
-              orow[mt * 16 + gq + 8] = __float2bfloat16_rn(o[nt][mt][2 + j] * inv);
+              orow[mt * 16 + gq] = ebits<H>(o[nt][mt][j] * inv);
+              orow[mt * 16 + gq + 8] = ebits<H>(o[nt][mt][2 + j] * inv);
             }
           }
         }
@@ -453,8 +453,8 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
                 if (lane * 4 < D) {
                   const float inv = ws > 0.f ? 1.f / ws : 0.f;
                   uint2 v;
-                  v.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-                  v.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+                  v.x = epack<H>(acc.x * inv, acc.y * inv);
+                  v.y = epack<H>(acc.z * inv, acc.w * inv);
                   *reinterpret_cast<uint2*>(
                       p.out + ((size_t)seg_q * p.num_q_heads + head0 + i / n_chunks) * D + lane * 4) = v;
                 }
@@ -519,8 +519,8 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
           if (lane * 4 < D) {
             const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
             uint2 v;
-            v.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-            v.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+            v.x = epack<H>(acc.x * inv, acc.y * inv);
+            v.y = epack<H>(acc.z * inv, acc.w * inv);
             *reinterpret_cast<uint2*>(p.out + ((size_t)seg_q * p.num_q_heads + head) * D + lane * 4) = v;
           }
         }
@@ -549,10 +549,10 @@ int heads_per_cta(int num_kv_heads) {
   return 1;
 }
 
-template <int D, int HPC, int NSTAGE, int NGT>
+template <int D, int HPC, int NSTAGE, int NGT, bool H>
 cudaError_t launch_t(const DecodeParams& p, int num_sms, cudaStream_t stream) {
   using Shape = DecodeShape<D, HPC, NSTAGE>;
-  auto kernel = decode_kernel<D, HPC, NSTAGE, NGT>;
+  auto kernel = decode_kernel<D, HPC, NSTAGE, NGT, H>;
   const int smem = Shape::smem_bytes(p.self_plan != 0);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -571,26 +571,34 @@ cudaError_t launch_t(const DecodeParams& p, int num_sms, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-template <int D, int NSTAGE, int NGT>
+template <int D, int NSTAGE, int NGT, bool H>
 cudaError_t launch_hpc(const DecodeParams& p, int hpc, int num_sms, cudaStream_t stream) {
   switch (hpc) {
-    case 8: return launch_t<D, 8, NSTAGE, NGT>(p, num_sms, stream);
-    case 4: return launch_t<D, 4, NSTAGE, NGT>(p, num_sms, stream);
-    case 2: return launch_t<D, 2, NSTAGE, NGT>(p, num_sms, stream);
-    default: return launch_t<D, 1, NSTAGE, NGT>(p, num_sms, stream);
+    case 8: return launch_t<D, 8, NSTAGE, NGT, H>(p, num_sms, stream);
+    case 4: return launch_t<D, 4, NSTAGE, NGT, H>(p, num_sms, stream);
+    case 2: return launch_t<D, 2, NSTAGE, NGT, H>(p, num_sms, stream);
+    default: return launch_t<D, 1, NSTAGE, NGT, H>(p, num_sms, stream);
   }
+}
+
+template <bool H>
+cudaError_t launch_decode_t(const DecodeParams& p, int head_dim, int num_sms,
+                            cudaStream_t stream) {
+  const int hpc = heads_per_cta(p.num_kv_heads);
+  if (head_dim == 128) {
+    if (p.group <= 8) return launch_hpc<128, 3, 1, H>(p, hpc, num_sms, stream);
+    return launch_hpc<128, 3, 2, H>(p, hpc, num_sms, stream);
+  }
+  if (p.group <= 8) return launch_hpc<64, 6, 1, H>(p, hpc, num_sms, stream);
+  return launch_hpc<64, 6, 2, H>(p, hpc, num_sms, stream);
 }
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeParams& p, int head_dim, int num_sms, cudaStream_t stream) {
-  const int hpc = heads_per_cta(p.num_kv_heads);
-  if (head_dim == 128) {
-    if (p.group <= 8) return launch_hpc<128, 3, 1>(p, hpc, num_sms, stream);
-    return launch_hpc<128, 3, 2>(p, hpc, num_sms, stream);
-  }
-  if (p.group <= 8) return launch_hpc<64, 6, 1>(p, hpc, num_sms, stream);
-  return launch_hpc<64, 6, 2>(p, hpc, num_sms, stream);
+cudaError_t launch_decode(const DecodeParams& p, int head_dim, bool fp16, int num_sms,
+                          cudaStream_t stream) {
+  return fp16 ? launch_decode_t<true>(p, head_dim, num_sms, stream)
+              : launch_decode_t<false>(p, head_dim, num_sms, stream);
 }
 
 }  // namespace pa

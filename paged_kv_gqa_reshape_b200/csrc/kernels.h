@@ -43,12 +43,13 @@ struct DecodeParams {
   long long block_stride;  // elements between consecutive cache blocks
   float scale_log2;  // scale * log2(e)
   int self_plan;     // 1: every CTA plans the decode work itself (num_seqs <= kSelfPlanMaxSeqs)
-  __nv_bfloat16* out;
+  uint16_t* out;     // elements of the kernel's type (bf16 or fp16)
   unsigned char* ws;
   WorkspaceLayout L;
 };
 // Persistent launch: one resident wave, num_sms from the device.
-cudaError_t launch_decode(const DecodeParams& p, int head_dim, int num_sms, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParams& p, int head_dim, bool fp16, int num_sms,
+                          cudaStream_t stream);
 
 // ---- tcgen05 prefill ------------------------------------------------------
 struct PrefillParams {
@@ -64,14 +65,14 @@ struct PrefillParams {
   const int32_t* span_offsets;  // full-attention spans (null: none)
   const int32_t* spans;
   int num_spans;
-  __nv_bfloat16* out;
+  uint16_t* out;  // [T, Hq, D] elements of the kernel's type (bf16 or fp16)
   unsigned char* ws;
   WorkspaceLayout L;
 };
 // Tensor maps are built by the host layer (they need the driver entry point).
 cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& q_map,
                            const CUtensorMap& k_map, const CUtensorMap& v_map, int head_dim,
-                           int grid, cudaStream_t stream);
+                           bool fp16, int grid, cudaStream_t stream);
 
 // ---- small-seq -------------------------------------------------------------
 struct SmallSeqParams {
@@ -85,10 +86,10 @@ struct SmallSeqParams {
   int group;
   int max_seqlen_kv;
   float scale_log2;
-  __nv_bfloat16* out;
+  uint16_t* out;  // elements of the kernel's type (bf16 or fp16)
   uint32_t* err;
 };
-cudaError_t launch_smallseq(const SmallSeqParams& p, int head_dim, int num_sms,
+cudaError_t launch_smallseq(const SmallSeqParams& p, int head_dim, bool fp16, int num_sms,
                             cudaStream_t stream);
 
 }  // namespace pa

@@ -104,7 +104,7 @@ __device__ __forceinline__ Work decode_work(int w, const int2* tiles, const int2
 
 }  // namespace
 
-template <int D>
+template <int D, bool H>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(PrefillParams p, const __grid_constant__ CUtensorMap q_map,
                    const __grid_constant__ CUtensorMap k_map,
@@ -229,8 +229,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------ MMA issuer --------------------------------
     if (lane == 0) {
-      constexpr uint32_t idesc_s = instr_desc_bf16(BM, BN, 0);
-      constexpr uint32_t idesc_o = instr_desc_bf16(BM, D, 1);
+      constexpr uint32_t idesc_s = instr_desc_f16kind(BM, BN, 0, H);
+      constexpr uint32_t idesc_o = instr_desc_f16kind(BM, D, 1, H);
       long long ld = 0;   // K/V tiles consumed (mirrors the producer)
       int tcount = 0;
       int s_it[2] = {0, 0}, pv_it[2] = {0, 0};
@@ -321,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool row_ok = r < rows;
       if (n == 0) {
         if (row_ok) {
-          __nv_bfloat16* orow =
+          uint16_t* orow =
               p.out + ((size_t)(wk.q_start + qrow) * p.num_q_heads + wk.head) * D;
 #pragma unroll
           for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = make_uint4(0, 0, 0, 0);
@@ -407,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                        scale2, nbase2);
             const uint64_t pp = f2_pack(fast_exp2(f2_lo(xx)), fast_exp2(f2_hi(xx)));
             rs2[e % (NP / 2)] = f2_add(rs2[e % (NP / 2)], pp);
-            pk[e] = pack_bf16x2(f2_lo(pp), f2_hi(pp));
+            pk[e] = epack<H>(f2_lo(pp), f2_hi(pp));
           }
           tmem_st16(s_col + h / 2, pk);
         }
@@ -441,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = p.out + ((size_t)(wk.q_start + qrow) * p.num_q_heads + wk.head) * D;
+      uint16_t* orow = p.out + ((size_t)(wk.q_start + qrow) * p.num_q_heads + wk.head) * D;
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t ov[32];
@@ -451,10 +451,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; i += 8) {
             uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(ov[i + 0]) * inv, __uint_as_float(ov[i + 1]) * inv);
-            v.y = pack_bf16x2(__uint_as_float(ov[i + 2]) * inv, __uint_as_float(ov[i + 3]) * inv);
-            v.z = pack_bf16x2(__uint_as_float(ov[i + 4]) * inv, __uint_as_float(ov[i + 5]) * inv);
-            v.w = pack_bf16x2(__uint_as_float(ov[i + 6]) * inv, __uint_as_float(ov[i + 7]) * inv);
+            v.x = epack<H>(__uint_as_float(ov[i + 0]) * inv, __uint_as_float(ov[i + 1]) * inv);
+            v.y = epack<H>(__uint_as_float(ov[i + 2]) * inv, __uint_as_float(ov[i + 3]) * inv);
+            v.z = epack<H>(__uint_as_float(ov[i + 4]) * inv, __uint_as_float(ov[i + 5]) * inv);
+            v.w = epack<H>(__uint_as_float(ov[i + 6]) * inv, __uint_as_float(ov[i + 7]) * inv);
             *reinterpret_cast<uint4*>(orow + c0 + i) = v;
           }
         }
@@ -477,23 +477,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool H>
 static cudaError_t launch_prefill_t(const PrefillParams& p, const CUtensorMap& q_map,
                                     const CUtensorMap& k_map, const CUtensorMap& v_map, int grid,
                                     cudaStream_t stream) {
   using SM = PrefillSmem<D>;
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>,
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, H>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc);
   if (e != cudaSuccess) return e;
-  prefill_kernel<D><<<grid, kThreads, SM::kAlloc, stream>>>(p, q_map, k_map, v_map);
+  prefill_kernel<D, H><<<grid, kThreads, SM::kAlloc, stream>>>(p, q_map, k_map, v_map);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& q_map,
                            const CUtensorMap& k_map, const CUtensorMap& v_map, int head_dim,
-                           int grid, cudaStream_t stream) {
-  if (head_dim == 128) return launch_prefill_t<128>(p, q_map, k_map, v_map, grid, stream);
-  return launch_prefill_t<64>(p, q_map, k_map, v_map, grid, stream);
+                           bool fp16, int grid, cudaStream_t stream) {
+  if (head_dim == 128)
+    return fp16 ? launch_prefill_t<128, true>(p, q_map, k_map, v_map, grid, stream)
+                : launch_prefill_t<128, false>(p, q_map, k_map, v_map, grid, stream);
+  return fp16 ? launch_prefill_t<64, true>(p, q_map, k_map, v_map, grid, stream)
+              : launch_prefill_t<64, false>(p, q_map, k_map, v_map, grid, stream);
 }
 
 }  // namespace pa

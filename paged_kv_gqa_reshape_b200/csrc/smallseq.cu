@@ -46,7 +46,7 @@ struct SmallSeqItem {
 
 }  // namespace
 
-template <int D>
+template <int D, bool H>
 __global__ void __launch_bounds__(256, 3) smallseq_kernel(SmallSeqParams p) {
   using It = SmallSeqItem<D>;
   constexpr int LPK = It::LPK, KPP = It::KPP, PASSES = It::PASSES;
@@ -113,8 +113,8 @@ __global__ void __launch_bounds__(256, 3) smallseq_kernel(SmallSeqParams p) {
       const uint32_t w[4] = {cur.q.x, cur.q.y, cur.q.z, cur.q.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        qf[2 * i] = bf16lo(w[i]) * p.scale_log2;
-        qf[2 * i + 1] = bf16hi(w[i]) * p.scale_log2;
+        qf[2 * i] = elo<H>(w[i]) * p.scale_log2;
+        qf[2 * i + 1] = ehi<H>(w[i]) * p.scale_log2;
       }
     }
     // NP passes of KPP keys, straight-line (the shuffle trees of all passes
@@ -129,8 +129,8 @@ __global__ void __launch_bounds__(256, 3) smallseq_kernel(SmallSeqParams p) {
         float dot = 0.f;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          dot = fmaf(qf[2 * i], bf16lo(w[i]), dot);
-          dot = fmaf(qf[2 * i + 1], bf16hi(w[i]), dot);
+          dot = fmaf(qf[2 * i], elo<H>(w[i]), dot);
+          dot = fmaf(qf[2 * i + 1], ehi<H>(w[i]), dot);
         }
         sc[pp] = dot;
       }
@@ -155,8 +155,8 @@ __global__ void __launch_bounds__(256, 3) smallseq_kernel(SmallSeqParams p) {
         const uint32_t w[4] = {cur.v[pp].x, cur.v[pp].y, cur.v[pp].z, cur.v[pp].w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          acc[2 * i] = fmaf(pw, bf16lo(w[i]), acc[2 * i]);
-          acc[2 * i + 1] = fmaf(pw, bf16hi(w[i]), acc[2 * i + 1]);
+          acc[2 * i] = fmaf(pw, elo<H>(w[i]), acc[2 * i]);
+          acc[2 * i + 1] = fmaf(pw, ehi<H>(w[i]), acc[2 * i + 1]);
         }
       }
     };
@@ -178,21 +178,22 @@ __global__ void __launch_bounds__(256, 3) smallseq_kernel(SmallSeqParams p) {
     if (sub == 0) {
       const float inv = sum > 0.f ? 1.f / sum : 0.f;  // an empty entry writes zeros
       uint4 ov;
-      ov.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-      ov.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-      ov.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
-      ov.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+      ov.x = epack<H>(acc[0] * inv, acc[1] * inv);
+      ov.y = epack<H>(acc[2] * inv, acc[3] * inv);
+      ov.z = epack<H>(acc[4] * inv, acc[5] * inv);
+      ov.w = epack<H>(acc[6] * inv, acc[7] * inv);
       __stcs(reinterpret_cast<uint4*>(p.out + ((size_t)b * p.num_q_heads + h) * D) + l, ov);
     }
   }
 }
 
-cudaError_t launch_smallseq(const SmallSeqParams& p, int head_dim, int num_sms,
+cudaError_t launch_smallseq(const SmallSeqParams& p, int head_dim, bool fp16, int num_sms,
                             cudaStream_t stream) {
   const long long warps = (long long)p.batch * p.num_q_heads;
   if (warps == 0) return cudaSuccess;
   const int threads = 256;
-  auto kernel = head_dim == 128 ? smallseq_kernel<128> : smallseq_kernel<64>;
+  auto kernel = head_dim == 128 ? (fp16 ? smallseq_kernel<128, true> : smallseq_kernel<128, false>)
+                                 : (fp16 ? smallseq_kernel<64, true> : smallseq_kernel<64, false>);
   int per_sm = 0;
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0);
   if (e != cudaSuccess) return e;
