@@ -317,6 +317,20 @@ def components(pa, hbm_peak, tc_peak, peak_kind):
     res["smallseq_batch"] = {"ms": round(ms, 4), "gbs": round(gbs, 1),
                              "frac": round(gbs / hbm_peak, 3), "unit": "GB/s", "of": peak_kind}
     del ss, out
+    # the same prefill and decode workloads with fp16 inputs
+    vc16 = workloads.varlen_prefill(device=dev, keep_logical=False, dtype=torch.float16)
+    ms = time_varlen_component(pa, vc16)
+    tf = attention_flops(vc16) / (ms * 1e-3) / 1e12
+    res["varlen_prefill_fp16"] = {"ms": round(ms, 4), "tflops": round(tf, 1),
+                                  "frac": round(tf / tc_peak, 3), "peak": tc_peak,
+                                  "unit": "TFLOP/s", "of": peak_kind}
+    del vc16
+    dc16 = workloads.decode_batch(device=dev, keep_logical=False, dtype=torch.float16)
+    ms = time_varlen_component(pa, dc16, iters=50)
+    gbs = attention_bytes(dc16) / (ms * 1e-3) / 1e9
+    res["decode_batch_fp16"] = {"ms": round(ms, 4), "gbs": round(gbs, 1),
+                                "frac": round(gbs / hbm_peak, 3), "unit": "GB/s", "of": peak_kind}
+    del dc16
     sc, so, sp = workloads.spans_prefill(device=dev, keep_logical=False)
     ms = time_spans_component(pa, sc, so, sp)
     pairs = workloads.spans_visible_pairs(sc.seq_lens.tolist(), sc.query_lens.tolist(),

@@ -250,22 +250,24 @@ def tiny_prefill(device="cpu", seed=1001) -> VarlenCase:
 
 
 def decode_batch(device="cpu", seed=1002, num_seqs=64, lo=256, hi=4096,
-                 num_q_heads=32, num_kv_heads=8, head_dim=128, keep_logical=True) -> VarlenCase:
+                 num_q_heads=32, num_kv_heads=8, head_dim=128, keep_logical=True,
+                 dtype=torch.bfloat16) -> VarlenCase:
     """64 sequences with one query each, context uniform in [256, 4096],
     Hq 32 / Hkv 8, D 128; the new token is scattered before attention."""
     lens = _uniform_ints(lo, hi, num_seqs, seed)
     return build_varlen_case("decode_batch", lens, [1] * num_seqs, num_q_heads, num_kv_heads,
-                             head_dim, True, seed, device=device, keep_logical=keep_logical)
+                             head_dim, True, seed, device=device, keep_logical=keep_logical,
+                             dtype=dtype)
 
 
 def varlen_prefill(device="cpu", seed=1003, lens=(2048, 3000, 4096, 8192),
                    num_q_heads=32, num_kv_heads=8, head_dim=128, causal=True,
-                   keep_logical=True) -> VarlenCase:
+                   keep_logical=True, dtype=torch.bfloat16) -> VarlenCase:
     """4 packed sequences of 2048, 3000, 4096 and 8192 tokens, causal,
     Hq 32 / Hkv 8, D 128, shuffled table."""
     return build_varlen_case("varlen_prefill", list(lens), list(lens), num_q_heads,
                              num_kv_heads, head_dim, causal, seed, device=device,
-                             keep_logical=keep_logical)
+                             keep_logical=keep_logical, dtype=dtype)
 
 
 def spans_prefill(device="cpu", seed=1006, num_seqs=4, text=512, cond=1536, target=2048,
