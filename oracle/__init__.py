@@ -69,6 +69,11 @@ def _load():
             p, p, p, p, p, p, i32, i32, i32, i32, f64, i32, i32, p, i64, p]
         lib.oracle_attention_smallseq_dtype.restype = i32
         lib.oracle_attention_smallseq_dtype.argtypes = [p, p, p, p, i32, i32, i32, i32, f64, i32, p]
+        lib.oracle_smallseq_weights.restype = i32
+        lib.oracle_smallseq_weights.argtypes = [p, p, p, i32, i32, i32, i32, f64, i32, i32, p]
+        lib.oracle_smallseq_backward.restype = i32
+        lib.oracle_smallseq_backward.argtypes = [p, p, p, p, p, i32, i32, i32, i32, f64, i32,
+                                                 p, p, p]
         lib.oracle_widen.restype = f64
         lib.oracle_widen.argtypes = [ctypes.c_uint16, i32]
         lib.oracle_attention_smallseq.restype = i32
@@ -160,6 +165,36 @@ def smallseq_dtype(q, k, v, cu_seqlens_kv, num_kv_heads, scale, dtype):
     if rc != 0:
         raise ValueError(f"oracle_attention_smallseq_dtype failed ({rc})")
     return out
+
+
+def smallseq_weights(q, k, cu_seqlens_kv, num_kv_heads, scale, wlen, dtype=0):
+    """Softmax weights [B, Hq, wlen] (float64; zeros past each entry's keys)."""
+    q, k = _arr(q, np.uint16), _arr(k, np.uint16)
+    cu = _arr(cu_seqlens_kv, np.int32)
+    b, hq, d = q.shape
+    w = np.zeros((b, hq, wlen), dtype=np.float64)
+    rc = _load().oracle_smallseq_weights(_ptr(q), _ptr(k), _ptr(cu), b, hq, num_kv_heads, d,
+                                         float(scale), int(dtype), int(wlen), _ptr(w))
+    if rc != 0:
+        raise ValueError(f"oracle_smallseq_weights failed ({rc})")
+    return w
+
+
+def smallseq_backward(q, k, v, dout, cu_seqlens_kv, num_kv_heads, scale, dtype=0):
+    """(dq [B, Hq, D], dk [N, Hkv, D], dv [N, Hkv, D]) in float64."""
+    q, k, v, dout = (_arr(x, np.uint16) for x in (q, k, v, dout))
+    cu = _arr(cu_seqlens_kv, np.int32)
+    b, hq, d = q.shape
+    n = k.shape[0]
+    dq = np.zeros((b, hq, d), dtype=np.float64)
+    dk = np.zeros((max(n, 1), num_kv_heads, d), dtype=np.float64)
+    dv = np.zeros((max(n, 1), num_kv_heads, d), dtype=np.float64)
+    rc = _load().oracle_smallseq_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(cu), b, hq,
+                                          num_kv_heads, d, float(scale), int(dtype), _ptr(dq),
+                                          _ptr(dk), _ptr(dv))
+    if rc != 0:
+        raise ValueError(f"oracle_smallseq_backward failed ({rc})")
+    return dq, dk[:n], dv[:n]
 
 
 def widen(bits: int, dtype: int) -> float:

@@ -500,6 +500,114 @@ int oracle_attention_smallseq_dtype(const uint16_t *q, const uint16_t *k,
                            head_dim, scale, dtype, out);
 }
 
+/*
+ * Small-seq attention weights and backward (ROCm/TransformerEngine PR #461,
+ * description: the forward also returns the attention weights, shaped
+ * [batch, Hq, 1, max_seqlen_kv]; the backward computes grad_V, grad_attn,
+ * the softmax backward and grad_Q / grad_K).  With s_j = scale * <q, k_j>,
+ * p = softmax(s) over the entry's keys and upstream gradient dO:
+ *     dV_j += p_j dO                    (summed over the query heads sharing
+ *     dP_j  = <dO, v_j>                  a KV head)
+ *     dS_j  = p_j (dP_j - sum_k p_k dP_k)
+ *     dQ    = scale * sum_j dS_j k_j
+ *     dK_j += scale * dS_j q
+ * weights: [batch, Hq, wlen] doubles (entry b's p in the first n_b slots,
+ * zeros after); dq [batch, Hq, D]; dk, dv [total keys, Hkv, D] doubles.
+ * An empty entry has no weights and contributes nothing.
+ */
+/* p_j = softmax_j(scale * <q, k_j>) over the n keys of one entry and KV head. */
+static void smallseq_probs(const uint16_t *q, const uint16_t *k, int64_t first, int64_t n,
+                           int kvh, int num_kv_heads, int head_dim, double scale,
+                           double (*widen)(uint16_t), double *p) {
+    double m = -INFINITY;
+    for (int64_t j = 0; j < n; ++j) {
+        const uint16_t *kr = k + ((first + j) * num_kv_heads + kvh) * (int64_t)head_dim;
+        double dot = 0.0;
+        for (int d = 0; d < head_dim; ++d) dot += widen(q[d]) * widen(kr[d]);
+        p[j] = scale * dot;
+        if (p[j] > m) m = p[j];
+    }
+    double denom = 0.0;
+    for (int64_t j = 0; j < n; ++j) {
+        p[j] = exp(p[j] - m);
+        denom += p[j];
+    }
+    for (int64_t j = 0; j < n; ++j) p[j] /= denom;
+}
+
+int oracle_smallseq_weights(const uint16_t *q, const uint16_t *k,
+                            const int32_t *cu_seqlens_kv, int batch, int num_q_heads,
+                            int num_kv_heads, int head_dim, double scale, int dtype,
+                            int wlen, double *weights) {
+    if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || wlen < 0) return -1;
+    double (*widen)(uint16_t) = dtype == 1 ? half_to_double : bf16_to_double;
+    int group = num_q_heads / num_kv_heads;
+    for (int b = 0; b < batch; ++b) {
+        int64_t first = cu_seqlens_kv[b], n = (int64_t)cu_seqlens_kv[b + 1] - first;
+        if (n > wlen) return -2;
+        for (int h = 0; h < num_q_heads; ++h) {
+            double *w = weights + ((int64_t)b * num_q_heads + h) * wlen;
+            for (int j = 0; j < wlen; ++j) w[j] = 0.0;
+            if (n <= 0) continue;
+            smallseq_probs(q + ((int64_t)b * num_q_heads + h) * head_dim, k, first, n,
+                           h / group, num_kv_heads, head_dim, scale, widen, w);
+        }
+    }
+    return 0;
+}
+
+int oracle_smallseq_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                             const uint16_t *dout, const int32_t *cu_seqlens_kv, int batch,
+                             int num_q_heads, int num_kv_heads, int head_dim, double scale,
+                             int dtype, double *dq, double *dk, double *dv) {
+    if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return -1;
+    double (*widen)(uint16_t) = dtype == 1 ? half_to_double : bf16_to_double;
+    int group = num_q_heads / num_kv_heads;
+    int64_t total = cu_seqlens_kv[batch];
+    for (int64_t i = 0; i < total * num_kv_heads * head_dim; ++i) dk[i] = dv[i] = 0.0;
+    for (int64_t i = 0; i < (int64_t)batch * num_q_heads * head_dim; ++i) dq[i] = 0.0;
+    int64_t max_len = 1;
+    for (int b = 0; b < batch; ++b) {
+        int64_t n = (int64_t)cu_seqlens_kv[b + 1] - cu_seqlens_kv[b];
+        if (n > max_len) max_len = n;
+    }
+    double *p = (double *)malloc(sizeof(double) * (size_t)max_len);
+    double *dp = (double *)malloc(sizeof(double) * (size_t)max_len);
+    for (int b = 0; b < batch; ++b) {
+        int64_t first = cu_seqlens_kv[b], n = (int64_t)cu_seqlens_kv[b + 1] - first;
+        if (n <= 0) continue;
+        for (int h = 0; h < num_q_heads; ++h) {
+            int kvh = h / group;
+            const uint16_t *qr = q + ((int64_t)b * num_q_heads + h) * head_dim;
+            const uint16_t *gr = dout + ((int64_t)b * num_q_heads + h) * head_dim;
+            smallseq_probs(qr, k, first, n, kvh, num_kv_heads, head_dim, scale, widen, p);
+            double sum_pdp = 0.0;
+            for (int64_t j = 0; j < n; ++j) {
+                const uint16_t *vr = v + ((first + j) * num_kv_heads + kvh) * (int64_t)head_dim;
+                double dot = 0.0;
+                for (int d = 0; d < head_dim; ++d) dot += widen(gr[d]) * widen(vr[d]);
+                dp[j] = dot;
+                sum_pdp += p[j] * dot;
+            }
+            double *dqr = dq + ((int64_t)b * num_q_heads + h) * head_dim;
+            for (int64_t j = 0; j < n; ++j) {
+                double ds = p[j] * (dp[j] - sum_pdp);
+                const uint16_t *kr = k + ((first + j) * num_kv_heads + kvh) * (int64_t)head_dim;
+                double *dkr = dk + ((first + j) * num_kv_heads + kvh) * (int64_t)head_dim;
+                double *dvr = dv + ((first + j) * num_kv_heads + kvh) * (int64_t)head_dim;
+                for (int d = 0; d < head_dim; ++d) {
+                    dqr[d] += scale * ds * widen(kr[d]);
+                    dkr[d] += scale * ds * widen(qr[d]);
+                    dvr[d] += p[j] * widen(gr[d]);
+                }
+            }
+        }
+    }
+    free(p);
+    free(dp);
+    return 0;
+}
+
 /* One element widened exactly (dtype 0 = bf16, 1 = fp16), for tests. */
 double oracle_widen(uint16_t bits, int dtype) {
     return dtype == 1 ? half_to_double(bits) : bf16_to_double(bits);
