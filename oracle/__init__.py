@@ -73,7 +73,7 @@ def _load():
         lib.oracle_smallseq_weights.argtypes = [p, p, p, i32, i32, i32, i32, f64, i32, i32, p]
         lib.oracle_smallseq_backward.restype = i32
         lib.oracle_smallseq_backward.argtypes = [p, p, p, p, p, i32, i32, i32, i32, f64, i32,
-                                                 p, p, p]
+                                                 p, i32, p, p, p]
         lib.oracle_widen.restype = f64
         lib.oracle_widen.argtypes = [ctypes.c_uint16, i32]
         lib.oracle_attention_smallseq.restype = i32
@@ -180,8 +180,10 @@ def smallseq_weights(q, k, cu_seqlens_kv, num_kv_heads, scale, wlen, dtype=0):
     return w
 
 
-def smallseq_backward(q, k, v, dout, cu_seqlens_kv, num_kv_heads, scale, dtype=0):
-    """(dq [B, Hq, D], dk [N, Hkv, D], dv [N, Hkv, D]) in float64."""
+def smallseq_backward(q, k, v, dout, cu_seqlens_kv, num_kv_heads, scale, dtype=0, weights=None):
+    """(dq [B, Hq, D], dk [N, Hkv, D], dv [N, Hkv, D]) in float64.  With
+    ``weights`` ([B, Hq, W] float64) the softmax weights are taken as given
+    (the forward's saved weights) instead of recomputed from q and k."""
     q, k, v, dout = (_arr(x, np.uint16) for x in (q, k, v, dout))
     cu = _arr(cu_seqlens_kv, np.int32)
     b, hq, d = q.shape
@@ -189,9 +191,15 @@ def smallseq_backward(q, k, v, dout, cu_seqlens_kv, num_kv_heads, scale, dtype=0
     dq = np.zeros((b, hq, d), dtype=np.float64)
     dk = np.zeros((max(n, 1), num_kv_heads, d), dtype=np.float64)
     dv = np.zeros((max(n, 1), num_kv_heads, d), dtype=np.float64)
+    wp, wlen = None, 0
+    if weights is not None:
+        weights = _arr(weights, np.float64)
+        if weights.shape[:2] != (b, hq):
+            raise ValueError("weights must be [batch, num_q_heads, W]")
+        wp, wlen = _ptr(weights), weights.shape[2]
     rc = _load().oracle_smallseq_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(cu), b, hq,
-                                          num_kv_heads, d, float(scale), int(dtype), _ptr(dq),
-                                          _ptr(dk), _ptr(dv))
+                                          num_kv_heads, d, float(scale), int(dtype), wp, wlen,
+                                          _ptr(dq), _ptr(dk), _ptr(dv))
     if rc != 0:
         raise ValueError(f"oracle_smallseq_backward failed ({rc})")
     return dq, dk[:n], dv[:n]

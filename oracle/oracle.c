@@ -513,6 +513,9 @@ int oracle_attention_smallseq_dtype(const uint16_t *q, const uint16_t *k,
  *     dK_j += scale * dS_j q
  * weights: [batch, Hq, wlen] doubles (entry b's p in the first n_b slots,
  * zeros after); dq [batch, Hq, D]; dk, dv [total keys, Hkv, D] doubles.
+ * The backward takes p either recomputed from q and k (weights NULL) or as
+ * given (the weights the forward saved, which is what the PR's backward
+ * reads); the formulas above are the same either way.
  * An empty entry has no weights and contributes nothing.
  */
 /* p_j = softmax_j(scale * <q, k_j>) over the n keys of one entry and KV head. */
@@ -559,8 +562,10 @@ int oracle_smallseq_weights(const uint16_t *q, const uint16_t *k,
 int oracle_smallseq_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                              const uint16_t *dout, const int32_t *cu_seqlens_kv, int batch,
                              int num_q_heads, int num_kv_heads, int head_dim, double scale,
-                             int dtype, double *dq, double *dk, double *dv) {
+                             int dtype, const double *weights, int wlen, double *dq,
+                             double *dk, double *dv) {
     if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return -1;
+    if (weights && wlen <= 0) return -1;
     double (*widen)(uint16_t) = dtype == 1 ? half_to_double : bf16_to_double;
     int group = num_q_heads / num_kv_heads;
     int64_t total = cu_seqlens_kv[batch];
@@ -580,7 +585,13 @@ int oracle_smallseq_backward(const uint16_t *q, const uint16_t *k, const uint16_
             int kvh = h / group;
             const uint16_t *qr = q + ((int64_t)b * num_q_heads + h) * head_dim;
             const uint16_t *gr = dout + ((int64_t)b * num_q_heads + h) * head_dim;
-            smallseq_probs(qr, k, first, n, kvh, num_kv_heads, head_dim, scale, widen, p);
+            if (weights) { /* the forward's saved weights, as the backward reads them */
+                if (n > wlen) { free(p); free(dp); return -2; }
+                const double *w = weights + ((int64_t)b * num_q_heads + h) * wlen;
+                for (int64_t j = 0; j < n; ++j) p[j] = w[j];
+            } else {
+                smallseq_probs(qr, k, first, n, kvh, num_kv_heads, head_dim, scale, widen, p);
+            }
             double sum_pdp = 0.0;
             for (int64_t j = 0; j < n; ++j) {
                 const uint16_t *vr = v + ((first + j) * num_kv_heads + kvh) * (int64_t)head_dim;

@@ -101,3 +101,46 @@ def test_backward_matches_finite_differences_of_the_forward():
         args_p[which], args_m[which] = plus, minus
         fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
         assert abs(fd - grad[idx]) < 1e-6, (idx, fd, grad[idx])
+
+
+def test_backward_from_given_weights_matches_torch_softmax_backward():
+    # The backward reads the forward's saved weights.  With arbitrary weights W
+    # (here the exact softmax rounded to bf16, as a 16-bit forward saves it,
+    # so W is no longer an exact softmax), the gradients are still
+    #   dV_j = sum_h W_hj dO_h,  dS = softmax_backward(dP, W),
+    #   dQ = scale dS K,  dK_j = scale sum_h dS_hj q_h,
+    # checked here with torch's own softmax backward on the output W.
+    lens = [4, 16, 0, 9]
+    c = case(lens, 4, 2, 64, seed=43)
+    g = c.num_q_heads // c.num_kv_heads
+    dout = workloads._randn_bf16((c.batch, c.num_q_heads, c.head_dim), workloads._gen(6, "cpu"),
+                                 "cpu")
+    exact = oracle.smallseq_weights(bits(c.q), bits(c.k), c.cu_seqlens_kv.numpy(), c.num_kv_heads,
+                                    c.scale, 16)
+    w = torch.from_numpy(exact).to(torch.bfloat16).double().numpy()
+    dq, dk, dv = oracle.smallseq_backward(bits(c.q), bits(c.k), bits(c.v), bits(dout),
+                                          c.cu_seqlens_kv.numpy(), c.num_kv_heads, c.scale,
+                                          weights=w)
+    cu = c.cu_seqlens_kv.tolist()
+    qd, kd, vd, gd = (t.double() for t in (c.q, c.k, c.v, dout))
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert not dq[b].any()
+            continue
+        kb = kd[cu[b]:cu[b + 1]].repeat_interleave(g, dim=1)      # [n, Hq, D]
+        vb = vd[cu[b]:cu[b + 1]].repeat_interleave(g, dim=1)
+        wb = torch.from_numpy(w[b, :, :n])                        # [Hq, n]
+        dp = torch.einsum("hd,nhd->hn", gd[b], vb)
+        ds = torch._softmax_backward_data(dp, wb, 1, torch.float64)
+        ref_dq = c.scale * torch.einsum("hn,nhd->hd", ds, kb)
+        ref_dk = c.scale * torch.einsum("hn,hd->nhd", ds, qd[b]).reshape(
+            n, c.num_kv_heads, g, c.head_dim).sum(2)
+        ref_dv = torch.einsum("hn,hd->nhd", wb, gd[b]).reshape(
+            n, c.num_kv_heads, g, c.head_dim).sum(2)
+        assert np.max(np.abs(dq[b] - ref_dq.numpy())) < 1e-10
+        assert np.max(np.abs(dk[cu[b]:cu[b + 1]] - ref_dk.numpy())) < 1e-10
+        assert np.max(np.abs(dv[cu[b]:cu[b + 1]] - ref_dv.numpy())) < 1e-10
+    # the rounded weights move the gradients, by about their own relative error
+    dq0, _, dv0 = oracle.smallseq_backward(bits(c.q), bits(c.k), bits(c.v), bits(dout),
+                                           c.cu_seqlens_kv.numpy(), c.num_kv_heads, c.scale)
+    assert 0 < np.max(np.abs(dv - dv0)) < 2 ** -8 * np.max(np.abs(dv0)) * 4
