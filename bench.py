@@ -289,6 +289,38 @@ def time_spans_component(pa, case, span_offsets, spans, iters=20, warmup=3):
     return statistics.mean(a.elapsed_time(b) for a, b in evs)
 
 
+def time_calls(fn, iters=20, warmup=3):
+    """Device time per call (ms) of `fn`, CUDA events on the current stream."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(iters):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def smallseq_weight_bytes(ss, wlen):
+    """Bytes of the attention-weights output: every [batch, Hq, wlen] slot is written."""
+    return ss.batch * ss.num_q_heads * wlen * 2
+
+
+def smallseq_bwd_bytes(ss):
+    """Algorithmic bytes of the small-seq backward: q, dout, k, v and each
+    entry's saved weights read once, dq, dk, dv written once, cu_seqlens_kv."""
+    total_keys = ss.k.shape[0]
+    row = ss.head_dim * 2
+    return (2 * ss.batch * ss.num_q_heads * row            # q, dout
+            + 2 * total_keys * ss.num_kv_heads * row       # k, v
+            + total_keys * ss.num_q_heads * 2              # weights of the entry's keys
+            + ss.batch * ss.num_q_heads * row              # dq
+            + 2 * total_keys * ss.num_kv_heads * row       # dk, dv
+            + 4 * (ss.batch + 1))
+
+
 def components(pa, hbm_peak, tc_peak, peak_kind):
     """Secondary single-GPU measurements on the other workloads (device time per call)."""
     res = {}
@@ -316,7 +348,22 @@ def components(pa, hbm_peak, tc_peak, peak_kind):
     gbs = nbytes / (ms * 1e-3) / 1e9
     res["smallseq_batch"] = {"ms": round(ms, 4), "gbs": round(gbs, 1),
                              "frac": round(gbs / hbm_peak, 3), "unit": "GB/s", "of": peak_kind}
-    del ss, out
+    # the same workload's forward with the attention-weights output, then the backward
+    w = torch.empty(ss.batch, ss.num_q_heads, 16, dtype=ss.q.dtype, device=dev)
+    ms = time_calls(lambda: pa.attention_smallseq(ss.q, ss.k, ss.v, ss.cu_seqlens_kv, ss.scale,
+                                                  out, weights=w))
+    gbs = (nbytes + smallseq_weight_bytes(ss, w.shape[2])) / (ms * 1e-3) / 1e9
+    res["smallseq_fwd_weights"] = {"ms": round(ms, 4), "gbs": round(gbs, 1),
+                                   "frac": round(gbs / hbm_peak, 3), "unit": "GB/s",
+                                   "of": peak_kind}
+    dout = torch.randn(ss.q.shape, generator=workloads._gen(1007, dev), device=dev).to(ss.q.dtype)
+    dq, dk, dv = torch.empty_like(ss.q), torch.empty_like(ss.k), torch.empty_like(ss.v)
+    ms = time_calls(lambda: pa.attention_smallseq_bwd(ss.q, ss.k, ss.v, dout, w,
+                                                      ss.cu_seqlens_kv, ss.scale, dq, dk, dv))
+    gbs = smallseq_bwd_bytes(ss) / (ms * 1e-3) / 1e9
+    res["smallseq_bwd"] = {"ms": round(ms, 4), "gbs": round(gbs, 1),
+                           "frac": round(gbs / hbm_peak, 3), "unit": "GB/s", "of": peak_kind}
+    del ss, out, w, dout, dq, dk, dv
     # the same prefill and decode workloads with fp16 inputs
     vc16 = workloads.varlen_prefill(device=dev, keep_logical=False, dtype=torch.float16)
     ms = time_varlen_component(pa, vc16)
@@ -476,6 +523,20 @@ def run_single_workload(args):
             pa.attention_smallseq(ss.q, ss.k, ss.v, ss.cu_seqlens_kv, ss.scale, out)
         work = (ss.k.numel() + ss.v.numel() + ss.q.numel() + out.numel()) * 2 + 4 * (ss.batch + 1)
         unit, scale_div, peak = "GB/s", 1e9, hbm_peak
+    elif name == "smallseq_bwd":
+        ss = workloads.smallseq_batch(device=dev)
+        out = torch.empty_like(ss.q)
+        w = torch.empty(ss.batch, ss.num_q_heads, 16, dtype=ss.q.dtype, device=dev)
+        pa.attention_smallseq(ss.q, ss.k, ss.v, ss.cu_seqlens_kv, ss.scale, out, weights=w)
+        dout = torch.randn(ss.q.shape, generator=workloads._gen(1007, dev),
+                           device=dev).to(ss.q.dtype)
+        dq, dk, dv = torch.empty_like(ss.q), torch.empty_like(ss.k), torch.empty_like(ss.v)
+
+        def step():
+            pa.attention_smallseq_bwd(ss.q, ss.k, ss.v, dout, w, ss.cu_seqlens_kv, ss.scale,
+                                      dq, dk, dv)
+        work = smallseq_bwd_bytes(ss)
+        unit, scale_div, peak = "GB/s", 1e9, hbm_peak
     else:
         case = workloads.NAMED[name](device=dev, keep_logical=False) if name != "tiny_prefill" \
             else workloads.tiny_prefill(device=dev)
@@ -634,7 +695,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--workload", default="decode_batch",
-                    choices=sorted(list(workloads.NAMED) + ["spans_prefill"]),
+                    choices=sorted(list(workloads.NAMED) + ["spans_prefill", "smallseq_bwd"]),
                     help="decode_batch is the headline; the others time one workload alone")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per dominant-kernel launch from an ncu capture, if current")

@@ -9,6 +9,7 @@
  *                          prefill and any mix of them in one batch)
  *   pa_attention_smallseq  one query per batch entry over a handful (<= 16) of
  *                          contiguous keys
+ *   pa_attention_smallseq_bwd  its gradients from the saved attention weights
  *
  * Conventions shared by every call
  * --------------------------------
@@ -299,16 +300,57 @@ pa_status pa_attention_smallseq(const void* q, const void* k, const void* v,
                                 void* out, void* workspace, void* stream);
 
 /*
- * pa_attention_smallseq_ex — pa_attention_smallseq with an element type
- * (PA_DTYPE_BF16 or PA_DTYPE_FP16 for q, k, v and out; the small-seq path of
- * ROCm/TransformerEngine PR #461 takes both).  Other arguments as
- * pa_attention_smallseq.
+ * pa_attention_smallseq_ex — pa_attention_smallseq with an element type and
+ * the attention-weights output of ROCm/TransformerEngine PR #461
+ * (description: the forward also returns the softmax weights, shaped
+ * [batch, Hq, 1, max_seqlen_kv], in the q/k/v dtype, for the backward).
+ *  dtype        PA_DTYPE_BF16 or PA_DTYPE_FP16 for q, k, v, out and weights
+ *  weights      NULL, or [batch, Hq, weights_len] of dtype: entry b's weights
+ *               in the first n_b slots (n_b its key count), zeros after
+ *  weights_len  > 0 when weights is set; an entry with more keys raises
+ *               PA_DEVERR_HINT and keeps its first weights_len weights
+ * Other arguments as pa_attention_smallseq.
  */
 pa_status pa_attention_smallseq_ex(const void* q, const void* k, const void* v,
                                    const int32_t* cu_seqlens_kv, int32_t batch,
                                    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                    int32_t max_seqlen_kv, float scale, int32_t dtype, void* out,
-                                   void* workspace, void* stream);
+                                   void* weights, int32_t weights_len, void* workspace,
+                                   void* stream);
+
+/*
+ * pa_attention_smallseq_bwd — gradients of pa_attention_smallseq_ex.
+ *
+ * Defined by ROCm/TransformerEngine PR #461 (description: the small-seq
+ * backward computes grad_V, grad_attn, the softmax backward and grad_Q /
+ * grad_K, and reads the attention weights the forward wrote into the softmax
+ * auxiliary buffer instead of recomputing them).  With P the saved weights of
+ * query head h over its entry's n keys and dO its upstream gradient:
+ *   dP_j = dO . v_j,  dS_j = P_j (dP_j - sum_k P_k dP_k),
+ *   dQ = scale sum_j dS_j k_j,  dK_j = scale sum_h dS_hj q_h,
+ *   dV_j = sum_h P_hj dO_h  (sums over h run over the query heads of the
+ *   KV head that owns key j).
+ *
+ *  q, dout, dq    [batch, num_q_heads, head_dim] of dtype
+ *  k, v, dk, dv   [cu_seqlens_kv[batch], num_kv_heads, head_dim] of dtype
+ *  weights        [batch, num_q_heads, weights_len] of dtype, as written by
+ *                 pa_attention_smallseq_ex (2-byte aligned)
+ *  weights_len    > 0; an entry with more keys than min(weights_len,
+ *                 max_seqlen_kv) raises PA_DEVERR_HINT and only its first
+ *                 keys are used (the others' dk/dv rows are left unwritten)
+ *  max_seqlen_kv  0..16, num_q_heads / num_kv_heads <= 16 (else
+ *                 PA_ERR_UNSUPPORTED)
+ *  workspace      NULL or the error word, as for the forward
+ * Every dq row is written (zeros for an entry with no keys); every dk/dv row
+ * of a key that belongs to some entry is written once.  Outputs must not
+ * alias inputs.  Supported: head_dim in {64, 128}.
+ */
+pa_status pa_attention_smallseq_bwd(const void* q, const void* k, const void* v,
+                                    const void* dout, const void* weights, int32_t weights_len,
+                                    const int32_t* cu_seqlens_kv, int32_t batch,
+                                    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                    int32_t max_seqlen_kv, float scale, int32_t dtype, void* dq,
+                                    void* dk, void* dv, void* workspace, void* stream);
 
 /*
  * pa_get_error — synchronise `stream`, read the workspace's error word into

@@ -11,7 +11,8 @@ Calls (names as in the C ABI, without the ``pa_`` prefix):
 * ``write_kv(k, v, slot_mapping, k_cache, v_cache)``
 * ``attention_varlen(q, k_cache, v_cache, block_tables, seq_lens,
   query_start_loc, num_kv_heads, scale, causal, out)``
-* ``attention_smallseq(q, k, v, cu_seqlens_kv, scale, out)``
+* ``attention_smallseq(q, k, v, cu_seqlens_kv, scale, out, weights=None)``
+* ``attention_smallseq_bwd(q, k, v, dout, weights, cu_seqlens_kv, scale, dq, dk, dv)``
 * ``get_error(workspace)`` / ``status_string(status)``
 """
 from __future__ import annotations
@@ -25,6 +26,7 @@ import torch
 
 __all__ = [
     "PaError", "library_path", "load", "write_kv", "attention_varlen", "attention_smallseq",
+    "attention_smallseq_bwd",
     "attention_varlen_static", "attention_varlen_spans", "STATIC_SCRATCH_BYTES",
     "varlen_workspace_size", "varlen_workspace", "error_workspace", "get_error",
     "status_string", "version", "EXPORTED_SYMBOLS",
@@ -44,7 +46,7 @@ EXPORTED_SYMBOLS = (
     "pa_write_kv", "pa_attention_varlen_workspace_size", "pa_attention_varlen",
     "pa_attention_smallseq", "pa_get_error", "pa_status_string", "pa_version",
     "pa_attention_varlen_static", "pa_attention_varlen_spans", "pa_write_kv_ex",
-    "pa_attention_varlen_ex", "pa_attention_smallseq_ex",
+    "pa_attention_varlen_ex", "pa_attention_smallseq_ex", "pa_attention_smallseq_bwd",
 )
 DTYPE_BF16, DTYPE_FP16 = 0, 1
 
@@ -106,7 +108,10 @@ def load(build_if_missing: bool = True):
             ctypes.c_float, p, p, i32, p, p, ctypes.c_size_t, p]
         lib.pa_attention_smallseq_ex.restype = ctypes.c_int
         lib.pa_attention_smallseq_ex.argtypes = [p, p, p, p, i32, i32, i32, i32, i32,
-                                                 ctypes.c_float, i32, p, p, p]
+                                                 ctypes.c_float, i32, p, p, i32, p, p]
+        lib.pa_attention_smallseq_bwd.restype = ctypes.c_int
+        lib.pa_attention_smallseq_bwd.argtypes = [p, p, p, p, p, i32, p, i32, i32, i32, i32, i32,
+                                                  ctypes.c_float, i32, p, p, p, p, p]
         lib.pa_attention_smallseq.restype = ctypes.c_int
         lib.pa_attention_smallseq.argtypes = [p, p, p, p, i32, i32, i32, i32, i32,
                                               ctypes.c_float, p, p, p]
@@ -339,9 +344,9 @@ def attention_varlen_static(q, k_cache, v_cache, block_tables, seq_lens, query_s
 
 
 def attention_smallseq(q, k, v, cu_seqlens_kv, scale, out, max_seqlen_kv=16, workspace=None,
-                       stream=None):
+                       stream=None, weights=None):
     """s_q = 1 attention over <= 16 contiguous keys per entry; writes out [B, Hq, D]
-    (bf16 or fp16, like q)."""
+    (bf16 or fp16, like q) and, if given, the attention weights [B, Hq, W]."""
     dt = _element_dtype(q, "q")
     _check(q, "q", dt, 3)
     _check(k, "k", dt, 3)
@@ -352,13 +357,43 @@ def attention_smallseq(q, k, v, cu_seqlens_kv, scale, out, max_seqlen_kv=16, wor
     _, hkv, d_k = k.shape
     if d_k != d or v.shape != k.shape or out.shape != q.shape or cu_seqlens_kv.shape[0] != b + 1:
         raise ValueError("inconsistent small-seq shapes")
+    wp, wlen = None, 0
+    if weights is not None:
+        _check(weights, "weights", dt, 3)
+        if weights.shape[:2] != (b, hq):
+            raise ValueError("weights must be [batch, num_q_heads, W]")
+        wp, wlen = weights.data_ptr(), weights.shape[2]
     ws = workspace.data_ptr() if workspace is not None else None
     st = load().pa_attention_smallseq_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                          cu_seqlens_kv.data_ptr(), b, hq, hkv, d,
                                          int(max_seqlen_kv), float(scale), _DTYPES[dt],
-                                         out.data_ptr(), ws, _stream(stream))
+                                         out.data_ptr(), wp, wlen, ws, _stream(stream))
     _raise(st, "pa_attention_smallseq_ex")
     return out
+
+
+def attention_smallseq_bwd(q, k, v, dout, weights, cu_seqlens_kv, scale, dq, dk, dv,
+                           max_seqlen_kv=16, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of attention_smallseq from its saved weights."""
+    dt = _element_dtype(q, "q")
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (dout, "dout"), (weights, "weights"),
+                    (dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _check(t, name, dt, 3)
+    _check(cu_seqlens_kv, "cu_seqlens_kv", torch.int32, 1)
+    b, hq, d = q.shape
+    _, hkv, d_k = k.shape
+    if (d_k != d or v.shape != k.shape or dk.shape != k.shape or dv.shape != k.shape
+            or dout.shape != q.shape or dq.shape != q.shape or weights.shape[:2] != (b, hq)
+            or cu_seqlens_kv.shape[0] != b + 1):
+        raise ValueError("inconsistent small-seq backward shapes")
+    ws = workspace.data_ptr() if workspace is not None else None
+    st = load().pa_attention_smallseq_bwd(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), weights.data_ptr(),
+        weights.shape[2], cu_seqlens_kv.data_ptr(), b, hq, hkv, d, int(max_seqlen_kv),
+        float(scale), _DTYPES[dt], dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws,
+        _stream(stream))
+    _raise(st, "pa_attention_smallseq_bwd")
+    return dq, dk, dv
 
 
 def get_error(workspace, stream=None):

@@ -332,16 +332,19 @@ pa_status pa_attention_smallseq(const void* q, const void* k, const void* v,
                                 int32_t num_kv_heads, int32_t head_dim, int32_t max_seqlen_kv,
                                 float scale, void* out, void* workspace, void* stream) {
   return pa_attention_smallseq_ex(q, k, v, cu_seqlens_kv, batch, num_q_heads, num_kv_heads,
-                                  head_dim, max_seqlen_kv, scale, PA_DTYPE_BF16, out, workspace,
-                                  stream);
+                                  head_dim, max_seqlen_kv, scale, PA_DTYPE_BF16, out, nullptr, 0,
+                                  workspace, stream);
 }
 
 pa_status pa_attention_smallseq_ex(const void* q, const void* k, const void* v,
                                    const int32_t* cu_seqlens_kv, int32_t batch,
                                    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                    int32_t max_seqlen_kv, float scale, int32_t dtype, void* out,
-                                   void* workspace, void* stream) {
+                                   void* weights, int32_t weights_len, void* workspace,
+                                   void* stream) {
   if (dtype != PA_DTYPE_BF16 && dtype != PA_DTYPE_FP16) return PA_ERR_INVALID_ARG;
+  if (weights && (weights_len <= 0 || (reinterpret_cast<uintptr_t>(weights) & 1u)))
+    return PA_ERR_INVALID_ARG;
   if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
       max_seqlen_kv < 0 || !isfinite(scale))
     return PA_ERR_INVALID_ARG;
@@ -365,8 +368,52 @@ pa_status pa_attention_smallseq_ex(const void* q, const void* k, const void* v,
   p.scale_log2 = scale * 1.4426950408889634f;
   p.out = static_cast<uint16_t*>(out);
   p.err = static_cast<uint32_t*>(workspace);
+  p.weights = static_cast<uint16_t*>(weights);
+  p.weights_len = weights ? weights_len : 0;
   cudaError_t e = pa::launch_smallseq(p, head_dim, dtype == PA_DTYPE_FP16, sm_count(),
                                       static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_attention_smallseq_bwd(const void* q, const void* k, const void* v,
+                                    const void* dout, const void* weights, int32_t weights_len,
+                                    const int32_t* cu_seqlens_kv, int32_t batch,
+                                    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                    int32_t max_seqlen_kv, float scale, int32_t dtype, void* dq,
+                                    void* dk, void* dv, void* workspace, void* stream) {
+  if (dtype != PA_DTYPE_BF16 && dtype != PA_DTYPE_FP16) return PA_ERR_INVALID_ARG;
+  if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
+      max_seqlen_kv < 0 || weights_len <= 0 || !isfinite(scale))
+    return PA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (max_seqlen_kv > 16 || num_q_heads / num_kv_heads > 16) return PA_ERR_UNSUPPORTED;
+  if (batch == 0) return PA_OK;
+  if (!q || !k || !v || !dout || !weights || !cu_seqlens_kv || !dq || !dk || !dv)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(weights) & 1u) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_kv) & 3u) || (workspace && !aligned16(workspace)))
+    return PA_ERR_INVALID_ARG;
+  pa::SmallSeqBwdParams p{};
+  p.q = static_cast<const uint16_t*>(q);
+  p.k = static_cast<const uint16_t*>(k);
+  p.v = static_cast<const uint16_t*>(v);
+  p.dout = static_cast<const uint16_t*>(dout);
+  p.weights = static_cast<const uint16_t*>(weights);
+  p.cu_seqlens_kv = cu_seqlens_kv;
+  p.batch = batch;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.group = num_q_heads / num_kv_heads;
+  p.max_seqlen_kv = max_seqlen_kv;
+  p.weights_len = weights_len;
+  p.scale = scale;
+  p.dq = static_cast<uint16_t*>(dq);
+  p.dk = static_cast<uint16_t*>(dk);
+  p.dv = static_cast<uint16_t*>(dv);
+  p.err = static_cast<uint32_t*>(workspace);
+  cudaError_t e = pa::launch_smallseq_bwd(p, head_dim, dtype == PA_DTYPE_FP16, sm_count(),
+                                          static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

@@ -76,6 +76,20 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // ---------------------------------------------------------------------------
 // packed fp32 pairs (one instruction on two lanes of a 64-bit register pair)
 // ---------------------------------------------------------------------------
+// Packed 16-bit multiply of two element pairs, round to nearest even.
+template <bool H>
+__device__ __forceinline__ uint32_t emul2(uint32_t a, uint32_t b) {
+  if constexpr (H) {
+    const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&a),
+                              *reinterpret_cast<const __half2*>(&b));
+    return *reinterpret_cast<const uint32_t*>(&r);
+  } else {
+    const __nv_bfloat162 r = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&a),
+                                     *reinterpret_cast<const __nv_bfloat162*>(&b));
+    return *reinterpret_cast<const uint32_t*>(&r);
+  }
+}
+
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   return ((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo);
 }
@@ -237,6 +251,16 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* map, uint6
       "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
+// Start the line holding `ptr` towards L1 (no register is written).
+__device__ __forceinline__ void prefetch_l1(const void* ptr) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(ptr));
+}
+
+// Start the line holding `ptr` towards L2.
+__device__ __forceinline__ void prefetch_l2(const void* ptr) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+}
+
 __device__ __forceinline__ void prefetch_tma_desc(const void* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }

@@ -88,8 +88,33 @@ struct SmallSeqParams {
   float scale_log2;
   uint16_t* out;  // elements of the kernel's type (bf16 or fp16)
   uint32_t* err;
+  uint16_t* weights;  // optional [batch, Hq, weights_len] attention weights
+  int weights_len;
 };
 cudaError_t launch_smallseq(const SmallSeqParams& p, int head_dim, bool fp16, int num_sms,
                             cudaStream_t stream);
+
+// Backward of the small-seq attention from the forward's saved weights.
+struct SmallSeqBwdParams {
+  const uint16_t* q;        // [batch, Hq, D]
+  const uint16_t* k;        // [total_kv, Hkv, D]
+  const uint16_t* v;        // [total_kv, Hkv, D]
+  const uint16_t* dout;     // [batch, Hq, D]
+  const uint16_t* weights;  // [batch, Hq, weights_len]
+  const int32_t* cu_seqlens_kv;
+  int batch;
+  int num_q_heads;
+  int num_kv_heads;
+  int group;
+  int max_seqlen_kv;
+  int weights_len;
+  float scale;
+  uint16_t* dq;  // [batch, Hq, D]
+  uint16_t* dk;  // [total_kv, Hkv, D]
+  uint16_t* dv;  // [total_kv, Hkv, D]
+  uint32_t* err;
+};
+cudaError_t launch_smallseq_bwd(const SmallSeqBwdParams& p, int head_dim, bool fp16, int num_sms,
+                                cudaStream_t stream);
 
 }  // namespace pa

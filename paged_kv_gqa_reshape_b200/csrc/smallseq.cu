@@ -120,6 +120,9 @@ __global__ void __launch_bounds__(256, 3) smallseq_kernel(SmallSeqParams p) {
     // NP passes of KPP keys, straight-line (the shuffle trees of all passes
     // overlap); NP is the smallest power of two covering the entry's keys
     float sum = 0.f, acc[8];
+    float pwv[PASSES];  // unnormalised weight of this lane's key in each pass
+#pragma unroll
+    for (int pp = 0; pp < PASSES; ++pp) pwv[pp] = 0.f;
     auto attend = [&](auto np_tag) {
       constexpr int NP = decltype(np_tag)::value;
       float sc[NP];
@@ -152,6 +155,7 @@ __global__ void __launch_bounds__(256, 3) smallseq_kernel(SmallSeqParams p) {
       for (int pp = 0; pp < NP; ++pp) {
         const float pw = (sc[pp] == -INFINITY) ? 0.f : fast_exp2(sc[pp] - m);
         sum += pw;
+        pwv[pp] = pw;
         const uint32_t w[4] = {cur.v[pp].x, cur.v[pp].y, cur.v[pp].z, cur.v[pp].w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -174,6 +178,18 @@ __global__ void __launch_bounds__(256, 3) smallseq_kernel(SmallSeqParams p) {
       sum += __shfl_xor_sync(0xffffffffu, sum, o);
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+    }
+    if (p.weights) {
+      // attention weights [batch, Hq, weights_len]: the entry's softmax, then zeros
+      const float winv = sum > 0.f ? 1.f / sum : 0.f;
+      uint16_t* wrow = p.weights + ((size_t)b * p.num_q_heads + h) * p.weights_len;
+      if (cur.n > p.weights_len && lane == 0) raise_error(p.err, PA_DEVERR_HINT);
+#pragma unroll
+      for (int pp = 0; pp < PASSES; ++pp) {
+        const int j = pp * KPP + sub;
+        if (l == 0 && j < cur.n && j < p.weights_len) wrow[j] = ebits<H>(pwv[pp] * winv);
+      }
+      for (int j = cur.n + lane; j < p.weights_len; j += 32) wrow[j] = 0;
     }
     if (sub == 0) {
       const float inv = sum > 0.f ? 1.f / sum : 0.f;  // an empty entry writes zeros
