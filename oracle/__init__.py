@@ -67,6 +67,10 @@ def _load():
         lib.oracle_attention_varlen_dtype.restype = i32
         lib.oracle_attention_varlen_dtype.argtypes = [
             p, p, p, p, p, p, i32, i32, i32, i32, f64, i32, i32, p, i64, p]
+        lib.oracle_attention_varlen_mods.restype = i32
+        lib.oracle_attention_varlen_mods.argtypes = [
+            p, p, p, p, p, p, i32, i32, i32, i32, f64, i32, i32, f64, p, p, i64, i64, p, i64,
+            p]
         lib.oracle_attention_smallseq_dtype.restype = i32
         lib.oracle_attention_smallseq_dtype.argtypes = [p, p, p, p, i32, i32, i32, i32, f64, i32, p]
         lib.oracle_smallseq_weights.restype = i32
@@ -150,6 +154,34 @@ def attention_varlen_dtype(q, k_seq, v_seq, kv_offsets, seq_lens, query_start_lo
         _ptr(rows_a), 0 if rows_a is None else len(rows_a), _ptr(out))
     if rc != 0:
         raise ValueError(f"oracle_attention_varlen_dtype failed ({rc})")
+    return out
+
+
+def attention_varlen_mods(q, k_seq, v_seq, kv_offsets, seq_lens, query_start_loc,
+                          num_kv_heads, scale, causal, dtype=0, softcap=0.0, alibi_slopes=None,
+                          mask=None, mask_head_stride=0, mask_token_stride=0, rows=None):
+    """attention_varlen with score modifiers: soft-cap (0 = off), ALiBi slopes
+    [Hq] float32 or None, an additive float32 mask (flat array addressed as
+    h * mask_head_stride + t * mask_token_stride + j) or None."""
+    q = _arr(q, np.uint16)
+    k_seq, v_seq = _arr(k_seq, np.uint16), _arr(v_seq, np.uint16)
+    kv_offsets = _arr(kv_offsets, np.int64)
+    seq_lens = _arr(seq_lens, np.int32)
+    qsl = _arr(query_start_loc, np.int32)
+    slopes = None if alibi_slopes is None else _arr(alibi_slopes, np.float32)
+    mk = None if mask is None else _arr(mask, np.float32)
+    t, hq, d = q.shape
+    if slopes is not None and slopes.shape != (hq,):
+        raise ValueError("alibi_slopes must be [num_q_heads]")
+    out = np.zeros((t, hq, d), dtype=np.float64)
+    rows_a = None if rows is None else _arr(rows, np.int64)
+    rc = _load().oracle_attention_varlen_mods(
+        _ptr(q), _ptr(k_seq), _ptr(v_seq), _ptr(kv_offsets), _ptr(seq_lens), _ptr(qsl),
+        len(seq_lens), hq, num_kv_heads, d, float(scale), int(bool(causal)), int(dtype),
+        float(softcap), _ptr(slopes), _ptr(mk), int(mask_head_stride), int(mask_token_stride),
+        _ptr(rows_a), 0 if rows_a is None else len(rows_a), _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_attention_varlen_mods failed ({rc})")
     return out
 
 

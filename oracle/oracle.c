@@ -201,14 +201,34 @@ static int64_t visible_keys_spans(int64_t p, int64_t len_kv, const int32_t *sp,
 }
 
 /*
+ * Score modifiers of one (query token, head) row, auto_round_kernel PR
+ * "Migrate CPU SDPA backend" (description: additive masks in the public
+ * sdpa(); ALiBi slopes and the TANH30 soft-cap among the kernel library's
+ * extensions).  Applied to s_j = scale * <q, k_j> in this order:
+ *   soft-cap  s_j <- softcap * tanh(s_j / softcap)          (softcap > 0)
+ *   ALiBi     s_j <- s_j + slope * (j - pos)                (has_alibi)
+ *   mask      s_j <- s_j + mask_row[j]                      (mask_row)
+ * where pos is the query's own key position.  Masking (causal, spans,
+ * sequence end) still decides which keys enter the softmax at all.
+ */
+typedef struct {
+    double softcap;
+    int has_alibi;
+    double slope;
+    int64_t pos;
+    const float *mask_row;
+} row_mods;
+
+/*
  * out[d] = sum_j w_j v_j[d],  w_j = exp(s_j) / sum_i exp(s_i),
- * s_j = scale * <q, k_j>, over keys j < n_vis.  n_vis == 0 gives zeros.
+ * s_j = scale * <q, k_j> (then the row's modifiers, if any), over keys
+ * j < n_vis.  n_vis == 0, or every visible s_j = -inf, gives zeros.
  * The maximum is subtracted inside exp only to keep it finite; it cancels in
  * the ratio.  Returns -1 if some key or value row is unreadable.
  */
 static int attention_row(const uint16_t *q, const kv_view *keys,
                          const kv_view *values, int64_t n_vis, int head_dim,
-                         double scale, double *out, double *weights,
+                         double scale, const row_mods *mods, double *out, double *weights,
                          double *s) {
     for (int d = 0; d < head_dim; ++d) out[d] = 0.0;
     if (n_vis <= 0) return 0;
@@ -220,8 +240,14 @@ static int attention_row(const uint16_t *q, const kv_view *keys,
         for (int d = 0; d < head_dim; ++d)
             dot += keys->widen(q[d]) * keys->widen(kr[d]);
         s[j] = scale * dot;
+        if (mods) {
+            if (mods->softcap > 0.0) s[j] = mods->softcap * tanh(s[j] / mods->softcap);
+            if (mods->has_alibi) s[j] += mods->slope * (double)(j - mods->pos);
+            if (mods->mask_row) s[j] += (double)mods->mask_row[j];
+        }
         if (s[j] > m) m = s[j];
     }
+    if (m == -INFINITY) return 0; /* every visible key masked out */
     double denom = 0.0;
     for (int64_t j = 0; j < n_vis; ++j) {
         s[j] = exp(s[j] - m);
@@ -241,6 +267,17 @@ static int attention_row(const uint16_t *q, const kv_view *keys,
 /* Variable-length attention (prefill, decode, chunked prefill)              */
 /* ------------------------------------------------------------------------ */
 
+/* Score modifiers of a whole call: alibi_slopes [num_q_heads] or NULL; mask
+   element (h, t, j) at mask[h * mask_head_stride + t * mask_token_stride + j]
+   (t the packed query-token index, j the key position) or NULL. */
+typedef struct {
+    double softcap;
+    const float *alibi_slopes;
+    const float *mask;
+    int64_t mask_head_stride;
+    int64_t mask_token_stride;
+} score_mods;
+
 /*
  * Shared driver.  For every requested query token t (all tokens if rows is
  * NULL): find its sequence s, its index i within the sequence, and for every
@@ -255,6 +292,7 @@ static int varlen_driver(const uint16_t *q, const uint16_t *k_base,
                          int num_seqs, int num_q_heads, int num_kv_heads,
                          int head_dim, double scale, int causal,
                          const int32_t *span_offsets, const int32_t *spans, int dtype,
+                         const score_mods *sm,
                          const int64_t *rows, int64_t num_rows, double *out) {
     double (*widen)(uint16_t) = dtype == 1 ? half_to_double : bf16_to_double;
     if (num_kv_heads <= 0 || num_q_heads <= 0 || num_q_heads % num_kv_heads != 0)
@@ -303,7 +341,18 @@ static int varlen_driver(const uint16_t *q, const uint16_t *k_base,
                 }
                 const uint16_t *qr = q + (t * num_q_heads + h) * (int64_t)head_dim;
                 double *o = out + (t * num_q_heads + h) * (int64_t)head_dim;
-                if (attention_row(qr, &kview, &vview, n_vis, head_dim, scale, o,
+                row_mods rm, *rmp = NULL;
+                if (sm) {
+                    rm.softcap = sm->softcap;
+                    rm.has_alibi = sm->alibi_slopes != NULL;
+                    rm.slope = sm->alibi_slopes ? (double)sm->alibi_slopes[h] : 0.0;
+                    rm.pos = (len_kv - len_q) + i;
+                    rm.mask_row = sm->mask ? sm->mask + h * sm->mask_head_stride +
+                                                 t * sm->mask_token_stride
+                                           : NULL;
+                    rmp = &rm;
+                }
+                if (attention_row(qr, &kview, &vview, n_vis, head_dim, scale, rmp, o,
                                   NULL, scratch) != 0) {
 #pragma omp atomic write
                     status = -2;
@@ -335,7 +384,7 @@ int oracle_attention_varlen(const uint16_t *q, const uint16_t *k_seq,
                             int64_t num_rows, double *out) {
     return varlen_driver(q, k_seq, v_seq, kv_offsets, NULL, 0, 1, 0, seq_lens,
                          query_start_loc, num_seqs, num_q_heads, num_kv_heads,
-                         head_dim, scale, causal, NULL, NULL, 0, rows, num_rows, out);
+                         head_dim, scale, causal, NULL, NULL, 0, NULL, rows, num_rows, out);
 }
 
 /*
@@ -352,7 +401,7 @@ int oracle_attention_varlen_dtype(const uint16_t *q, const uint16_t *k_seq,
     if (dtype != 0 && dtype != 1) return -1;
     return varlen_driver(q, k_seq, v_seq, kv_offsets, NULL, 0, 1, 0, seq_lens,
                          query_start_loc, num_seqs, num_q_heads, num_kv_heads,
-                         head_dim, scale, causal, NULL, NULL, dtype, rows, num_rows, out);
+                         head_dim, scale, causal, NULL, NULL, dtype, NULL, rows, num_rows, out);
 }
 
 /*
@@ -372,7 +421,29 @@ int oracle_attention_varlen_spans(const uint16_t *q, const uint16_t *k_seq,
     if (!span_offsets || !spans) return -1;
     return varlen_driver(q, k_seq, v_seq, kv_offsets, NULL, 0, 1, 0, seq_lens,
                          query_start_loc, num_seqs, num_q_heads, num_kv_heads,
-                         head_dim, scale, 1, span_offsets, spans, 0, rows, num_rows, out);
+                         head_dim, scale, 1, span_offsets, spans, 0, NULL, rows, num_rows, out);
+}
+
+/*
+ * Logical form with score modifiers (see row_mods) and an element type:
+ * softcap (0 = off), alibi_slopes [num_q_heads] fp32 or NULL, an additive
+ * fp32 mask or NULL with its head / token strides in elements (head stride 0
+ * = one mask for every head).  Otherwise as oracle_attention_varlen_dtype.
+ */
+int oracle_attention_varlen_mods(const uint16_t *q, const uint16_t *k_seq,
+                                 const uint16_t *v_seq, const int64_t *kv_offsets,
+                                 const int32_t *seq_lens,
+                                 const int32_t *query_start_loc, int num_seqs,
+                                 int num_q_heads, int num_kv_heads, int head_dim,
+                                 double scale, int causal, int dtype, double softcap,
+                                 const float *alibi_slopes, const float *mask,
+                                 int64_t mask_head_stride, int64_t mask_token_stride,
+                                 const int64_t *rows, int64_t num_rows, double *out) {
+    if ((dtype != 0 && dtype != 1) || softcap < 0.0) return -1;
+    score_mods sm = {softcap, alibi_slopes, mask, mask_head_stride, mask_token_stride};
+    return varlen_driver(q, k_seq, v_seq, kv_offsets, NULL, 0, 1, 0, seq_lens,
+                         query_start_loc, num_seqs, num_q_heads, num_kv_heads,
+                         head_dim, scale, causal, NULL, NULL, dtype, &sm, rows, num_rows, out);
 }
 
 /*
@@ -392,7 +463,7 @@ int oracle_attention_varlen_paged(const uint16_t *q, const uint16_t *k_cache,
     return varlen_driver(q, k_cache, v_cache, NULL, block_tables,
                          max_blocks_per_seq, block_size, num_blocks, seq_lens,
                          query_start_loc, num_seqs, num_q_heads, num_kv_heads,
-                         head_dim, scale, causal, NULL, NULL, 0, rows, num_rows, out);
+                         head_dim, scale, causal, NULL, NULL, 0, NULL, rows, num_rows, out);
 }
 
 /*
@@ -426,7 +497,7 @@ int64_t oracle_attention_weights(const uint16_t *q, const uint16_t *k_seq,
     double *scratch = (double *)malloc(sizeof(double) * (size_t)(len_kv > 0 ? len_kv : 1));
     for (int64_t j = 0; j < len_kv; ++j) weights[j] = 0.0;
     const uint16_t *qr = q + (t * num_q_heads + h) * (int64_t)head_dim;
-    attention_row(qr, &kview, &vview, n_vis, head_dim, scale, out, weights, scratch);
+    attention_row(qr, &kview, &vview, n_vis, head_dim, scale, NULL, out, weights, scratch);
     free(out);
     free(scratch);
     return n_vis;
@@ -473,7 +544,7 @@ static int smallseq_driver(const uint16_t *q, const uint16_t *k,
                 kview.widen = vview.widen = widen;
                 const uint16_t *qr = q + ((int64_t)b * num_q_heads + h) * head_dim;
                 double *o = out + ((int64_t)b * num_q_heads + h) * head_dim;
-                attention_row(qr, &kview, &vview, n, head_dim, scale, o, NULL,
+                attention_row(qr, &kview, &vview, n, head_dim, scale, NULL, o, NULL,
                               scratch);
             }
         }
