@@ -14,6 +14,7 @@ oracle on a bounded sample of the same workload instead.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -41,8 +42,8 @@ WORKLOAD = ("decode_batch: 64 seqs x 1 query token, context U[256,4096], Hq 32 /
 # DRAM bytes (read + write) of one decode-kernel launch on the decode batch, from
 # one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), valid only
 # while the decode kernel's sources hash to the recorded value.
-DECODE_TRAFFIC = {"sources_sha256": "07ce11a1d40b6984b387a080d68b9b495006c352d187f420f1dc59f28686cd59",
-                  "bytes_per_launch": 598826325}
+DECODE_TRAFFIC = {"sources_sha256": "27d1950fd81545274f0896d06a290df7089fd77daaec348d0dcdc1957b9c94eb",
+                  "bytes_per_launch": 599209899}
 DECODE_SOURCES = ("decode.cu", "common.cuh", "layout.h")
 
 
@@ -227,8 +228,9 @@ def device_case(case, dev):
     return type(case)(**kw)
 
 
-def time_varlen_component(pa, case, iters=20, warmup=3, with_scatter=False):
-    """Average device time (ms) of one attention_varlen call on `case` (device tensors)."""
+def time_varlen_component(pa, case, iters=20, warmup=3, with_scatter=False, **mods):
+    """Average device time (ms) of one attention_varlen call on `case` (device
+    tensors); `mods` (softcap, alibi_slopes, mask) go to the call."""
     ws = pa.varlen_workspace(case.num_seqs, case.num_q_tokens, case.num_q_heads,
                              case.num_kv_heads, case.head_dim)
     out = torch.empty_like(case.q)
@@ -239,7 +241,7 @@ def time_varlen_component(pa, case, iters=20, warmup=3, with_scatter=False):
             pa.write_kv(case.k_new, case.v_new, case.slot_mapping, case.k_cache, case.v_cache)
         pa.attention_varlen(case.q, case.k_cache, case.v_cache, case.block_tables, case.seq_lens,
                             case.query_start_loc, case.num_kv_heads, case.scale, case.causal, out,
-                            max_query_len=mql, max_seq_len=msl, workspace=ws)
+                            max_query_len=mql, max_seq_len=msl, workspace=ws, **mods)
 
     if not with_scatter:
         pa.write_kv(case.k_new, case.v_new, case.slot_mapping, case.k_cache, case.v_cache)
@@ -378,6 +380,32 @@ def components(pa, hbm_peak, tc_peak, peak_kind):
     res["decode_batch_fp16"] = {"ms": round(ms, 4), "gbs": round(gbs, 1),
                                 "frac": round(gbs / hbm_peak, 3), "unit": "GB/s", "of": peak_kind}
     del dc16
+    # score modifiers: the prefill workload with ALiBi slopes and the TANH30
+    # soft-cap (no extra bytes); the decode workload over head-major caches
+    # with a shared additive mask (its [64, 4096] fp32 rows are counted)
+    vc = workloads.varlen_prefill(device=dev, keep_logical=False)
+    slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / vc.num_q_heads)
+                           for h in range(vc.num_q_heads)], device=dev)
+    ms = time_varlen_component(pa, vc, softcap=30.0, alibi_slopes=slopes)
+    tf = attention_flops(vc) / (ms * 1e-3) / 1e12
+    res["varlen_prefill_alibi_softcap"] = {"ms": round(ms, 4), "tflops": round(tf, 1),
+                                           "frac": round(tf / tc_peak, 3), "peak": tc_peak,
+                                           "unit": "TFLOP/s", "of": peak_kind}
+    del vc, slopes
+    dc = workloads.decode_batch(device=dev, keep_logical=False)
+    hnd = dataclasses.replace(
+        dc, k_cache=dc.k_cache.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3),
+        v_cache=dc.v_cache.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3))
+    del dc
+    mlen = (hnd.max_seq_len + 3) // 4 * 4
+    mask = torch.randn(hnd.num_q_tokens, mlen, generator=workloads._gen(1008, dev), device=dev)
+    ms = time_varlen_component(pa, hnd, iters=50, mask=mask)
+    mask_bytes = 4 * sum(int(x) for x in hnd.seq_lens.tolist())
+    gbs = (attention_bytes(hnd) + mask_bytes) / (ms * 1e-3) / 1e9
+    res["decode_batch_hnd_mask"] = {"ms": round(ms, 4), "gbs": round(gbs, 1),
+                                    "frac": round(gbs / hbm_peak, 3), "unit": "GB/s",
+                                    "of": peak_kind}
+    del hnd, mask
     sc, so, sp = workloads.spans_prefill(device=dev, keep_logical=False)
     ms = time_spans_component(pa, sc, so, sp)
     pairs = workloads.spans_visible_pairs(sc.seq_lens.tolist(), sc.query_lens.tolist(),

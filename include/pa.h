@@ -10,12 +10,15 @@
  *   pa_attention_smallseq  one query per batch entry over a handful (<= 16) of
  *                          contiguous keys
  *   pa_attention_smallseq_bwd  its gradients from the saved attention weights
+ *   pa_attention_varlen_mods   varlen attention with score modifiers (soft-cap,
+ *                          ALiBi, additive mask) and head-major layouts
  *
  * Conventions shared by every call
  * --------------------------------
  *  - Element type: bfloat16 for every Q/K/V/cache/output tensor (passed as
  *    void*, 2 bytes per element).  Index tensors are int32 unless stated.
- *  - Layout: token-major ("NHD"), dense, innermost dimension last:
+ *  - Layout (every entry point but the _mods / _strided ones, which take
+ *    pa_strides): token-major ("NHD"), dense, innermost dimension last:
  *      q, out           [num_tokens, num_q_heads, head_dim]
  *      k, v (new rows)  [num_tokens, num_kv_heads, head_dim]
  *      k_cache, v_cache [num_blocks, block_size, num_kv_heads, head_dim]
@@ -274,6 +277,82 @@ pa_status pa_attention_varlen_static(const void* q, const void* k_cache, const v
                                      int32_t head_dim, int32_t block_size, int64_t num_blocks,
                                      int32_t max_query_len, int32_t max_seq_len, float scale,
                                      int32_t causal, void* out, void* stream);
+
+/*
+ * Layouts: element strides of q, out and the paged caches (the innermost
+ * head_dim elements of a row are always contiguous).  The HND / NHD layouts
+ * of auto_round_kernel PR "Migrate CPU SDPA backend" (description: the public
+ * sdpa() takes head-major or token-major tensors) are two settings of it:
+ *   q / out NHD [T, H, D]: token = H*D, head = D
+ *   q / out HND [H, T, D]: token = D,   head = T*D
+ *   cache NHD [num_blocks, block_size, Hkv, D]: block = BS*Hkv*D, slot = Hkv*D, head = D
+ *   cache HND [num_blocks, Hkv, block_size, D]: block = BS*Hkv*D, slot = D, head = BS*D
+ * (padding between rows or blocks is allowed).  A pair (token, head) or
+ * triple (block, slot, head) of zeros means the dense NHD layout.  Every
+ * stride is a multiple of 8 elements; rows must not overlap: either
+ * head >= D and token >= H*head (token-major) or token >= D and head >=
+ * T*token (head-major); for the cache either head >= D and slot >=
+ * Hkv*head, or slot >= D and head >= block_size*slot, and block >= the
+ * extent of one block.  Anything else is PA_ERR_UNSUPPORTED.
+ */
+typedef struct pa_strides {
+  int64_t q_token, q_head;
+  int64_t out_token, out_head;
+  int64_t cache_block, cache_slot, cache_head;
+} pa_strides;
+
+/*
+ * Score modifiers (auto_round_kernel PR "Migrate CPU SDPA backend",
+ * description: additive masks in the public sdpa(); ALiBi slopes and the
+ * TANH30 soft-cap among the library's extensions).  With s = scale*<q, k_j>
+ * for query token t (key position pos within its sequence) and head h:
+ *   softcap > 0:   s <- softcap * tanh(s / softcap)      (TANH30: softcap = 30)
+ *   alibi_slopes:  s <- s + alibi_slopes[h] * (j - pos)
+ *   mask:          s <- s + mask[h * mask_head_stride + t * mask_token_stride + j]
+ * in that order; causal / span / sequence-end masking then decides which
+ * keys enter the softmax, and a row whose visible scores are all -inf gives
+ * zeros.  alibi_slopes: NULL or [num_q_heads] fp32.  mask: NULL or fp32,
+ * 16-byte aligned, entries finite or -inf; t is the packed query-token
+ * index; mask_head_stride 0 shares one mask across heads; both strides are
+ * multiples of 4; mask_len is the number of keys a mask row holds: a key at
+ * or beyond it gets no mask value and raises PA_DEVERR_HINT.
+ */
+typedef struct pa_score_mods {
+  float softcap;
+  const float* alibi_slopes;
+  const float* mask;
+  int64_t mask_head_stride;
+  int64_t mask_token_stride;
+  int64_t mask_len;
+} pa_score_mods;
+
+/*
+ * pa_write_kv_strided — pa_write_kv_ex into caches of any layout above
+ * (strides NULL: dense NHD).  k and v stay dense [num_tokens, Hkv, D].
+ */
+pa_status pa_write_kv_strided(const void* k, const void* v, const int64_t* slot_mapping,
+                              int64_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                              void* k_cache, void* v_cache, int64_t num_blocks,
+                              int32_t block_size, const pa_strides* strides, int32_t dtype,
+                              void* workspace, void* stream);
+
+/*
+ * pa_attention_varlen_mods — pa_attention_varlen_ex with layouts (strides:
+ * NULL = dense NHD everywhere; its cache_block replaces block_stride) and
+ * score modifiers (mods: NULL or all off = none).  Other arguments, the
+ * workspace and the errors as pa_attention_varlen_ex.
+ */
+pa_status pa_attention_varlen_mods(const void* q, const void* k_cache, const void* v_cache,
+                                   const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                   const int32_t* seq_lens, const int32_t* query_start_loc,
+                                   int32_t num_seqs, int64_t num_q_tokens, int32_t num_q_heads,
+                                   int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                   int64_t num_blocks, int32_t dtype, int32_t max_query_len,
+                                   int32_t max_seq_len, float scale, int32_t causal,
+                                   const int32_t* span_offsets, const int32_t* spans,
+                                   int32_t num_spans, const pa_strides* strides,
+                                   const pa_score_mods* mods, void* out, void* workspace,
+                                   size_t workspace_bytes, void* stream);
 
 /*
  * pa_attention_smallseq — s_q = 1 cross attention over short contiguous KV.

@@ -47,6 +47,7 @@ EXPORTED_SYMBOLS = (
     "pa_attention_smallseq", "pa_get_error", "pa_status_string", "pa_version",
     "pa_attention_varlen_static", "pa_attention_varlen_spans", "pa_write_kv_ex",
     "pa_attention_varlen_ex", "pa_attention_smallseq_ex", "pa_attention_smallseq_bwd",
+    "pa_write_kv_strided", "pa_attention_varlen_mods",
 )
 DTYPE_BF16, DTYPE_FP16 = 0, 1
 
@@ -102,6 +103,12 @@ def load(build_if_missing: bool = True):
         lib.pa_attention_varlen_ex.argtypes = [
             p, p, p, p, i32, p, p, i32, i64, i32, i32, i32, i32, i64, i64, i32, i32, i32,
             ctypes.c_float, i32, p, p, i32, p, p, ctypes.c_size_t, p]
+        lib.pa_write_kv_strided.restype = ctypes.c_int
+        lib.pa_write_kv_strided.argtypes = [p, p, p, i64, i32, i32, p, p, i64, i32, p, i32, p, p]
+        lib.pa_attention_varlen_mods.restype = ctypes.c_int
+        lib.pa_attention_varlen_mods.argtypes = [
+            p, p, p, p, i32, p, p, i32, i64, i32, i32, i32, i32, i64, i32, i32, i32,
+            ctypes.c_float, i32, p, p, i32, p, p, p, p, ctypes.c_size_t, p]
         lib.pa_attention_varlen_spans.restype = ctypes.c_int
         lib.pa_attention_varlen_spans.argtypes = [
             p, p, p, p, i32, p, p, i32, i64, i32, i32, i32, i32, i64, i32, i32,
@@ -185,10 +192,26 @@ def _element_dtype(t, name):
     return t.dtype
 
 
+class _Strides(ctypes.Structure):
+    """pa_strides (include/pa.h)."""
+    _fields_ = [("q_token", ctypes.c_int64), ("q_head", ctypes.c_int64),
+                ("out_token", ctypes.c_int64), ("out_head", ctypes.c_int64),
+                ("cache_block", ctypes.c_int64), ("cache_slot", ctypes.c_int64),
+                ("cache_head", ctypes.c_int64)]
+
+
+class _ScoreMods(ctypes.Structure):
+    """pa_score_mods (include/pa.h)."""
+    _fields_ = [("softcap", ctypes.c_float), ("alibi_slopes", ctypes.c_void_p),
+                ("mask", ctypes.c_void_p), ("mask_head_stride", ctypes.c_int64),
+                ("mask_token_stride", ctypes.c_int64), ("mask_len", ctypes.c_int64)]
+
+
 def _check_caches(k_cache, v_cache, dtype):
-    """Caches [NB, BS, Hkv, D] whose rows are contiguous and whose blocks are
-    block_stride elements apart (views of one [NB, 2, BS, Hkv, D] tensor are
-    fine).  Returns block_stride."""
+    """Caches indexed [NB, BS, Hkv, D] with D contiguous and any block / slot /
+    head strides (views of one [NB, 2, BS, Hkv, D] tensor, or a head-major
+    [NB, Hkv, BS, D] tensor permuted to [NB, BS, Hkv, D], are fine).  Returns
+    the (block, slot, head) element strides; the library checks the layout."""
     for t, name in ((k_cache, "k_cache"), (v_cache, "v_cache")):
         if not isinstance(t, torch.Tensor) or t.dtype != dtype:
             raise TypeError(f"{name} must be a {dtype} tensor")
@@ -196,26 +219,41 @@ def _check_caches(k_cache, v_cache, dtype):
             raise ValueError(f"{name} must be a CUDA tensor")
         if t.dim() != 4:
             raise ValueError(f"{name} must have 4 dims [NB, BS, Hkv, D]")
-        nb, bs, hkv, d = t.shape
-        if t.stride(3) != 1 or t.stride(2) != d or t.stride(1) != hkv * d or t.stride(0) < bs * hkv * d:
-            raise ValueError(f"{name}: rows must be contiguous [BS, Hkv, D] blocks")
+        if t.stride(3) != 1:
+            raise ValueError(f"{name}: head_dim must be contiguous")
     if v_cache.shape != k_cache.shape or v_cache.stride() != k_cache.stride():
         raise ValueError("k_cache and v_cache must have the same shape and strides")
-    return k_cache.stride(0)
+    return k_cache.stride(0), k_cache.stride(1), k_cache.stride(2)
+
+
+def _dense_rows(cstr, hkv, d):
+    return cstr[1] == hkv * d and cstr[2] == d
+
+
+def _check_rows(t, name, dtype):
+    """[T, H, D] with D contiguous and any token / head strides; returns them."""
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype:
+        raise TypeError(f"{name} must be a {dtype} tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != 3 or t.stride(2) != 1:
+        raise ValueError(f"{name} must be [T, H, D] with D contiguous")
+    return t.stride(0), t.stride(1)
 
 
 def write_kv(k, v, slot_mapping, k_cache, v_cache, workspace=None, stream=None):
     """Scatter k/v [T, Hkv, D] into the paged caches at slot_mapping (int64 [T]).
 
-    k_cache / v_cache: [NB, BS, Hkv, D], bf16 or fp16 like k and v; separate
-    tensors, or the two halves kv[:, 0] / kv[:, 1] of one [NB, 2, BS, Hkv, D]
-    cache.
+    k_cache / v_cache: indexed [NB, BS, Hkv, D], bf16 or fp16 like k and v;
+    separate tensors, the two halves kv[:, 0] / kv[:, 1] of one
+    [NB, 2, BS, Hkv, D] cache, or head-major caches [NB, Hkv, BS, D] passed
+    as their .permute(0, 2, 1, 3) views.
     """
     dt = _element_dtype(k, "k")
     _check(k, "k", dt, 3)
     _check(v, "v", dt, 3)
     _check(slot_mapping, "slot_mapping", torch.int64, 1)
-    stride = _check_caches(k_cache, v_cache, dt)
+    cstr = _check_caches(k_cache, v_cache, dt)
     t, hkv, d = k.shape
     if v.shape != k.shape or slot_mapping.shape[0] != t:
         raise ValueError("k, v and slot_mapping disagree on the token count / shape")
@@ -223,22 +261,53 @@ def write_kv(k, v, slot_mapping, k_cache, v_cache, workspace=None, stream=None):
     if hkv_c != hkv or d_c != d:
         raise ValueError("cache shape does not match k/v")
     ws = workspace.data_ptr() if workspace is not None else None
-    st = load().pa_write_kv_ex(k.data_ptr(), v.data_ptr(), slot_mapping.data_ptr(), t, hkv, d,
-                               k_cache.data_ptr(), v_cache.data_ptr(), nb, bs, stride,
-                               _DTYPES[dt], ws, _stream(stream))
-    _raise(st, "pa_write_kv_ex")
+    if _dense_rows(cstr, hkv, d):
+        st = load().pa_write_kv_ex(k.data_ptr(), v.data_ptr(), slot_mapping.data_ptr(), t, hkv,
+                                   d, k_cache.data_ptr(), v_cache.data_ptr(), nb, bs, cstr[0],
+                                   _DTYPES[dt], ws, _stream(stream))
+        _raise(st, "pa_write_kv_ex")
+        return
+    strides = _Strides(0, 0, 0, 0, *cstr)
+    st = load().pa_write_kv_strided(k.data_ptr(), v.data_ptr(), slot_mapping.data_ptr(), t, hkv,
+                                    d, k_cache.data_ptr(), v_cache.data_ptr(), nb, bs,
+                                    ctypes.byref(strides), _DTYPES[dt], ws, _stream(stream))
+    _raise(st, "pa_write_kv_strided")
+
+
+def _score_mods(softcap, alibi_slopes, mask, hq):
+    """pa_score_mods for the call, or None when every modifier is off."""
+    if not softcap and alibi_slopes is None and mask is None:
+        return None
+    m = _ScoreMods(float(softcap or 0.0), None, None, 0, 0, 0)
+    if alibi_slopes is not None:
+        _check(alibi_slopes, "alibi_slopes", torch.float32, 1)
+        if alibi_slopes.shape[0] != hq:
+            raise ValueError("alibi_slopes must be [num_q_heads]")
+        m.alibi_slopes = alibi_slopes.data_ptr()
+    if mask is not None:
+        if not isinstance(mask, torch.Tensor) or mask.dtype != torch.float32 or not mask.is_cuda:
+            raise TypeError("mask must be a float32 CUDA tensor")
+        if mask.dim() not in (2, 3) or mask.stride(-1) != 1:
+            raise ValueError("mask must be [T, L] or [Hq, T, L] with L contiguous")
+        if mask.dim() == 3 and mask.shape[0] != hq:
+            raise ValueError("a 3-D mask must be [num_q_heads, T, L]")
+        m.mask = mask.data_ptr()
+        m.mask_token_stride = mask.stride(-2)
+        m.mask_head_stride = mask.stride(0) if mask.dim() == 3 else 0
+        m.mask_len = mask.shape[-1]
+    return m
 
 
 def _varlen_ex(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc, num_kv_heads,
                scale, causal, span_offsets, spans, out, max_query_len, max_seq_len, workspace,
-               stream, what):
+               stream, what, softcap=0.0, alibi_slopes=None, mask=None):
     dt = _element_dtype(q, "q")
-    _check(q, "q", dt, 3)
-    stride = _check_caches(k_cache, v_cache, dt)
+    qstr = _check_rows(q, "q", dt)
+    cstr = _check_caches(k_cache, v_cache, dt)
     _check(block_tables, "block_tables", torch.int32, 2)
     _check(seq_lens, "seq_lens", torch.int32, 1)
     _check(query_start_loc, "query_start_loc", torch.int32, 1)
-    _check(out, "out", dt, 3)
+    ostr = _check_rows(out, "out", dt)
     t, hq, d = q.shape
     nb, bs, hkv, d_c = k_cache.shape
     if hkv != num_kv_heads or d_c != d:
@@ -262,29 +331,47 @@ def _varlen_ex(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc, num
     msl = mb * bs if max_seq_len is None else int(max_seq_len)
     if workspace is None:
         workspace = varlen_workspace(s, t, hq, hkv, d, device=q.device)
-    st = load().pa_attention_varlen_ex(
+    mods = _score_mods(softcap, alibi_slopes, mask, hq)
+    dense = qstr == (hq * d, d) and ostr == (hq * d, d) and _dense_rows(cstr, hkv, d)
+    if dense and mods is None:
+        st = load().pa_attention_varlen_ex(
+            q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(), mb,
+            seq_lens.data_ptr(), query_start_loc.data_ptr(), s, t, hq, hkv, d, bs, nb, cstr[0],
+            _DTYPES[dt], mql, msl, float(scale), int(bool(causal)), so_ptr, sp_ptr, n_spans,
+            out.data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+            _stream(stream))
+        _raise(st, what)
+        return out
+    strides = _Strides(*qstr, *ostr, *cstr)
+    st = load().pa_attention_varlen_mods(
         q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(), mb,
-        seq_lens.data_ptr(), query_start_loc.data_ptr(), s, t, hq, hkv, d, bs, nb, stride,
-        _DTYPES[dt], mql, msl, float(scale), int(bool(causal)), so_ptr, sp_ptr, n_spans,
+        seq_lens.data_ptr(), query_start_loc.data_ptr(), s, t, hq, hkv, d, bs, nb, _DTYPES[dt],
+        mql, msl, float(scale), int(bool(causal)), so_ptr, sp_ptr, n_spans,
+        ctypes.byref(strides), ctypes.byref(mods) if mods is not None else None,
         out.data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
         _stream(stream))
-    _raise(st, what)
+    _raise(st, "pa_attention_varlen_mods")
     return out
 
 
 def attention_varlen(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc,
                      num_kv_heads, scale, causal, out, max_query_len=None, max_seq_len=None,
-                     workspace=None, stream=None):
+                     workspace=None, stream=None, softcap=0.0, alibi_slopes=None, mask=None):
     """Paged varlen attention; writes out [T, Hq, D] (q's dtype).
 
     max_query_len / max_seq_len are host-side hints (the metadata builder's
     maxima); when omitted the safe bounds (all tokens / the block table's
     reach) are used, which never forces a device synchronisation.  The caches
-    may be separate tensors or the halves of one [NB, 2, BS, Hkv, D] cache.
+    may be separate tensors, the halves of one [NB, 2, BS, Hkv, D] cache, or
+    head-major [NB, Hkv, BS, D] caches passed as .permute(0, 2, 1, 3) views;
+    q and out may be head-major [Hq, T, D] tensors passed as
+    .transpose(0, 1) views.  Score modifiers: softcap (> 0: s <- c tanh(s/c)),
+    alibi_slopes (float32 [Hq]: s += slope_h (j - query position)), mask
+    (float32 [T, L] or [Hq, T, L]: s += mask[h, t, j]).
     """
     return _varlen_ex(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc,
                       num_kv_heads, scale, causal, None, None, out, max_query_len, max_seq_len,
-                      workspace, stream, "pa_attention_varlen_ex")
+                      workspace, stream, "pa_attention_varlen_ex", softcap, alibi_slopes, mask)
 
 
 def attention_varlen_spans(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc,

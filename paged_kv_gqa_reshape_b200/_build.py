@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpa.so")
 SOURCES = ["api.cu", "api_static.cu", "plan.cu", "scatter.cu", "smallseq.cu", "smallseq_bwd.cu", "decode.cu", "prefill_sm100.cu"]
-HEADERS = ["common.cuh", "kernels.h", "layout.h"]
+HEADERS = ["common.cuh", "kernels.h", "layout.h", "spans.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -29,18 +29,35 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    """Build libpa.so if any source is newer than it; returns its path."""
+    """Build libpa.so if any source is newer than it; returns its path.
+
+    Each source compiles to an object in its own nvcc process (in parallel),
+    then one nvcc call links the shared library."""
     if not force and not _stale():
         return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
-           "-Xcompiler", "-fPIC", "-shared", "-o", tmp]
+    import concurrent.futures
+    import tempfile
+    flags = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
+             "-Xcompiler", "-fPIC"]
     if ptxas_info:
-        cmd += ["-Xptxas", "-v"]
-    cmd += [os.path.join(CSRC, s) for s in SOURCES]
-    if verbose:
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.check_call(cmd, cwd=CSRC)
+        flags += ["-Xptxas", "-v"]
+    with tempfile.TemporaryDirectory(prefix="pa_build_") as tmpdir:
+        objs = [os.path.join(tmpdir, os.path.splitext(src)[0] + ".o") for src in SOURCES]
+
+        def compile_one(i):
+            cmd = [_nvcc(), *flags, "-c", os.path.join(CSRC, SOURCES[i]), "-o", objs[i]]
+            if verbose:
+                print(" ".join(cmd), file=sys.stderr)
+            subprocess.check_call(cmd, cwd=CSRC)
+
+        workers = max(1, min(len(SOURCES), os.cpu_count() or 1))
+        with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as pool:
+            list(pool.map(compile_one, range(len(SOURCES))))
+        tmp = LIB + ".tmp%d" % os.getpid()
+        cmd = [_nvcc(), *ARCH, "-shared", "-o", tmp, *objs]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        subprocess.check_call(cmd, cwd=CSRC)
     os.replace(tmp, LIB)
     return LIB
 

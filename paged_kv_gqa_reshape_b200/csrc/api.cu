@@ -87,6 +87,97 @@ bool make_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* di
   return r == CUDA_SUCCESS;
 }
 
+// Element strides of q, out and the caches after defaults and checks.
+struct Strides {
+  int64_t qt, qh, ot, oh;  // q / out: token, head
+  int64_t cb, cs, ch;      // cache: block, slot, head
+  bool q_hnd, kv_hnd;      // head-major q; head-major cache rows within a block
+};
+
+// A (token, head) pair for T tokens of H heads of D elements: (0, 0) is dense
+// NHD; otherwise token-major (head >= D, token >= H*head) or head-major
+// (token >= D, head >= T*token), every stride a positive multiple of 8.
+pa_status resolve_rows(int64_t tok, int64_t head, int64_t T, int64_t H, int64_t D, int64_t* rt,
+                       int64_t* rh, bool* hnd) {
+  if (tok == 0 && head == 0) {
+    *rt = H * D;
+    *rh = D;
+    *hnd = false;
+    return PA_OK;
+  }
+  if (tok <= 0 || head <= 0 || tok % 8 || head % 8) return PA_ERR_INVALID_ARG;
+  if (head >= D && tok >= H * head) {
+    *hnd = false;
+  } else if (tok >= D && head >= T * tok) {
+    *hnd = true;
+  } else {
+    return PA_ERR_UNSUPPORTED;
+  }
+  *rt = tok;
+  *rh = head;
+  return PA_OK;
+}
+
+// Cache strides: slot and head 0 mean dense [Hkv, D] rows per slot, with
+// block 0 meaning BS*Hkv*D; otherwise slot-major (head >= D, slot >=
+// Hkv*head) or head-major (slot >= D, head >= BS*slot) rows, and a block
+// stride covering one block's rows.
+pa_status resolve_cache(const pa_strides* st, int64_t BS, int64_t Hkv, int64_t D, Strides* r) {
+  int64_t cb = st ? st->cache_block : 0, cs = st ? st->cache_slot : 0,
+          ch = st ? st->cache_head : 0;
+  if (cs == 0 && ch == 0) {
+    cs = Hkv * D;
+    ch = D;
+    r->kv_hnd = false;
+    if (cb == 0) cb = BS * Hkv * D;
+  } else {
+    if (cs <= 0 || ch <= 0 || cs % 8 || ch % 8) return PA_ERR_INVALID_ARG;
+    if (ch >= D && cs >= Hkv * ch) {
+      r->kv_hnd = false;
+    } else if (cs >= D && ch >= BS * cs) {
+      r->kv_hnd = true;
+    } else {
+      return PA_ERR_UNSUPPORTED;
+    }
+  }
+  const int64_t extent = r->kv_hnd ? Hkv * ch : BS * cs;
+  if (cb < extent || cb % 8) return PA_ERR_INVALID_ARG;
+  r->cb = cb;
+  r->cs = cs;
+  r->ch = ch;
+  return PA_OK;
+}
+
+pa_status resolve_strides(const pa_strides* st, int64_t T, int64_t Hq, int64_t Hkv, int64_t D,
+                          int64_t BS, Strides* r) {
+  bool o_hnd = false;
+  pa_status e = resolve_rows(st ? st->q_token : 0, st ? st->q_head : 0, T, Hq, D, &r->qt, &r->qh,
+                             &r->q_hnd);
+  if (e != PA_OK) return e;
+  e = resolve_rows(st ? st->out_token : 0, st ? st->out_head : 0, T, Hq, D, &r->ot, &r->oh, &o_hnd);
+  if (e != PA_OK) return e;
+  return resolve_cache(st, BS, Hkv, D, r);
+}
+
+// Score modifiers after checks (mods NULL or all off: none).
+pa_status resolve_mods(const pa_score_mods* m, pa::ScoreMods* r) {
+  *r = pa::ScoreMods{};
+  if (!m) return PA_OK;
+  if (!(m->softcap >= 0.f) || !isfinite(m->softcap)) return PA_ERR_INVALID_ARG;
+  if (m->alibi_slopes && (reinterpret_cast<uintptr_t>(m->alibi_slopes) & 3u))
+    return PA_ERR_INVALID_ARG;
+  if (m->mask && (!aligned16(m->mask) || m->mask_head_stride < 0 || m->mask_token_stride < 0 ||
+                  m->mask_head_stride % 4 || m->mask_token_stride % 4 || m->mask_len <= 0))
+    return PA_ERR_INVALID_ARG;
+  r->softcap = m->softcap;
+  r->alibi = m->alibi_slopes;
+  r->mask = m->mask;
+  r->mask_head = m->mask ? m->mask_head_stride : 0;
+  r->mask_tok = m->mask ? m->mask_token_stride : 0;
+  r->mask_len = m->mask ? m->mask_len : 0;
+  return PA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -117,13 +208,29 @@ pa_status pa_write_kv_ex(const void* k, const void* v, const int64_t* slot_mappi
                          int64_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
                          void* k_cache, void* v_cache, int64_t num_blocks, int32_t block_size,
                          int64_t block_stride, int32_t dtype, void* workspace, void* stream) {
+  if (block_stride < 0) return PA_ERR_INVALID_ARG;
+  pa_strides st{};
+  st.cache_block = block_stride;
+  return pa_write_kv_strided(k, v, slot_mapping, num_tokens, num_kv_heads, head_dim, k_cache,
+                             v_cache, num_blocks, block_size, &st, dtype, workspace, stream);
+}
+
+pa_status pa_write_kv_strided(const void* k, const void* v, const int64_t* slot_mapping,
+                              int64_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                              void* k_cache, void* v_cache, int64_t num_blocks,
+                              int32_t block_size, const pa_strides* strides, int32_t dtype,
+                              void* workspace, void* stream) {
   if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || head_dim % 8 != 0 ||
       num_blocks <= 0 || block_size <= 0)
     return PA_ERR_INVALID_ARG;
   if (dtype != PA_DTYPE_BF16 && dtype != PA_DTYPE_FP16) return PA_ERR_INVALID_ARG;
-  const int64_t block_elems = (int64_t)block_size * num_kv_heads * head_dim;
-  if (block_stride == 0) block_stride = block_elems;
-  if (block_stride < block_elems || block_stride % 8 != 0) return PA_ERR_INVALID_ARG;
+  Strides sd{};
+  pa_status rs = resolve_cache(strides, block_size, num_kv_heads, head_dim, &sd);
+  if (rs != PA_OK) return rs;
+  int dshift = 0;
+  while ((1 << dshift) < head_dim / 8) ++dshift;
+  const bool dense = sd.cs == (int64_t)num_kv_heads * head_dim && sd.ch == head_dim;
+  if (!dense && (1 << dshift) != head_dim / 8) return PA_ERR_UNSUPPORTED;
   if (num_tokens == 0) return PA_OK;
   if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PA_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
@@ -132,8 +239,8 @@ pa_status pa_write_kv_ex(const void* k, const void* v, const int64_t* slot_mappi
   const int row_vecs = num_kv_heads * head_dim / 8;
   uint32_t* err = workspace ? static_cast<uint32_t*>(workspace) : nullptr;
   cudaError_t e = pa::launch_write_kv(k, v, slot_mapping, num_tokens, row_vecs, k_cache, v_cache,
-                                      num_blocks * (int64_t)block_size, block_size,
-                                      block_stride / 8, err, sm_count(),
+                                      num_blocks * (int64_t)block_size, block_size, sd.cb / 8,
+                                      sd.cs / 8, sd.ch / 8, dshift, err, sm_count(),
                                       static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
@@ -154,10 +261,11 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
                                 const int32_t* seq_lens, const int32_t* query_start_loc,
                                 int32_t num_seqs, int64_t num_q_tokens, int32_t num_q_heads,
                                 int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
-                                int64_t num_blocks, int64_t block_stride, int32_t dtype,
+                                int64_t num_blocks, const pa_strides* strides, int32_t dtype,
                                 int32_t max_query_len, int32_t max_seq_len,
                                 float scale, int32_t causal, const int32_t* span_offsets,
-                                const int32_t* spans, int32_t num_spans, void* out,
+                                const int32_t* spans, int32_t num_spans,
+                                const pa_score_mods* score_mods, void* out,
                                 void* workspace, size_t workspace_bytes, void* stream) {
   // ---- host-visible checks (nothing launched yet) ----
   if (dtype != PA_DTYPE_BF16 && dtype != PA_DTYPE_FP16) return PA_ERR_INVALID_ARG;
@@ -184,9 +292,13 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
       (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
       (reinterpret_cast<uintptr_t>(query_start_loc) & 3u))
     return PA_ERR_INVALID_ARG;
-  const int64_t block_elems = (int64_t)block_size * num_kv_heads * head_dim;
-  if (block_stride == 0) block_stride = block_elems;
-  if (block_stride < block_elems || block_stride % 8 != 0) return PA_ERR_INVALID_ARG;
+  Strides sd{};
+  pa_status rs = resolve_strides(strides, num_q_tokens, num_q_heads, num_kv_heads, head_dim,
+                                 block_size, &sd);
+  if (rs != PA_OK) return rs;
+  pa::ScoreMods mods{};
+  rs = resolve_mods(score_mods, &mods);
+  if (rs != PA_OK) return rs;
   const WorkspaceLayout L =
       pa::make_layout(num_seqs, num_q_tokens, num_q_heads, num_kv_heads, head_dim);
   if (workspace_bytes < L.total) return PA_ERR_INVALID_ARG;
@@ -199,15 +311,25 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
 
   CUtensorMap q_map, k_map, v_map;
   if (run_prefill) {
-    const cuuint32_t box_q[3] = {64, 1, (cuuint32_t)pa::kPrefillTileM};
-    const cuuint64_t dq[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_q_heads,
-                              (cuuint64_t)num_q_tokens};
-    const cuuint64_t sq[2] = {(cuuint64_t)head_dim * 2, (cuuint64_t)num_q_heads * head_dim * 2};
-    const cuuint32_t box_kv[4] = {64, 1, (cuuint32_t)pa::kPageKeys, 1};
-    const cuuint64_t dkv[4] = {(cuuint64_t)head_dim, (cuuint64_t)num_kv_heads,
-                               (cuuint64_t)block_size, (cuuint64_t)num_blocks};
-    const cuuint64_t skv[3] = {(cuuint64_t)head_dim * 2, (cuuint64_t)num_kv_heads * head_dim * 2,
-                               (cuuint64_t)block_stride * 2};
+    // dimensions ordered by increasing stride: (D, head, token) for a
+    // token-major q, (D, token, head) for a head-major one; the kernel
+    // swaps its coordinates to match (likewise slot and head of the cache)
+    const cuuint32_t box_q[3] = {64, sd.q_hnd ? (cuuint32_t)pa::kPrefillTileM : 1u,
+                                 sd.q_hnd ? 1u : (cuuint32_t)pa::kPrefillTileM};
+    const cuuint64_t dq[3] = {(cuuint64_t)head_dim,
+                              (cuuint64_t)(sd.q_hnd ? num_q_tokens : num_q_heads),
+                              (cuuint64_t)(sd.q_hnd ? num_q_heads : num_q_tokens)};
+    const cuuint64_t sq[2] = {(cuuint64_t)(sd.q_hnd ? sd.qt : sd.qh) * 2,
+                              (cuuint64_t)(sd.q_hnd ? sd.qh : sd.qt) * 2};
+    const cuuint32_t box_kv[4] = {64, sd.kv_hnd ? (cuuint32_t)pa::kPageKeys : 1u,
+                                  sd.kv_hnd ? 1u : (cuuint32_t)pa::kPageKeys, 1};
+    const cuuint64_t dkv[4] = {(cuuint64_t)head_dim,
+                               (cuuint64_t)(sd.kv_hnd ? block_size : num_kv_heads),
+                               (cuuint64_t)(sd.kv_hnd ? num_kv_heads : block_size),
+                               (cuuint64_t)num_blocks};
+    const cuuint64_t skv[3] = {(cuuint64_t)(sd.kv_hnd ? sd.cs : sd.ch) * 2,
+                               (cuuint64_t)(sd.kv_hnd ? sd.ch : sd.cs) * 2,
+                               (cuuint64_t)sd.cb * 2};
     if (!make_map(&q_map, q, 3, dq, sq, box_q, fp16) ||
         !make_map(&k_map, k_cache, 4, dkv, skv, box_kv, fp16) ||
         !make_map(&v_map, v_cache, 4, dkv, skv, box_kv, fp16))
@@ -240,6 +362,12 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
     pp.span_offsets = span_offsets;
     pp.spans = spans;
     pp.num_spans = num_spans;
+    pp.q_hnd = sd.q_hnd ? 1 : 0;
+    pp.kv_hnd = sd.kv_hnd ? 1 : 0;
+    pp.o_tok = sd.ot;
+    pp.o_head = sd.oh;
+    pp.scale = scale;
+    pp.mods = mods;
     pp.out = static_cast<uint16_t*>(out);
     pp.ws = ws;
     pp.L = L;
@@ -264,7 +392,15 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
   dp.num_kv_heads = num_kv_heads;
   dp.group = group;
   dp.num_blocks = num_blocks;
-  dp.block_stride = block_stride;
+  dp.block_stride = sd.cb;
+  dp.c_slot = sd.cs;
+  dp.c_head = sd.ch;
+  dp.q_tok = sd.qt;
+  dp.q_head = sd.qh;
+  dp.o_tok = sd.ot;
+  dp.o_head = sd.oh;
+  dp.scale = scale;
+  dp.mods = mods;
   dp.scale_log2 = scale_log2;
   dp.out = static_cast<uint16_t*>(out);
   dp.ws = ws;
@@ -288,9 +424,9 @@ pa_status pa_attention_varlen(const void* q, const void* k_cache, const void* v_
                               size_t workspace_bytes, void* stream) {
   return attention_varlen_impl(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
                                query_start_loc, num_seqs, num_q_tokens, num_q_heads, num_kv_heads,
-                               head_dim, block_size, num_blocks, 0, PA_DTYPE_BF16, max_query_len,
-                               max_seq_len, scale, causal, nullptr, nullptr, 0, out, workspace,
-                               workspace_bytes, stream);
+                               head_dim, block_size, num_blocks, nullptr, PA_DTYPE_BF16,
+                               max_query_len, max_seq_len, scale, causal, nullptr, nullptr, 0,
+                               nullptr, out, workspace, workspace_bytes, stream);
 }
 
 pa_status pa_attention_varlen_spans(const void* q, const void* k_cache, const void* v_cache,
@@ -305,9 +441,9 @@ pa_status pa_attention_varlen_spans(const void* q, const void* k_cache, const vo
   if (!span_offsets && num_seqs > 0) return PA_ERR_INVALID_ARG;
   return attention_varlen_impl(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
                                query_start_loc, num_seqs, num_q_tokens, num_q_heads, num_kv_heads,
-                               head_dim, block_size, num_blocks, 0, PA_DTYPE_BF16, max_query_len,
-                               max_seq_len, scale, 1, span_offsets, spans, num_spans, out, workspace,
-                               workspace_bytes, stream);
+                               head_dim, block_size, num_blocks, nullptr, PA_DTYPE_BF16,
+                               max_query_len, max_seq_len, scale, 1, span_offsets, spans,
+                               num_spans, nullptr, out, workspace, workspace_bytes, stream);
 }
 
 pa_status pa_attention_varlen_ex(const void* q, const void* k_cache, const void* v_cache,
@@ -320,11 +456,32 @@ pa_status pa_attention_varlen_ex(const void* q, const void* k_cache, const void*
                                  int32_t causal, const int32_t* span_offsets, const int32_t* spans,
                                  int32_t num_spans, void* out, void* workspace,
                                  size_t workspace_bytes, void* stream) {
+  if (block_stride < 0) return PA_ERR_INVALID_ARG;
+  pa_strides st{};
+  st.cache_block = block_stride;
   return attention_varlen_impl(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
                                query_start_loc, num_seqs, num_q_tokens, num_q_heads, num_kv_heads,
-                               head_dim, block_size, num_blocks, block_stride, dtype, max_query_len,
+                               head_dim, block_size, num_blocks, &st, dtype, max_query_len,
                                max_seq_len, scale, span_offsets ? 1 : causal, span_offsets, spans,
-                               num_spans, out, workspace, workspace_bytes, stream);
+                               num_spans, nullptr, out, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_attention_varlen_mods(const void* q, const void* k_cache, const void* v_cache,
+                                   const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                   const int32_t* seq_lens, const int32_t* query_start_loc,
+                                   int32_t num_seqs, int64_t num_q_tokens, int32_t num_q_heads,
+                                   int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                   int64_t num_blocks, int32_t dtype, int32_t max_query_len,
+                                   int32_t max_seq_len, float scale, int32_t causal,
+                                   const int32_t* span_offsets, const int32_t* spans,
+                                   int32_t num_spans, const pa_strides* strides,
+                                   const pa_score_mods* mods, void* out, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  return attention_varlen_impl(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                               query_start_loc, num_seqs, num_q_tokens, num_q_heads, num_kv_heads,
+                               head_dim, block_size, num_blocks, strides, dtype, max_query_len,
+                               max_seq_len, scale, span_offsets ? 1 : causal, span_offsets, spans,
+                               num_spans, mods, out, workspace, workspace_bytes, stream);
 }
 
 pa_status pa_attention_smallseq(const void* q, const void* k, const void* v,

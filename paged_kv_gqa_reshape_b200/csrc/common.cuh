@@ -76,6 +76,17 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // ---------------------------------------------------------------------------
 // packed fp32 pairs (one instruction on two lanes of a 64-bit register pair)
 // ---------------------------------------------------------------------------
+constexpr float kLog2e = 1.4426950408889634f;
+
+// tanh(x) from the identity tanh x = 1 - 2 / (e^{2x} + 1), with e^{2x} from
+// the SFU exponential (2^(2 x log2 e)).  |x| is clamped to 20, where tanh is
+// +-1 in fp32, so the exponential stays finite; absolute error ~1e-7.
+__device__ __forceinline__ float tanh_sfu(float x) {
+  x = fminf(fmaxf(x, -20.f), 20.f);
+  const float e = fast_exp2(x * (2.f * kLog2e));
+  return 1.f - __fdividef(2.f, e + 1.f);
+}
+
 // Packed 16-bit multiply of two element pairs, round to nearest even.
 template <bool H>
 __device__ __forceinline__ uint32_t emul2(uint32_t a, uint32_t b) {

@@ -68,7 +68,7 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
 
 }  // namespace
 
-template <int D, int HPC, int NSTAGE, int NGT, bool H>
+template <int D, int HPC, int NSTAGE, int NGT, bool H, bool MODS>
 __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams p) {
   using Shape = DecodeShape<D, HPC, NSTAGE>;
   constexpr int CH = Shape::kChunks;
@@ -170,8 +170,9 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
   // single-query sequences with no key: zero output rows (spread over the ranges)
   for (long long s = c; s < S; s += G) {
     if (is_decode((int)s) && seq_kv((int)s) == 0) {
-      uint16_t* o0 = p.out + ((size_t)seq_q((int)s) * p.num_q_heads + head0) * D;
-      for (int i = lane; i < g * D; i += 32) o0[i] = 0;  // +0 in both element types
+      uint16_t* o0 = p.out + (size_t)seq_q((int)s) * p.o_tok + (size_t)head0 * p.o_head;
+      for (int i = lane; i < g * D; i += 32)
+        o0[(size_t)(i / D) * p.o_head + i % D] = 0;  // +0 in both element types
     }
   }
   if (P == 0) return;
@@ -198,7 +199,6 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
   if (b0 >= b1) return;
 
   // ---------------- producer: pages [x_p, b1) in order ----------------------
-  const size_t row_stride = (size_t)Hkv * D;
   long long x_p = b0;
   int seq_p = seq_of(b0);
   long long p_first = pfx(seq_p), p_end = pfx(seq_p + 1);
@@ -211,7 +211,8 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
         p.block_tables[(size_t)seq_p * p.max_blocks_per_seq + (x_p - p_first)];
     const bool block_ok = block >= 0 && block < p.num_blocks;
     if (!block_ok && tid == 0) raise_error(err, PA_DEVERR_BLOCK);
-    const size_t base = (size_t)(block_ok ? block : 0) * p.block_stride + (size_t)hg * HPC * D;
+    const size_t base =
+        (size_t)(block_ok ? block : 0) * p.block_stride + (size_t)hg * HPC * p.c_head;
     __nv_bfloat16* kdst = ring + (size_t)stage * 2 * Shape::kTensorStage;
     __nv_bfloat16* vdst = kdst + Shape::kTensorStage;
 #pragma unroll
@@ -221,7 +222,7 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
       const int rem = ci - r * (HPC * CH);
       const int h = rem / CH, cc = rem - h * CH;
       const bool ok = block_ok && (key0 + r < p_kv);
-      const size_t src = base + (size_t)r * row_stride + h * D + cc * 8;
+      const size_t src = base + (size_t)r * p.c_slot + (size_t)h * p.c_head + cc * 8;
       const int dst = (h * kPageKeys + r) * D + ((cc ^ (r & 7)) * 8);
       cp_async_16(smem_u32(kdst + dst), p.k_cache + (ok ? src : 0), ok);
       cp_async_16(smem_u32(vdst + dst), p.v_cache + (ok ? src : 0), ok);
@@ -262,7 +263,7 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
     for (int nt = 0; nt < NGT; ++nt) {
       const int hl = nt * 8 + gq;
       const bool hv = hl < g;
-      const size_t row = ((size_t)seg_q * p.num_q_heads + head0 + (hv ? hl : 0)) * D;
+      const size_t row = (size_t)seg_q * p.q_tok + (size_t)(head0 + (hv ? hl : 0)) * p.q_head;
 #pragma unroll
       for (int ks = 0; ks < KSTEPS; ++ks) {
         qb[nt][ks][0] = hv ? q32[(row + ks * 16 + 2 * tq) / 2] : 0u;
@@ -309,10 +310,37 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
       uint32_t pb[NGT][2];
 #pragma unroll
       for (int nt = 0; nt < NGT; ++nt) {
-        float s0 = ok0 ? sc[nt][0] * p.scale_log2 : -INFINITY;
-        float s1 = ok0 ? sc[nt][1] * p.scale_log2 : -INFINITY;
-        float s2 = ok1 ? sc[nt][2] * p.scale_log2 : -INFINITY;
-        float s3 = ok1 ? sc[nt][3] * p.scale_log2 : -INFINITY;
+        float s0, s1, s2, s3;
+        if constexpr (MODS) {
+          // soft-cap, ALiBi, additive mask on scale * s (then log2 units);
+          // the query sits at key position seg_kv - 1
+          const int hl0 = nt * 8 + 2 * tq;
+          auto mod = [&](float raw, int hl, int key) {
+            float t = raw * p.scale;
+            if (p.mods.softcap > 0.f) t = p.mods.softcap * tanh_sfu(t * (1.f / p.mods.softcap));
+            if (hl < g) {
+              const int h = head0 + hl;
+              if (p.mods.alibi) t = fmaf(__ldg(p.mods.alibi + h), (float)(key - (seg_kv - 1)), t);
+              if (p.mods.mask) {
+                if (key < p.mods.mask_len)
+                  t += __ldg(p.mods.mask + (size_t)h * p.mods.mask_head +
+                             (size_t)seg_q * p.mods.mask_tok + key);
+                else
+                  raise_error(err, PA_DEVERR_HINT);
+              }
+            }
+            return t * kLog2e;
+          };
+          s0 = ok0 ? mod(sc[nt][0], hl0, key0 + gq) : -INFINITY;
+          s1 = ok0 ? mod(sc[nt][1], hl0 + 1, key0 + gq) : -INFINITY;
+          s2 = ok1 ? mod(sc[nt][2], hl0, key0 + gq + 8) : -INFINITY;
+          s3 = ok1 ? mod(sc[nt][3], hl0 + 1, key0 + gq + 8) : -INFINITY;
+        } else {
+          s0 = ok0 ? sc[nt][0] * p.scale_log2 : -INFINITY;
+          s1 = ok0 ? sc[nt][1] * p.scale_log2 : -INFINITY;
+          s2 = ok1 ? sc[nt][2] * p.scale_log2 : -INFINITY;
+          s3 = ok1 ? sc[nt][3] * p.scale_log2 : -INFINITY;
+        }
         float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
 #pragma unroll
         for (int o2 = 4; o2 < 32; o2 <<= 1) {
@@ -372,7 +400,7 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
           const int hl = nt * 8 + 2 * tq + j;
           if (hl < g) {
             const float inv = l[nt][j] > 0.f ? 1.f / l[nt][j] : 0.f;
-            uint16_t* orow = p.out + ((size_t)seg_q * p.num_q_heads + head0 + hl) * D;
+            uint16_t* orow = p.out + (size_t)seg_q * p.o_tok + (size_t)(head0 + hl) * p.o_head;
 #pragma unroll
             for (int mt = 0; mt < KSTEPS; ++mt) {
               orow[mt * 16 + gq] = ebits<H>(o[nt][mt][j] * inv);
@@ -455,8 +483,8 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
                   uint2 v;
                   v.x = epack<H>(acc.x * inv, acc.y * inv);
                   v.y = epack<H>(acc.z * inv, acc.w * inv);
-                  *reinterpret_cast<uint2*>(
-                      p.out + ((size_t)seg_q * p.num_q_heads + head0 + i / n_chunks) * D + lane * 4) = v;
+                  *reinterpret_cast<uint2*>(p.out + (size_t)seg_q * p.o_tok +
+                                            (size_t)(head0 + i / n_chunks) * p.o_head + lane * 4) = v;
                 }
                 acc = make_float4(0.f, 0.f, 0.f, 0.f);
               }
@@ -521,7 +549,8 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
             uint2 v;
             v.x = epack<H>(acc.x * inv, acc.y * inv);
             v.y = epack<H>(acc.z * inv, acc.w * inv);
-            *reinterpret_cast<uint2*>(p.out + ((size_t)seg_q * p.num_q_heads + head) * D + lane * 4) = v;
+            *reinterpret_cast<uint2*>(p.out + (size_t)seg_q * p.o_tok + (size_t)head * p.o_head +
+                                      lane * 4) = v;
           }
         }
         }
@@ -549,10 +578,10 @@ int heads_per_cta(int num_kv_heads) {
   return 1;
 }
 
-template <int D, int HPC, int NSTAGE, int NGT, bool H>
+template <int D, int HPC, int NSTAGE, int NGT, bool H, bool MODS>
 cudaError_t launch_t(const DecodeParams& p, int num_sms, cudaStream_t stream) {
   using Shape = DecodeShape<D, HPC, NSTAGE>;
-  auto kernel = decode_kernel<D, HPC, NSTAGE, NGT, H>;
+  auto kernel = decode_kernel<D, HPC, NSTAGE, NGT, H, MODS>;
   const int smem = Shape::smem_bytes(p.self_plan != 0);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -571,34 +600,37 @@ cudaError_t launch_t(const DecodeParams& p, int num_sms, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-template <int D, int NSTAGE, int NGT, bool H>
+template <int D, int NSTAGE, int NGT, bool H, bool MODS>
 cudaError_t launch_hpc(const DecodeParams& p, int hpc, int num_sms, cudaStream_t stream) {
   switch (hpc) {
-    case 8: return launch_t<D, 8, NSTAGE, NGT, H>(p, num_sms, stream);
-    case 4: return launch_t<D, 4, NSTAGE, NGT, H>(p, num_sms, stream);
-    case 2: return launch_t<D, 2, NSTAGE, NGT, H>(p, num_sms, stream);
-    default: return launch_t<D, 1, NSTAGE, NGT, H>(p, num_sms, stream);
+    case 8: return launch_t<D, 8, NSTAGE, NGT, H, MODS>(p, num_sms, stream);
+    case 4: return launch_t<D, 4, NSTAGE, NGT, H, MODS>(p, num_sms, stream);
+    case 2: return launch_t<D, 2, NSTAGE, NGT, H, MODS>(p, num_sms, stream);
+    default: return launch_t<D, 1, NSTAGE, NGT, H, MODS>(p, num_sms, stream);
   }
 }
 
-template <bool H>
+template <bool H, bool MODS>
 cudaError_t launch_decode_t(const DecodeParams& p, int head_dim, int num_sms,
                             cudaStream_t stream) {
   const int hpc = heads_per_cta(p.num_kv_heads);
   if (head_dim == 128) {
-    if (p.group <= 8) return launch_hpc<128, 3, 1, H>(p, hpc, num_sms, stream);
-    return launch_hpc<128, 3, 2, H>(p, hpc, num_sms, stream);
+    if (p.group <= 8) return launch_hpc<128, 3, 1, H, MODS>(p, hpc, num_sms, stream);
+    return launch_hpc<128, 3, 2, H, MODS>(p, hpc, num_sms, stream);
   }
-  if (p.group <= 8) return launch_hpc<64, 6, 1, H>(p, hpc, num_sms, stream);
-  return launch_hpc<64, 6, 2, H>(p, hpc, num_sms, stream);
+  if (p.group <= 8) return launch_hpc<64, 6, 1, H, MODS>(p, hpc, num_sms, stream);
+  return launch_hpc<64, 6, 2, H, MODS>(p, hpc, num_sms, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const DecodeParams& p, int head_dim, bool fp16, int num_sms,
                           cudaStream_t stream) {
-  return fp16 ? launch_decode_t<true>(p, head_dim, num_sms, stream)
-              : launch_decode_t<false>(p, head_dim, num_sms, stream);
+  if (p.mods.any())
+    return fp16 ? launch_decode_t<true, true>(p, head_dim, num_sms, stream)
+                : launch_decode_t<false, true>(p, head_dim, num_sms, stream);
+  return fp16 ? launch_decode_t<true, false>(p, head_dim, num_sms, stream)
+              : launch_decode_t<false, false>(p, head_dim, num_sms, stream);
 }
 
 }  // namespace pa

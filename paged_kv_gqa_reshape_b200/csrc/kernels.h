@@ -11,9 +11,13 @@
 namespace pa {
 
 // ---- KV scatter ------------------------------------------------------------
+// Cache destination of vector c of head h of slot s: (s / block_size) *
+// block_vecs + (s % block_size) * slot_vecs + h * head_vecs + c (16-byte
+// vectors; a head row holds 1 << dshift of them).
 cudaError_t launch_write_kv(const void* k, const void* v, const int64_t* slot_mapping,
                             int64_t num_tokens, int row_vecs, void* k_cache, void* v_cache,
-                            int64_t num_slots, int block_size, int64_t block_vecs, uint32_t* err,
+                            int64_t num_slots, int block_size, int64_t block_vecs,
+                            int64_t slot_vecs, int64_t head_vecs, int dshift, uint32_t* err,
                             int num_sms, cudaStream_t stream);
 
 // ---- plan ------------------------------------------------------------------
@@ -24,6 +28,16 @@ void launch_plan(const int32_t* query_start_loc, const int32_t* seq_lens, int nu
                  unsigned char* ws, const WorkspaceLayout& L, cudaStream_t stream);
 
 // ---- split-KV decode -------------------------------------------------------
+// Score modifiers of a varlen call (soft-cap, ALiBi, additive mask), as the
+// C ABI's pa_score_mods; kernels take a template flag when any is on.
+struct ScoreMods {
+  float softcap;        // > 0: s <- softcap * tanh(s / softcap)
+  const float* alibi;   // [Hq] slopes or null
+  const float* mask;    // additive fp32 mask or null
+  long long mask_head, mask_tok, mask_len;
+  bool any() const { return softcap > 0.f || alibi != nullptr || mask != nullptr; }
+};
+
 struct DecodeParams {
   const __nv_bfloat16* q;
   const __nv_bfloat16* k_cache;
@@ -41,6 +55,11 @@ struct DecodeParams {
   int group;  // num_q_heads / num_kv_heads, <= 16
   long long num_blocks;
   long long block_stride;  // elements between consecutive cache blocks
+  long long c_slot, c_head;  // elements between slots of a block / KV heads of a slot
+  long long q_tok, q_head;   // q strides (elements)
+  long long o_tok, o_head;   // out strides (elements)
+  float scale;       // softmax scale (used with modifiers)
+  ScoreMods mods;
   float scale_log2;  // scale * log2(e)
   int self_plan;     // 1: every CTA plans the decode work itself (num_seqs <= kSelfPlanMaxSeqs)
   uint16_t* out;     // elements of the kernel's type (bf16 or fp16)
@@ -65,7 +84,12 @@ struct PrefillParams {
   const int32_t* span_offsets;  // full-attention spans (null: none)
   const int32_t* spans;
   int num_spans;
-  uint16_t* out;  // [T, Hq, D] elements of the kernel's type (bf16 or fp16)
+  int q_hnd;    // the q map's dims are (D, T, Hq) instead of (D, Hq, T)
+  int kv_hnd;   // the cache maps' dims are (D, BS, Hkv, blocks) instead of (D, Hkv, BS, blocks)
+  long long o_tok, o_head;  // out strides (elements)
+  float scale;
+  ScoreMods mods;
+  uint16_t* out;  // elements of the kernel's type (bf16 or fp16)
   unsigned char* ws;
   WorkspaceLayout L;
 };

@@ -104,7 +104,14 @@ __device__ __forceinline__ Work decode_work(int w, const int2* tiles, const int2
 
 }  // namespace
 
-template <int D, bool H>
+// Element offset of out row (token t, head h): dense [T, Hq, D] unless STRIDED.
+template <int D, bool STRIDED>
+__device__ __forceinline__ size_t out_offset(const PrefillParams& p, int t, int h) {
+  if constexpr (STRIDED) return (size_t)t * p.o_tok + (size_t)h * p.o_head;
+  return ((size_t)t * p.num_q_heads + h) * D;
+}
+
+template <int D, bool H, bool MODS, bool STRIDED>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(PrefillParams p, const __grid_constant__ CUtensorMap q_map,
                    const __grid_constant__ CUtensorMap k_map,
@@ -178,10 +185,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       long long ld = 0;  // K/V tiles loaded so far (slot = ld % kRing)
       int tcount = 0;
       bool ok = true;
+      // head-major q / cache swap two tensor-map coordinates (strided
+      // instantiation only; the dense one keeps token-major order)
+      const bool q_hnd = STRIDED && p.q_hnd != 0, kv_hnd = STRIDED && p.kv_hnd != 0;
       for (int w = blockIdx.x; w < num_work && ok; w += gridDim.x) {
         const Work wk = decode_work(w, tiles, tile_n, info, p.num_q_heads);
         if (wk.nmax == 0) continue;
         const int kvh = wk.head / p.group;
+        const int kv_c1 = kv_hnd ? 0 : kvh, kv_c2 = kv_hnd ? kvh : 0;  // (head, slot) or (slot, head)
         if (tcount > 0) ok = mbar_wait_bounded(q_empty, (tcount - 1) & 1, abort_flag, err);
         if (!ok) break;
         mbar_arrive_expect_tx(q_full, 2 * SM::kQBytes);
@@ -189,8 +200,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int x = 0; x < 2; ++x)
 #pragma unroll
           for (int dh = 0; dh < D / 64; ++dh)
-            tma_load_3d(q_s + x * SM::kQBytes + dh * (BM * 128), &q_map, q_full, dh * 64, wk.head,
-                        wk.q_start + wk.row0 + x * BM);
+            tma_load_3d(q_s + x * SM::kQBytes + dh * (BM * 128), &q_map, q_full, dh * 64,
+                        q_hnd ? wk.q_start + wk.row0 + x * BM : wk.head,
+                        q_hnd ? wk.head : wk.q_start + wk.row0 + x * BM);
         const int32_t* table = p.block_tables + (size_t)wk.seq * p.max_blocks_per_seq;
         for (int j = 0; j < wk.nmax && ok; ++j) {
           int blk[BN / kPageKeys];
@@ -220,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int dh = 0; dh < D / 64; ++dh)
                 tma_load_4d(ring_s + st * SM::kKVBytes + dh * (BN * 128) + pg * (kPageKeys * 128),
-                            map, slot_full + st, dh * 64, kvh, 0, blk[pg]);
+                            map, slot_full + st, dh * 64, kv_c1, kv_c2, blk[pg]);
           }
         }
         ++tcount;
@@ -321,8 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool row_ok = r < rows;
       if (n == 0) {
         if (row_ok) {
-          uint16_t* orow =
-              p.out + ((size_t)(wk.q_start + qrow) * p.num_q_heads + wk.head) * D;
+          uint16_t* orow = p.out + out_offset<D, STRIDED>(p, wk.q_start + qrow, wk.head);
 #pragma unroll
           for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = make_uint4(0, 0, 0, 0);
         }
@@ -336,6 +347,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         limit = span_visible(sl, pos, pos, nullptr) - 1;
       } else if (p.causal) {
         limit = min(limit, pos);
+      }
+      // score modifiers of this row (head wk.head, query token q_start + qrow)
+      float slope = 0.f;
+      const float* mrow = nullptr;
+      if constexpr (MODS) {
+        if (p.mods.alibi) slope = __ldg(p.mods.alibi + wk.head);
+        if (p.mods.mask && row_ok)
+          mrow = p.mods.mask + (size_t)wk.head * p.mods.mask_head +
+                 (size_t)(wk.q_start + qrow) * p.mods.mask_tok;
       }
       float m_use = -INFINITY, l = 0.f;
       for (int j = 0; j < n; ++j) {
@@ -361,6 +381,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < BN; c += 32)
           tmem_ld32(s_col + c, *reinterpret_cast<uint32_t(*)[32]>(&sv[c]));
         tmem_ld_wait();
+        if constexpr (MODS) {
+          // soft-cap, ALiBi and the additive mask on scale * s, to log2 units;
+          // keys past `valid` get -inf below, so their mask values are not read
+          const int vis = masked_tile ? max(0, min(valid, BN)) : BN;
+          int mlim = 0;  // keys of this tile with a mask value
+          if (mrow) {
+            const long long left = p.mods.mask_len - key0;
+            mlim = (int)max(0ll, min((long long)vis, left));
+            if (mlim < vis) raise_error(err, PA_DEVERR_HINT);
+          }
+          const float cap = p.mods.softcap, inv_cap = cap > 0.f ? 1.f / cap : 0.f;
+          const float rel0 = (float)(key0 - pos);
+#pragma unroll
+          for (int c = 0; c < BN; c += 4) {
+            float4 mv = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (mrow) {
+              if (c + 4 <= mlim) {
+                mv = __ldg(reinterpret_cast<const float4*>(mrow + key0 + c));
+              } else if (c < mlim) {
+                mv.x = __ldg(mrow + key0 + c);
+                if (c + 1 < mlim) mv.y = __ldg(mrow + key0 + c + 1);
+                if (c + 2 < mlim) mv.z = __ldg(mrow + key0 + c + 2);
+              }
+            }
+            const float m4[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float t = __uint_as_float(sv[c + e]) * p.scale;
+              if (cap > 0.f) t = cap * tanh_sfu(t * inv_cap);
+              t = fmaf(slope, rel0 + (float)(c + e), t) + m4[e];
+              sv[c + e] = __float_as_uint(t * kLog2e);
+            }
+          }
+        }
         // Tiles crossing the diagonal or the sequence end set hidden keys to
         // -inf once; the others skip every per-key test.
         if (masked_tile) {
@@ -379,7 +433,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int wdt = NP / 2; wdt >= 1; wdt >>= 1)
 #pragma unroll
           for (int i = 0; i < wdt; ++i) mp[i] = fmaxf(mp[i], mp[i + wdt]);
-        const float m_tile = mp[0] * p.scale_log2;  // scale_log2 > 0: max commutes with it
+        // with MODS the scores are already in log2 units; else the scale
+        // (> 0, so the max commutes with it) is applied here
+        const float m_tile = mp[0] * (MODS ? 1.f : p.scale_log2);
         const float m_old = m_use;
         const bool grow =
             m_tile > m_old + kRescaleThreshold || (m_old == -INFINITY && m_tile > -INFINITY);
@@ -390,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // p = 2^(scale_log2 * s - base), rounded to bf16 and written to TMEM as
         // the A operand of O += P.V.  Scaling and row sums run on packed fp32
         // pairs; the exponentials on the SFU.
-        const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t scale2 = MODS ? f2_pack(1.f, 1.f) : f2_pack(p.scale_log2, p.scale_log2);
         const uint64_t nbase2 = f2_pack(-base, -base);
         uint64_t rs2[NP / 2];
 #pragma unroll
@@ -441,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      uint16_t* orow = p.out + ((size_t)(wk.q_start + qrow) * p.num_q_heads + wk.head) * D;
+      uint16_t* orow = p.out + out_offset<D, STRIDED>(p, wk.q_start + qrow, wk.head);
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t ov[32];
@@ -477,16 +533,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+template <int D, bool H, bool MODS, bool STRIDED>
+static cudaError_t launch_prefill_m(const PrefillParams& p, const CUtensorMap& q_map,
+                                    const CUtensorMap& k_map, const CUtensorMap& v_map, int grid,
+                                    cudaStream_t stream) {
+  using SM = PrefillSmem<D>;
+  auto kernel = prefill_kernel<D, H, MODS, STRIDED>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc);
+  if (e != cudaSuccess) return e;
+  kernel<<<grid, kThreads, SM::kAlloc, stream>>>(p, q_map, k_map, v_map);
+  return cudaGetLastError();
+}
+
 template <int D, bool H>
 static cudaError_t launch_prefill_t(const PrefillParams& p, const CUtensorMap& q_map,
                                     const CUtensorMap& k_map, const CUtensorMap& v_map, int grid,
                                     cudaStream_t stream) {
-  using SM = PrefillSmem<D>;
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, H>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc);
-  if (e != cudaSuccess) return e;
-  prefill_kernel<D, H><<<grid, kThreads, SM::kAlloc, stream>>>(p, q_map, k_map, v_map);
-  return cudaGetLastError();
+  const bool strided = p.q_hnd || p.kv_hnd || p.o_tok != (long long)p.num_q_heads * D ||
+                       p.o_head != D;
+  if (p.mods.any())
+    return strided ? launch_prefill_m<D, H, true, true>(p, q_map, k_map, v_map, grid, stream)
+                   : launch_prefill_m<D, H, true, false>(p, q_map, k_map, v_map, grid, stream);
+  return strided ? launch_prefill_m<D, H, false, true>(p, q_map, k_map, v_map, grid, stream)
+                 : launch_prefill_m<D, H, false, false>(p, q_map, k_map, v_map, grid, stream);
 }
 
 cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& q_map,

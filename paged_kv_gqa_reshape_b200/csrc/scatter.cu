@@ -2,9 +2,10 @@
 // PR #853 "Pytorch Native Attention on Spyre", description, step 1).
 //
 // One warp per token: it reads the token's K and V rows (num_kv_heads *
-// head_dim bf16 each, contiguous) with 16-byte loads and stores them to slot
-// slot_mapping[t] of the caches, whose rows are contiguous too
-// ([num_blocks, block_size, Hkv, D] => slot s starts at s * Hkv * D).  Pure
+// head_dim elements each, contiguous) with 16-byte loads and stores them to
+// slot slot_mapping[t] of the caches: a dense NHD cache holds the slot's
+// [Hkv, D] row contiguously; other layouts (HND: each head's D elements of
+// the slot at their own stride) take the per-head destination.  Pure
 // bandwidth: every byte is read once and written once.  A negative slot marks
 // a padding token (skipped); a slot beyond the pool is skipped and reported.
 #include "common.cuh"
@@ -19,7 +20,12 @@ __global__ void __launch_bounds__(256) write_kv_kernel(const uint4* __restrict__
                                                        uint4* __restrict__ k_cache,
                                                        uint4* __restrict__ v_cache,
                                                        long long num_slots, int block_size,
-                                                       long long block_vecs, uint32_t* err) {
+                                                       long long block_vecs, long long slot_vecs,
+                                                       long long head_vecs, int dshift,
+                                                       uint32_t* err) {
+  // dense rows ([Hkv, D] contiguous per slot): vector idx of the token row
+  // lands at vector idx of the slot row
+  const bool dense = head_vecs == (1ll << dshift) && slot_vecs == row_vecs;
   const int lane = threadIdx.x & 31;
   const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
   for (long long t = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -33,9 +39,13 @@ __global__ void __launch_bounds__(256) write_kv_kernel(const uint4* __restrict__
     const uint4* ks = k + t * row_vecs;
     const uint4* vs = v + t * row_vecs;
     // block slot / block_size, row slot % block_size (blocks block_vecs apart)
-    const long long at = (slot / block_size) * block_vecs + (slot % block_size) * row_vecs;
+    const long long at = (slot / block_size) * block_vecs + (slot % block_size) * slot_vecs;
     uint4* kd = k_cache + at;
     uint4* vd = v_cache + at;
+    // vector idx = head * (D / 8) + c of the token row goes to head * head_vecs + c
+    auto dst = [&](int idx) -> long long {
+      return dense ? idx : (long long)(idx >> dshift) * head_vecs + (idx & ((1 << dshift) - 1));
+    };
     // issue all loads of this lane before its stores (row_vecs <= 32 * 8 here)
     constexpr int kMaxPerLane = 8;
     uint4 kr[kMaxPerLane], vr[kMaxPerLane];
@@ -51,21 +61,22 @@ __global__ void __launch_bounds__(256) write_kv_kernel(const uint4* __restrict__
     for (int i = 0; i < kMaxPerLane; ++i) {
       const int idx = i * 32 + lane;
       if (idx < row_vecs) {
-        kd[idx] = kr[i];
-        vd[idx] = vr[i];
+        kd[dst(idx)] = kr[i];
+        vd[dst(idx)] = vr[i];
       }
     }
     // rows wider than 32 * 8 vectors (Hkv * D > 2048) continue here
     for (int idx = kMaxPerLane * 32 + lane; idx < row_vecs; idx += 32) {
-      kd[idx] = __ldcs(ks + idx);
-      vd[idx] = __ldcs(vs + idx);
+      kd[dst(idx)] = __ldcs(ks + idx);
+      vd[dst(idx)] = __ldcs(vs + idx);
     }
   }
 }
 
 cudaError_t launch_write_kv(const void* k, const void* v, const int64_t* slot_mapping,
                             int64_t num_tokens, int row_vecs, void* k_cache, void* v_cache,
-                            int64_t num_slots, int block_size, int64_t block_vecs, uint32_t* err,
+                            int64_t num_slots, int block_size, int64_t block_vecs,
+                            int64_t slot_vecs, int64_t head_vecs, int dshift, uint32_t* err,
                             int num_sms, cudaStream_t stream) {
   if (num_tokens <= 0) return cudaSuccess;
   const int threads = 256;
@@ -76,7 +87,7 @@ cudaError_t launch_write_kv(const void* k, const void* v, const int64_t* slot_ma
   write_kv_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
       static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping, num_tokens,
       row_vecs, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), num_slots, block_size,
-      block_vecs, err);
+      block_vecs, slot_vecs, head_vecs, dshift, err);
   return cudaGetLastError();
 }
 

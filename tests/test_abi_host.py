@@ -165,3 +165,90 @@ def test_python_binding_rejects_cpu_and_wrong_dtypes():
                             2, 0.1, True, q)
     with pytest.raises(TypeError):
         pa.write_kv(q.float(), q, torch.zeros(4, dtype=torch.int64), kc, kc)
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    # the C structs of include/pa.h, laid out by the C compiler, against the
+    # ctypes mirrors the binding passes by pointer
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stddef.h>\n#include <stdio.h>\n#include "pa.h"\n'
+        'int main(void) {\n'
+        '  printf("%zu %zu %zu %zu %zu %zu\\n", sizeof(pa_score_mods),\n'
+        '         offsetof(pa_score_mods, alibi_slopes), offsetof(pa_score_mods, mask),\n'
+        '         offsetof(pa_score_mods, mask_len), sizeof(pa_strides),\n'
+        '         offsetof(pa_strides, cache_head));\n'
+        '  return 0;\n}\n')
+    exe = tmp_path / "layout"
+    import subprocess
+    subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    got = [int(x) for x in subprocess.check_output([str(exe)]).split()]
+    want = [ctypes.sizeof(pa._ScoreMods), pa._ScoreMods.alibi_slopes.offset,
+            pa._ScoreMods.mask.offset, pa._ScoreMods.mask_len.offset, ctypes.sizeof(pa._Strides),
+            pa._Strides.cache_head.offset]
+    assert got == want
+
+
+def _mods_call(lib, strides=None, mods=None, **over):
+    a = dict(q=1 << 12, kc=1 << 12, vc=1 << 12, bt=1 << 12, mb=4, sl=1 << 12, qsl=1 << 12,
+             S=2, T=4, Hq=4, Hkv=2, D=64, BS=16, NB=8, dtype=0, mql=4, msl=64, scale=0.125,
+             causal=1, so=None, sp=None, nsp=0)
+    a.update(over)
+    return lib.pa_attention_varlen_mods(
+        *a.values(), ctypes.byref(strides) if strides is not None else None,
+        ctypes.byref(mods) if mods is not None else None, 1 << 12, 1 << 12, 1 << 30, None)
+
+
+def test_varlen_mods_rejects_layouts_and_modifiers_before_launch():
+    lib = pa.load()
+    S = pa._Strides
+    # q: head stride below D with a token stride that is not head-major either
+    assert _mods_call(lib, S(64, 32, 0, 0, 0, 0, 0)) == 2
+    # q stride not a multiple of 8 elements
+    assert _mods_call(lib, S(4 * 64 + 4, 64, 0, 0, 0, 0, 0)) == 1
+    # cache: overlapping head rows, then a block stride smaller than a block
+    assert _mods_call(lib, S(0, 0, 0, 0, 16 * 96, 96, 32)) == 2
+    assert _mods_call(lib, S(0, 0, 0, 0, 8, 2 * 64, 64)) == 1
+    # head-major cache with a block stride short of its extent
+    assert _mods_call(lib, S(0, 0, 0, 0, 2 * 16 * 64 - 8, 64, 16 * 64)) == 1
+    M = pa._ScoreMods
+    assert _mods_call(lib, None, M(-1.0, None, None, 0, 0, 0)) == 1            # negative cap
+    assert _mods_call(lib, None, M(float("inf"), None, None, 0, 0, 0)) == 1
+    assert _mods_call(lib, None, M(0.0, (1 << 12) + 2, None, 0, 0, 0)) == 1    # slopes misaligned
+    assert _mods_call(lib, None, M(0.0, None, (1 << 12) + 4, 0, 64, 64)) == 1  # mask misaligned
+    assert _mods_call(lib, None, M(0.0, None, 1 << 12, 0, 66, 64)) == 1        # row stride % 4
+    assert _mods_call(lib, None, M(0.0, None, 1 << 12, 0, 64, 0)) == 1         # mask_len 0
+    assert _mods_call(lib, None, M(0.0, None, None, 0, 0, 0), S=0) == 0       # empty batch
+
+
+def test_write_kv_strided_rejects_before_launch():
+    lib = pa.load()
+    S = pa._Strides
+
+    def wkv(strides, **over):
+        a = dict(k=1 << 12, v=1 << 12, sm=1 << 12, T=4, Hkv=2, D=64, kc=1 << 12, vc=1 << 12,
+                 NB=8, BS=16)
+        a.update(over)
+        return lib.pa_write_kv_strided(*a.values(), ctypes.byref(strides), 0, None, None)
+    assert wkv(S(0, 0, 0, 0, 16 * 96, 96, 32)) == 2       # overlapping rows
+    assert wkv(S(0, 0, 0, 0, 2 * 16 * 64, 64, 16 * 64 + 4)) == 1
+    assert wkv(S(0, 0, 0, 0, 2 * 16 * 64, 64, 16 * 64), D=48) == 2   # D/8 not a power of two
+    assert wkv(S(0, 0, 0, 0, 2 * 16 * 64, 64, 16 * 64), T=0) == 0
+
+
+def test_smallseq_bwd_rejects_before_launch():
+    lib = pa.load()
+
+    def bwd(**over):
+        a = dict(q=1 << 12, k=1 << 12, v=1 << 12, do=1 << 12, w=1 << 12, wl=16, cu=1 << 12,
+                 B=4, Hq=4, Hkv=2, D=128, mx=16, scale=0.1, dtype=0, dq=1 << 12, dk=1 << 12,
+                 dv=1 << 12, ws=None, stream=None)
+        a.update(over)
+        return lib.pa_attention_smallseq_bwd(*a.values())
+    assert bwd(mx=17) == 2
+    assert bwd(Hq=34, Hkv=2) == 2        # 17 query heads per KV head
+    assert bwd(wl=0) == 1
+    assert bwd(w=(1 << 12) + 1) == 1
+    assert bwd(dk=(1 << 12) + 8) == 1
+    assert bwd(D=96) == 2
+    assert bwd(B=0) == 0
