@@ -144,7 +144,9 @@ size_t pa_attention_varlen_workspace_size(int32_t num_seqs, int64_t num_q_tokens
  *                   the prefill kernel is not launched).  A violated hint
  *                   raises PA_DEVERR_HINT.
  *  max_seq_len      host hint: >= every Lkv; checked like max_query_len.
- *  scale            multiplies q . k (usually 1/sqrt(head_dim))
+ *  scale            multiplies q . k (usually 1/sqrt(head_dim)); finite, >= 0 (the
+ *                   prefill takes its row maxima before scaling), else
+ *                   PA_ERR_INVALID_ARG
  *  causal           0 or 1
  *  out              [num_q_tokens, num_q_heads, head_dim] bf16, written for
  *                   every token that belongs to a sequence

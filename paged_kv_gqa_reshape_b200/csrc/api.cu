@@ -273,7 +273,7 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
   if (num_seqs < 0 || num_q_tokens < 0 || num_q_tokens > 0x7fffffffll || num_q_heads <= 0 ||
       num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || max_blocks_per_seq <= 0 ||
       num_blocks <= 0 || num_blocks > 0x7fffffffll || max_query_len < 0 || max_seq_len < 0 ||
-      (causal != 0 && causal != 1) || !isfinite(scale))
+      (causal != 0 && causal != 1) || !isfinite(scale) || scale < 0.f)
     return PA_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (block_size != pa::kPageKeys) return PA_ERR_UNSUPPORTED;

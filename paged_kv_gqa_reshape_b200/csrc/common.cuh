@@ -78,13 +78,18 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // ---------------------------------------------------------------------------
 constexpr float kLog2e = 1.4426950408889634f;
 
-// tanh(x) from the identity tanh x = 1 - 2 / (e^{2x} + 1), with e^{2x} from
-// the SFU exponential (2^(2 x log2 e)).  |x| is clamped to 20, where tanh is
-// +-1 in fp32, so the exponential stays finite; absolute error ~1e-7.
+// Hardware reciprocal approximation (rcp.approx; rcp(+inf) = +0).
+__device__ __forceinline__ float fast_rcp(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// tanh(x) from the identity tanh x = 1 - 2 / (e^{2x} + 1), with e^{2x} and
+// the reciprocal on the SFU.  Saturates without a clamp: e^{2x} = +inf gives
+// rcp = 0 (tanh 1), e^{2x} -> 0 gives rcp(1) (tanh -1); absolute error ~1e-7.
 __device__ __forceinline__ float tanh_sfu(float x) {
-  x = fminf(fmaxf(x, -20.f), 20.f);
-  const float e = fast_exp2(x * (2.f * kLog2e));
-  return 1.f - __fdividef(2.f, e + 1.f);
+  return fmaf(-2.f, fast_rcp(fast_exp2(x * (2.f * kLog2e)) + 1.f), 1.f);
 }
 
 // Packed 16-bit multiply of two element pairs, round to nearest even.
@@ -140,6 +145,13 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, bool valid) {
   int src_bytes = valid ? 16 : 0;  // 0 => the 16 destination bytes are zero-filled
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+// cp.async of 16 bytes reading only the first src_bytes (0..16) from src;
+// the rest of the destination is zero-filled.
+__device__ __forceinline__ void cp_async_16n(uint32_t dst, const void* src, int src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
                "r"(src_bytes)
                : "memory");

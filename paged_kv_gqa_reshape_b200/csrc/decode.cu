@@ -99,7 +99,12 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
   float* part_buf = reinterpret_cast<float*>(ws + p.L.partial);
 
   __nv_bfloat16* ring = reinterpret_cast<__nv_bfloat16*>(smem);
-  int* s_pg = reinterpret_cast<int*>(smem + Shape::kRingBytes);  // [S + 1] page prefix
+  // with an additive mask, each ring stage also holds the page's 16 mask
+  // values of every query head of the CTA (copied with the page's K/V)
+  constexpr int kMaskHeads = HPC * NGT * 8;
+  constexpr int kMaskStage = MODS ? kMaskHeads * kPageKeys : 0;  // floats per stage
+  float* mring = reinterpret_cast<float*>(smem + Shape::kRingBytes);
+  int* s_pg = reinterpret_cast<int*>(smem + Shape::kRingBytes + NSTAGE * kMaskStage * 4);  // [S + 1] page prefix
   int* s_kv = s_pg + kSelfPlanMaxSeqs + 1;                       // [S] decode kv_len or -1
   __shared__ uint32_t s_err;
   __shared__ int s_scan[HPC];
@@ -203,6 +208,7 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
   int seq_p = seq_of(b0);
   long long p_first = pfx(seq_p), p_end = pfx(seq_p + 1);
   int p_kv = seq_kv(seq_p);
+  [[maybe_unused]] int p_tok = MODS ? seq_q(seq_p) : 0;  // the sequence's query token
   long long x = b0;  // consumer position
   auto issue_page = [&]() {
     const int stage = (int)((x_p - b0) % NSTAGE);
@@ -213,6 +219,26 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
     if (!block_ok && tid == 0) raise_error(err, PA_DEVERR_BLOCK);
     const size_t base =
         (size_t)(block_ok ? block : 0) * p.block_stride + (size_t)hg * HPC * p.c_head;
+    if constexpr (MODS) {
+      if (p.mods.mask) {
+        // the page's mask values: 16 keys (4 chunks of 4) for each query-head
+        // slot (warp w's local head hl) of the CTA; keys past the sequence
+        // end or the mask row read nothing and are zero-filled
+        float* mdst = mring + (size_t)stage * kMaskStage;
+        const long long lim = min((long long)p_kv, p.mods.mask_len);
+        for (int ci = tid; ci < kMaskHeads * 4; ci += NT) {
+          const int hs = ci >> 2, q4 = ci & 3;
+          const int w = hs / (NGT * 8), hl = hs - w * (NGT * 8);
+          const int k = key0 + 4 * q4;
+          const int nb = (hl < g) ? (int)max(0ll, min(4ll, lim - k)) * 4 : 0;
+          const float* src = p.mods.mask + (size_t)((hg * HPC + w) * g + hl) * p.mods.mask_head +
+                             (size_t)p_tok * p.mods.mask_tok + k;
+          cp_async_16n(smem_u32(mdst + hs * kPageKeys + 4 * q4), nb ? src : p.mods.mask, nb);
+        }
+        if (tid == 0 && min((long long)p_kv, (long long)key0 + kPageKeys) > p.mods.mask_len)
+          raise_error(err, PA_DEVERR_HINT);
+      }
+    }
     __nv_bfloat16* kdst = ring + (size_t)stage * 2 * Shape::kTensorStage;
     __nv_bfloat16* vdst = kdst + Shape::kTensorStage;
 #pragma unroll
@@ -236,6 +262,7 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
       p_first = pfx(seq_p);
       p_end = pfx(seq_p + 1);
       p_kv = seq_kv(seq_p);
+      if constexpr (MODS) p_tok = seq_q(seq_p);
     }
   };
   auto fill = [&]() {
@@ -280,6 +307,19 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
       for (int mt = 0; mt < KSTEPS; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
     }
 
+    // ALiBi slopes (log2 units) of this lane's heads, two per n-tile
+    [[maybe_unused]] float msl[NGT][2];
+    if constexpr (MODS) {
+#pragma unroll
+      for (int nt = 0; nt < NGT; ++nt) {
+        const int hl0 = nt * 8 + 2 * tq;
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+          msl[nt][j] = (p.mods.alibi && hl0 + j < g) ? __ldg(p.mods.alibi + head0 + hl0 + j) * kLog2e
+                                                      : 0.f;
+      }
+    }
+
     for (; x < seg_end; ++x) {
       cp_async_wait_dyn((int)(x_p - x - 1));  // my copies of page x have landed
       __syncthreads();  // everyone's have, and page x-1's stage is free
@@ -312,29 +352,29 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
       for (int nt = 0; nt < NGT; ++nt) {
         float s0, s1, s2, s3;
         if constexpr (MODS) {
-          // soft-cap, ALiBi, additive mask on scale * s (then log2 units);
-          // the query sits at key position seg_kv - 1
-          const int hl0 = nt * 8 + 2 * tq;
-          auto mod = [&](float raw, int hl, int key) {
-            float t = raw * p.scale;
-            if (p.mods.softcap > 0.f) t = p.mods.softcap * tanh_sfu(t * (1.f / p.mods.softcap));
-            if (hl < g) {
-              const int h = head0 + hl;
-              if (p.mods.alibi) t = fmaf(__ldg(p.mods.alibi + h), (float)(key - (seg_kv - 1)), t);
-              if (p.mods.mask) {
-                if (key < p.mods.mask_len)
-                  t += __ldg(p.mods.mask + (size_t)h * p.mods.mask_head +
-                             (size_t)seg_q * p.mods.mask_tok + key);
-                else
-                  raise_error(err, PA_DEVERR_HINT);
-              }
-            }
-            return t * kLog2e;
+          // soft-cap, ALiBi, additive mask on scale * s, in log2 units; the
+          // query sits at key position seg_kv - 1
+          const float cap = p.mods.softcap;
+          const float a1 = cap > 0.f ? p.scale / cap : p.scale_log2, a2 = cap * kLog2e;
+          auto mod = [&](float raw, float slope2, float mv, int key) {
+            const float x = raw * a1;
+            const float t = cap > 0.f ? a2 * tanh_sfu(x) : x;
+            return fmaf(slope2, (float)(key - (seg_kv - 1)), t) + mv;
           };
-          s0 = ok0 ? mod(sc[nt][0], hl0, key0 + gq) : -INFINITY;
-          s1 = ok0 ? mod(sc[nt][1], hl0 + 1, key0 + gq) : -INFINITY;
-          s2 = ok1 ? mod(sc[nt][2], hl0, key0 + gq + 8) : -INFINITY;
-          s3 = ok1 ? mod(sc[nt][3], hl0 + 1, key0 + gq + 8) : -INFINITY;
+          // this page's mask values (log2 units) from the ring stage
+          float mv[4] = {0.f, 0.f, 0.f, 0.f};
+          if (p.mods.mask) {
+            const float* mst = mring + (size_t)((x - b0) % NSTAGE) * kMaskStage +
+                               (size_t)(warp * NGT * 8 + nt * 8 + 2 * tq) * kPageKeys + gq;
+            mv[0] = mst[0] * kLog2e;
+            mv[1] = mst[kPageKeys] * kLog2e;
+            mv[2] = mst[8] * kLog2e;
+            mv[3] = mst[kPageKeys + 8] * kLog2e;
+          }
+          s0 = ok0 ? mod(sc[nt][0], msl[nt][0], mv[0], key0 + gq) : -INFINITY;
+          s1 = ok0 ? mod(sc[nt][1], msl[nt][1], mv[1], key0 + gq) : -INFINITY;
+          s2 = ok1 ? mod(sc[nt][2], msl[nt][0], mv[2], key0 + gq + 8) : -INFINITY;
+          s3 = ok1 ? mod(sc[nt][3], msl[nt][1], mv[3], key0 + gq + 8) : -INFINITY;
         } else {
           s0 = ok0 ? sc[nt][0] * p.scale_log2 : -INFINITY;
           s1 = ok0 ? sc[nt][1] * p.scale_log2 : -INFINITY;
@@ -582,7 +622,8 @@ template <int D, int HPC, int NSTAGE, int NGT, bool H, bool MODS>
 cudaError_t launch_t(const DecodeParams& p, int num_sms, cudaStream_t stream) {
   using Shape = DecodeShape<D, HPC, NSTAGE>;
   auto kernel = decode_kernel<D, HPC, NSTAGE, NGT, H, MODS>;
-  const int smem = Shape::smem_bytes(p.self_plan != 0);
+  const int smem =
+      Shape::smem_bytes(p.self_plan != 0) + (MODS ? NSTAGE * HPC * NGT * 8 * kPageKeys * 4 : 0);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
@@ -618,8 +659,10 @@ cudaError_t launch_decode_t(const DecodeParams& p, int head_dim, int num_sms,
     if (p.group <= 8) return launch_hpc<128, 3, 1, H, MODS>(p, hpc, num_sms, stream);
     return launch_hpc<128, 3, 2, H, MODS>(p, hpc, num_sms, stream);
   }
-  if (p.group <= 8) return launch_hpc<64, 6, 1, H, MODS>(p, hpc, num_sms, stream);
-  return launch_hpc<64, 6, 2, H, MODS>(p, hpc, num_sms, stream);
+  // head_dim 64 with modifiers: 4 stages, so the mask stages fit beside the ring
+  constexpr int kStages64 = MODS ? 4 : 6;
+  if (p.group <= 8) return launch_hpc<64, kStages64, 1, H, MODS>(p, hpc, num_sms, stream);
+  return launch_hpc<64, kStages64, 2, H, MODS>(p, hpc, num_sms, stream);
 }
 
 }  // namespace

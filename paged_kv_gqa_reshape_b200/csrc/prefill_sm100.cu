@@ -382,21 +382,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(s_col + c, *reinterpret_cast<uint32_t(*)[32]>(&sv[c]));
         tmem_ld_wait();
         if constexpr (MODS) {
-          // soft-cap, ALiBi and the additive mask on scale * s, to log2 units;
-          // keys past `valid` get -inf below, so their mask values are not read
-          const int vis = masked_tile ? max(0, min(valid, BN)) : BN;
-          int mlim = 0;  // keys of this tile with a mask value
-          if (mrow) {
-            const long long left = p.mods.mask_len - key0;
-            mlim = (int)max(0ll, min((long long)vis, left));
-            if (mlim < vis) raise_error(err, PA_DEVERR_HINT);
-          }
-          const float cap = p.mods.softcap, inv_cap = cap > 0.f ? 1.f / cap : 0.f;
-          const float rel0 = (float)(key0 - pos);
+          // The modifiers act in raw-score units, so the plain path's scaling
+          // (after the max, in the exponent) still applies: raw <- (cap /
+          // scale) tanh(raw scale / cap), then + (slope (j - pos) + mask) /
+          // scale.  One uniform branch per modifier; keys past `valid` get
+          // -inf below, so their mask values are not read.
+          if (p.mods.softcap > 0.f) {
+            const float a1 = p.scale / p.mods.softcap, capr = p.mods.softcap / p.scale;
 #pragma unroll
-          for (int c = 0; c < BN; c += 4) {
-            float4 mv = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (mrow) {
+            for (int c = 0; c < BN; ++c)
+              sv[c] = __float_as_uint(capr * tanh_sfu(__uint_as_float(sv[c]) * a1));
+          }
+          if (slope != 0.f) {
+            // + slope' (key0 - pos + c), slope' = slope / scale, on fp32 pairs
+            const float sr = slope / p.scale;
+            const uint64_t step2 = f2_pack(sr, sr);
+            const float b0 = sr * (float)(key0 - pos);
+#pragma unroll
+            for (int c = 0; c < BN; c += 2) {
+              const uint64_t bias = f2_fma(step2, f2_pack((float)c, (float)(c + 1)), f2_pack(b0, b0));
+              const uint64_t v = f2_add(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
+                                        bias);
+              sv[c] = __float_as_uint(f2_lo(v));
+              sv[c + 1] = __float_as_uint(f2_hi(v));
+            }
+          }
+          if (mrow) {
+            const int vis = masked_tile ? max(0, min(valid, BN)) : BN;
+            const long long left = p.mods.mask_len - key0;
+            const int mlim = (int)max(0ll, min((long long)vis, left));  // keys with a mask value
+            if (mlim < vis) raise_error(err, PA_DEVERR_HINT);
+            const float is = 1.f / p.scale;
+            const uint64_t is2 = f2_pack(is, is);
+#pragma unroll
+            for (int c = 0; c < BN; c += 4) {
+              float4 mv = make_float4(0.f, 0.f, 0.f, 0.f);
               if (c + 4 <= mlim) {
                 mv = __ldg(reinterpret_cast<const float4*>(mrow + key0 + c));
               } else if (c < mlim) {
@@ -404,14 +424,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (c + 1 < mlim) mv.y = __ldg(mrow + key0 + c + 1);
                 if (c + 2 < mlim) mv.z = __ldg(mrow + key0 + c + 2);
               }
-            }
-            const float m4[4] = {mv.x, mv.y, mv.z, mv.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float t = __uint_as_float(sv[c + e]) * p.scale;
-              if (cap > 0.f) t = cap * tanh_sfu(t * inv_cap);
-              t = fmaf(slope, rel0 + (float)(c + e), t) + m4[e];
-              sv[c + e] = __float_as_uint(t * kLog2e);
+              const uint64_t v0 = f2_fma(f2_pack(mv.x, mv.y), is2,
+                                         f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])));
+              const uint64_t v1 = f2_fma(f2_pack(mv.z, mv.w), is2,
+                                         f2_pack(__uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3])));
+              sv[c] = __float_as_uint(f2_lo(v0));
+              sv[c + 1] = __float_as_uint(f2_hi(v0));
+              sv[c + 2] = __float_as_uint(f2_lo(v1));
+              sv[c + 3] = __float_as_uint(f2_hi(v1));
             }
           }
         }
@@ -433,9 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int wdt = NP / 2; wdt >= 1; wdt >>= 1)
 #pragma unroll
           for (int i = 0; i < wdt; ++i) mp[i] = fmaxf(mp[i], mp[i + wdt]);
-        // with MODS the scores are already in log2 units; else the scale
-        // (> 0, so the max commutes with it) is applied here
-        const float m_tile = mp[0] * (MODS ? 1.f : p.scale_log2);
+        const float m_tile = mp[0] * p.scale_log2;  // scale_log2 > 0: max commutes with it
         const float m_old = m_use;
         const bool grow =
             m_tile > m_old + kRescaleThreshold || (m_old == -INFINITY && m_tile > -INFINITY);
@@ -446,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // p = 2^(scale_log2 * s - base), rounded to bf16 and written to TMEM as
         // the A operand of O += P.V.  Scaling and row sums run on packed fp32
         // pairs; the exponentials on the SFU.
-        const uint64_t scale2 = MODS ? f2_pack(1.f, 1.f) : f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
         const uint64_t nbase2 = f2_pack(-base, -base);
         uint64_t rs2[NP / 2];
 #pragma unroll

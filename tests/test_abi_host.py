@@ -62,6 +62,7 @@ def _varlen(lib, **over):
     (dict(Hq=34, Hkv=2), 2),          # GQA group > 16
     (dict(causal=2), 1),
     (dict(scale=float("nan")), 1),
+    (dict(scale=-0.125), 1),          # negative scale
     (dict(q=0), 1),                   # null pointer
     (dict(q=(1 << 12) + 2), 1),       # misaligned
     (dict(wsb=16), 1),                # workspace too small
