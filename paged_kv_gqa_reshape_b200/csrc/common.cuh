@@ -274,6 +274,18 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* map, uint6
       "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start before its predecessor finishes; griddep_wait
+// blocks the calling thread until the predecessor grids have completed and
+// their memory is visible; griddep_launch_dependents lets the next grid
+// start early.  Both are no-ops for an ordinary launch.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Start the line holding `ptr` towards L1 (no register is written).
 __device__ __forceinline__ void prefetch_l1(const void* ptr) {
   asm volatile("prefetch.global.L1 [%0];" ::"l"(ptr));

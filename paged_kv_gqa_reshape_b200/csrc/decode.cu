@@ -77,6 +77,11 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
   constexpr unsigned FULL = 0xffffffffu;
 
   extern __shared__ __align__(128) unsigned char smem[];
+  // Launched with programmatic stream serialisation: when the previous
+  // kernel lets this one start early (the cache scatter does), the CTAs are
+  // resident before it ends and wait here, before reading any input, until
+  // it has completed and its writes are visible.
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int tid = threadIdx.x;
@@ -637,8 +642,17 @@ cudaError_t launch_t(const DecodeParams& p, int num_sms, cudaStream_t stream) {
   const long long cap = (kDecodeMaxWarps + p.num_kv_heads - 1) / p.num_kv_heads;
   if (ranges > cap) ranges = cap;
   if (ranges < 1) ranges = 1;
-  kernel<<<(unsigned)(ranges * groups), HPC * 32, smem, stream>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(ranges * groups));
+  cfg.blockDim = dim3(HPC * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
 template <int D, int NSTAGE, int NGT, bool H, bool MODS>

@@ -26,6 +26,9 @@ __global__ void __launch_bounds__(256) write_kv_kernel(const uint4* __restrict__
   // dense rows ([Hkv, D] contiguous per slot): vector idx of the token row
   // lands at vector idx of the slot row
   const bool dense = head_vecs == (1ll << dshift) && slot_vecs == row_vecs;
+  // the attention call that follows reads the caches only after this grid has
+  // completed (griddep_wait); its planning may overlap this scatter
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
   for (long long t = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
