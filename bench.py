@@ -230,7 +230,8 @@ def device_case(case, dev):
 
 def time_varlen_component(pa, case, iters=20, warmup=3, with_scatter=False, **mods):
     """Average device time (ms) of one attention_varlen call on `case` (device
-    tensors); `mods` (softcap, alibi_slopes, mask) go to the call."""
+    tensors): CUDA events around back-to-back calls.  `mods` (softcap,
+    alibi_slopes, mask) go to the call."""
     ws = pa.varlen_workspace(case.num_seqs, case.num_q_tokens, case.num_q_heads,
                              case.num_kv_heads, case.head_dim)
     out = torch.empty_like(case.q)
@@ -248,17 +249,23 @@ def time_varlen_component(pa, case, iters=20, warmup=3, with_scatter=False, **mo
     for _ in range(warmup):
         run()
     torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(iters)]
-    for a, b in evs:
-        a.record()
-        run()
-        b.record()
-    torch.cuda.synchronize()
+    ms = b2b_ms(run, iters)
     st, bits = pa.get_error(ws)
     if st != 0:
         raise RuntimeError(f"device error word {bits:#x}")
-    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+    return ms
+
+
+def b2b_ms(fn, iters):
+    """Device time (ms) per call of fn: CUDA events around `iters` back-to-back
+    calls on the launching stream (no event between calls)."""
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(iters):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
 
 
 def time_spans_component(pa, case, span_offsets, spans, iters=20, warmup=3):
@@ -278,31 +285,19 @@ def time_spans_component(pa, case, span_offsets, spans, iters=20, warmup=3):
     for _ in range(warmup):
         run()
     torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(iters)]
-    for a, b in evs:
-        a.record()
-        run()
-        b.record()
-    torch.cuda.synchronize()
+    ms = b2b_ms(run, iters)
     st, bits = pa.get_error(ws)
     if st != 0:
         raise RuntimeError(f"device error word {bits:#x}")
-    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+    return ms
 
 
 def time_calls(fn, iters=20, warmup=3):
-    """Device time per call (ms) of `fn`, CUDA events on the current stream."""
+    """Device time per call (ms) of `fn`: back-to-back calls (b2b_ms)."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(iters):
-        fn()
-    b.record()
-    torch.cuda.synchronize()
-    return a.elapsed_time(b) / iters
+    return b2b_ms(fn, iters)
 
 
 def smallseq_weight_bytes(ss, wlen):
@@ -333,19 +328,18 @@ def components(pa, hbm_peak, tc_peak, peak_kind):
     res["varlen_prefill"] = {"ms": round(ms, 4), "tflops": round(tf, 1),
                              "frac": round(tf / tc_peak, 3), "peak": tc_peak,
                              "unit": "TFLOP/s", "of": peak_kind}
+    # the scatter alone: the same step's 17 336 new tokens into the paged caches
+    ms = time_calls(lambda: pa.write_kv(vc.k_new, vc.v_new, vc.slot_mapping, vc.k_cache,
+                                        vc.v_cache), iters=50)
+    gbs = scatter_bytes(vc) / (ms * 1e-3) / 1e9
+    res["scatter_varlen_prefill"] = {"ms": round(ms, 4), "gbs": round(gbs, 1),
+                                     "frac": round(gbs / hbm_peak, 3), "unit": "GB/s",
+                                     "of": peak_kind}
     del vc
     ss = workloads.smallseq_batch(device=dev)
     out = torch.empty_like(ss.q)
-    for _ in range(3):
-        pa.attention_smallseq(ss.q, ss.k, ss.v, ss.cu_seqlens_kv, ss.scale, out)
-    torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(20):
-        pa.attention_smallseq(ss.q, ss.k, ss.v, ss.cu_seqlens_kv, ss.scale, out)
-    b.record()
-    torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / 20
+    ms = time_calls(lambda: pa.attention_smallseq(ss.q, ss.k, ss.v, ss.cu_seqlens_kv, ss.scale,
+                                                  out))
     nbytes = (ss.k.numel() + ss.v.numel() + ss.q.numel() + out.numel()) * 2 + 4 * (ss.batch + 1)
     gbs = nbytes / (ms * 1e-3) / 1e9
     res["smallseq_batch"] = {"ms": round(ms, 4), "gbs": round(gbs, 1),
@@ -425,8 +419,10 @@ def components(pa, hbm_peak, tc_peak, peak_kind):
     pre_fl = fl - 4 * mx.head_dim * mx.num_q_heads * sum(
         int(l) for l, q in zip(mx.seq_lens.tolist(), mx.query_lens.tolist()) if q == 1)
     t_roof = dec_bytes / (hbm_peak * 1e9) + pre_fl / (tc_peak * 1e12)
+    t_max = max(dec_bytes / (hbm_peak * 1e9), pre_fl / (tc_peak * 1e12))
     res["mixed_step"] = {"ms": round(ms, 4), "roofline_ms": round(t_roof * 1e3, 4),
                          "frac_serial": round(t_roof / (ms * 1e-3), 3),
+                         "frac_max": round(t_max / (ms * 1e-3), 3),
                          "decode_gb": round(dec_bytes / 1e9, 2), "prefill_tflop": round(pre_fl / 1e12, 3),
                          "of": peak_kind}
     del mx
@@ -499,9 +495,9 @@ def run_ours(args, rank, world, local_rank):
     if st != 0:
         raise RuntimeError(f"device error word {bits:#x} after warm-up")
 
-    # The step as a serving loop runs it: captured once as a CUDA graph
-    # (write_kv + attention) and replayed, one replay per step.
-    g_step = None if args.no_graph else capture_graph(step, 1)
+    # K steps of stream launches (write_kv + attention); with --graph the step
+    # is captured once as a CUDA graph and replayed once per step
+    g_step = capture_graph(step, 1) if args.graph else None
     if g_step is not None:
         for _ in range(args.warmup):
             g_step.replay()
@@ -527,9 +523,9 @@ def run_ours(args, rank, world, local_rank):
     if st != 0:
         raise RuntimeError(f"device error word {bits:#x} in the timed region")
     del g_step
-    # the decode kernel alone (the roofline's kernel): a graph of 20 attention
-    # calls, CUDA events around each replay on the launching stream
-    attn_ms = time_graph(attention, 20, reps=max(5, min(50, args.steps // 20)))
+    # the decode kernel alone (the roofline's kernel): CUDA events around
+    # back-to-back attention calls on the launching stream
+    attn_ms = b2b_ms(attention, max(20, min(1000, args.steps)))
 
     max_ms = max_over_ranks(elapsed_ms, world, dev)
     bytes_step = scatter_bytes(case) + attention_bytes(case)
@@ -550,16 +546,16 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": WORKLOAD, "global_batch": 64 * world, "seq_len": "256-4096",
                    "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
                    "l2": "inputs larger than L2 (0.57 GB of K/V per step vs 126 MB L2)",
-                   "launch": ("stream launches, one pair of library calls per step" if args.no_graph
-                              else "one CUDA graph of the step (write_kv + attention), "
-                                   "replayed once per step")},
+                   "launch": ("one CUDA graph of the step (write_kv + attention), replayed "
+                              "once per step" if args.graph
+                              else "stream launches, one pair of library calls per step")},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                      "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                      "traffic": args.traffic if args.traffic is not None else recorded_traffic(),
                      "kernel": "decode_kernel (split-KV decode; the call launches only it), "
-                               "CUDA events around replays of a graph of 20 calls",
+                               "CUDA events around back-to-back calls",
                      "peak_kind": peak_kind},
         "clocks": clk,
         "gpu_launches": launches_per_step(case) * args.steps,
@@ -596,6 +592,13 @@ def run_single_workload(args):
         def step():
             pa.attention_smallseq(ss.q, ss.k, ss.v, ss.cu_seqlens_kv, ss.scale, out)
         work = (ss.k.numel() + ss.v.numel() + ss.q.numel() + out.numel()) * 2 + 4 * (ss.batch + 1)
+        unit, scale_div, peak = "GB/s", 1e9, hbm_peak
+    elif name == "scatter_varlen":
+        vc = workloads.varlen_prefill(device=dev, keep_logical=False)
+
+        def step():
+            pa.write_kv(vc.k_new, vc.v_new, vc.slot_mapping, vc.k_cache, vc.v_cache)
+        work = scatter_bytes(vc)
         unit, scale_div, peak = "GB/s", 1e9, hbm_peak
     elif name == "smallseq_bwd":
         ss = workloads.smallseq_batch(device=dev)
@@ -673,9 +676,9 @@ def run_e2e(pa, case, args, dev, ws):
     for _ in range(3):
         step()
     torch.cuda.synchronize()
-    # one CUDA graph of the whole step: the host-to-device copies of its
-    # inputs, the two library calls, the copy of the output back to the host
-    g = None if args.no_graph else capture_graph(step, 1)
+    # with --graph: one CUDA graph of the whole step (the host-to-device copies
+    # of its inputs, the two library calls, the copy of the output back)
+    g = capture_graph(step, 1) if args.graph else None
     if g is not None:
         for _ in range(3):
             g.replay()
@@ -718,6 +721,18 @@ def time_oracle_step(case):
     return time.perf_counter() - t0
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (first `model name` of /proc/cpuinfo)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(budget_s=12.0):
     import oracle
     oracle.build()
@@ -729,7 +744,7 @@ def cpu_baseline(budget_s=12.0):
         times.append(time_oracle_step(case))
     gbs = nbytes * len(times) / sum(times) / 1e9
     return {"value": round(gbs, 4), "unit": "GB/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
+            "cpu": cpu_model(), "kind": "oracle",
             "sample": f"the full 64-sequence decode batch (seed 1002), {len(times)} passes of "
                       f"oracle write_kv + fp64 attention ({sum(times):.1f} s)"}
 
@@ -763,7 +778,7 @@ def run_reference(args, rank, world):
         "config": {"workload": WORKLOAD, "global_batch": 64, "seq_len": "256-4096",
                    "parallelism": "cpu"},
         "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": oracle.num_threads(),
-                         "kind": "oracle",
+                         "cpu": cpu_model(), "kind": "oracle",
                          "sample": "each step: one decode sequence drawn from the workload's "
                                    "distribution (context U[256,4096]), oracle write + attention"},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -779,10 +794,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-components", action="store_true")
-    ap.add_argument("--no-graph", action="store_true",
-                    help="time the step with stream launches instead of a CUDA graph replay")
+    ap.add_argument("--graph", action="store_true",
+                    help="time the step (and the end-to-end leg) as replays of a CUDA graph")
     ap.add_argument("--workload", default="decode_batch",
-                    choices=sorted(list(workloads.NAMED) + ["spans_prefill", "smallseq_bwd"]),
+                    choices=sorted(list(workloads.NAMED) + ["spans_prefill", "smallseq_bwd",
+                                                           "scatter_varlen"]),
                     help="decode_batch is the headline; the others time one workload alone")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per dominant-kernel launch from an ncu capture, if current")
