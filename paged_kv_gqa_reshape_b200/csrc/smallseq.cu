@@ -184,12 +184,17 @@ __global__ void __launch_bounds__(256, 3) smallseq_kernel(SmallSeqParams p) {
       const float winv = sum > 0.f ? 1.f / sum : 0.f;
       uint16_t* wrow = p.weights + ((size_t)b * p.num_q_heads + h) * p.weights_len;
       if (cur.n > p.weights_len && lane == 0) raise_error(p.err, PA_DEVERR_HINT);
+      // lane t writes weight t (one coalesced row store): key t's weight is
+      // pass t / KPP of key group t % KPP, whose lanes all hold it
+      float wt = 0.f;
+      const int src = (lane % KPP) * LPK;
 #pragma unroll
       for (int pp = 0; pp < PASSES; ++pp) {
-        const int j = pp * KPP + sub;
-        if (l == 0 && j < cur.n && j < p.weights_len) wrow[j] = ebits<H>(pwv[pp] * winv);
+        const float v = __shfl_sync(0xffffffffu, pwv[pp], src);
+        if (lane / KPP == pp) wt = v;
       }
-      for (int j = cur.n + lane; j < p.weights_len; j += 32) wrow[j] = 0;
+      for (int t = lane; t < p.weights_len; t += 32)
+        wrow[t] = (t < cur.n && t == lane) ? ebits<H>(wt * winv) : (uint16_t)0;
     }
     if (sub == 0) {
       const float inv = sum > 0.f ? 1.f / sum : 0.f;  // an empty entry writes zeros
