@@ -69,8 +69,8 @@ def _load():
             p, p, p, p, p, p, i32, i32, i32, i32, f64, i32, i32, p, i64, p]
         lib.oracle_attention_varlen_mods.restype = i32
         lib.oracle_attention_varlen_mods.argtypes = [
-            p, p, p, p, p, p, i32, i32, i32, i32, f64, i32, i32, f64, p, p, i64, i64, p, i64,
-            p]
+            p, p, p, p, p, p, i32, i32, i32, i32, f64, i32, i32, f64, p, p, i64, i64, p, p, p,
+            i64, p]
         lib.oracle_attention_smallseq_dtype.restype = i32
         lib.oracle_attention_smallseq_dtype.argtypes = [p, p, p, p, i32, i32, i32, i32, f64, i32, p]
         lib.oracle_smallseq_weights.restype = i32
@@ -159,7 +159,8 @@ def attention_varlen_dtype(q, k_seq, v_seq, kv_offsets, seq_lens, query_start_lo
 
 def attention_varlen_mods(q, k_seq, v_seq, kv_offsets, seq_lens, query_start_loc,
                           num_kv_heads, scale, causal, dtype=0, softcap=0.0, alibi_slopes=None,
-                          mask=None, mask_head_stride=0, mask_token_stride=0, rows=None):
+                          mask=None, mask_head_stride=0, mask_token_stride=0, rows=None,
+                          span_offsets=None, spans=None):
     """attention_varlen with score modifiers: soft-cap (0 = off), ALiBi slopes
     [Hq] float32 or None, an additive float32 mask (flat array addressed as
     h * mask_head_stride + t * mask_token_stride + j) or None."""
@@ -175,11 +176,16 @@ def attention_varlen_mods(q, k_seq, v_seq, kv_offsets, seq_lens, query_start_loc
         raise ValueError("alibi_slopes must be [num_q_heads]")
     out = np.zeros((t, hq, d), dtype=np.float64)
     rows_a = None if rows is None else _arr(rows, np.int64)
+    so = sp = None
+    if span_offsets is not None:
+        so = _arr(span_offsets, np.int32)
+        sp = np.asarray(spans).reshape(-1, 2)
+        sp = _arr(sp if sp.size else np.zeros((1, 2), np.int32), np.int32)
     rc = _load().oracle_attention_varlen_mods(
         _ptr(q), _ptr(k_seq), _ptr(v_seq), _ptr(kv_offsets), _ptr(seq_lens), _ptr(qsl),
         len(seq_lens), hq, num_kv_heads, d, float(scale), int(bool(causal)), int(dtype),
         float(softcap), _ptr(slopes), _ptr(mk), int(mask_head_stride), int(mask_token_stride),
-        _ptr(rows_a), 0 if rows_a is None else len(rows_a), _ptr(out))
+        _ptr(so), _ptr(sp), _ptr(rows_a), 0 if rows_a is None else len(rows_a), _ptr(out))
     if rc != 0:
         raise ValueError(f"oracle_attention_varlen_mods failed ({rc})")
     return out

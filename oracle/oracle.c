@@ -428,7 +428,9 @@ int oracle_attention_varlen_spans(const uint16_t *q, const uint16_t *k_seq,
  * Logical form with score modifiers (see row_mods) and an element type:
  * softcap (0 = off), alibi_slopes [num_q_heads] fp32 or NULL, an additive
  * fp32 mask or NULL with its head / token strides in elements (head stride 0
- * = one mask for every head).  Otherwise as oracle_attention_varlen_dtype.
+ * = one mask for every head), and optional full-attention spans as in
+ * oracle_attention_varlen_spans (then causal is implied).  Otherwise as
+ * oracle_attention_varlen_dtype.
  */
 int oracle_attention_varlen_mods(const uint16_t *q, const uint16_t *k_seq,
                                  const uint16_t *v_seq, const int64_t *kv_offsets,
@@ -438,12 +440,15 @@ int oracle_attention_varlen_mods(const uint16_t *q, const uint16_t *k_seq,
                                  double scale, int causal, int dtype, double softcap,
                                  const float *alibi_slopes, const float *mask,
                                  int64_t mask_head_stride, int64_t mask_token_stride,
+                                 const int32_t *span_offsets, const int32_t *spans,
                                  const int64_t *rows, int64_t num_rows, double *out) {
     if ((dtype != 0 && dtype != 1) || softcap < 0.0) return -1;
+    if (span_offsets && !spans) return -1;
     score_mods sm = {softcap, alibi_slopes, mask, mask_head_stride, mask_token_stride};
     return varlen_driver(q, k_seq, v_seq, kv_offsets, NULL, 0, 1, 0, seq_lens,
                          query_start_loc, num_seqs, num_q_heads, num_kv_heads,
-                         head_dim, scale, causal, NULL, NULL, dtype, &sm, rows, num_rows, out);
+                         head_dim, scale, span_offsets ? 1 : causal, span_offsets, spans, dtype,
+                         &sm, rows, num_rows, out);
 }
 
 /*

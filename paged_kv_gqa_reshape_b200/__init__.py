@@ -376,19 +376,22 @@ def attention_varlen(q, k_cache, v_cache, block_tables, seq_lens, query_start_lo
 
 def attention_varlen_spans(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc,
                            num_kv_heads, scale, span_offsets, spans, out, max_query_len=None,
-                           max_seq_len=None, workspace=None, stream=None):
+                           max_seq_len=None, workspace=None, stream=None, softcap=0.0,
+                           alibi_slopes=None, mask=None):
     """Paged varlen attention with full-attention spans inside causal sequences.
 
     span_offsets: int32 [S+1] (sequence s owns spans span_offsets[s] ..
     span_offsets[s+1]-1); spans: int32 [N, 2] (start, end) key positions.
     A query whose key position lies in a span [start, end) sees keys
-    0 .. end-1; every other query is causal.  Writes out [T, Hq, D].
+    0 .. end-1; every other query is causal.  Writes out [T, Hq, D].  Layouts
+    and score modifiers as attention_varlen.
     """
     if span_offsets is None or spans is None:
         raise ValueError("span_offsets and spans are required")
     return _varlen_ex(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc,
                       num_kv_heads, scale, True, span_offsets, spans, out, max_query_len,
-                      max_seq_len, workspace, stream, "pa_attention_varlen_ex")
+                      max_seq_len, workspace, stream, "pa_attention_varlen_ex", softcap,
+                      alibi_slopes, mask)
 
 
 def attention_varlen_static(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc,

@@ -225,3 +225,32 @@ def test_layout_rejections():
                             dev.query_start_loc, 2, dev.scale, True, out, workspace=ws,
                             mask=mask)
     assert torch.count_nonzero(out) == 0
+
+
+def test_spans_with_modifiers():
+    # full-attention spans (visibility) with ALiBi and a per-head additive mask (scores)
+    lens, qlens = [600, 300], [600, 200]
+    cpu = make(lens, qlens, 8, 2, 128, True, seed=50)
+    so = torch.tensor([0, 2, 3], dtype=torch.int32)
+    sp = torch.tensor([[40, 170], [300, 420], [150, 260]], dtype=torch.int32)
+    t, ld = cpu.num_q_tokens, 608
+    mask = torch.randn(8, t, ld, generator=torch.Generator().manual_seed(10))
+    sl = slopes_for(8)
+    dev = case_to(cpu, "cuda")
+    kc, vc = dev.k_cache.clone(), dev.v_cache.clone()
+    ws = pa.varlen_workspace(dev.num_seqs, dev.num_q_tokens, 8, 2, 128)
+    pa.write_kv(dev.k_new, dev.v_new, dev.slot_mapping, kc, vc, workspace=ws)
+    out = torch.full_like(dev.q, float("nan"))
+    pa.attention_varlen_spans(dev.q, kc, vc, dev.block_tables, dev.seq_lens, dev.query_start_loc,
+                              2, dev.scale, so.cuda(), sp.cuda(), out,
+                              max_query_len=dev.max_query_len, max_seq_len=dev.max_seq_len,
+                              workspace=ws, alibi_slopes=sl.cuda(), mask=mask.cuda())
+    torch.cuda.synchronize()
+    ref = oracle.attention_varlen_mods(
+        workloads.bf16_bits(cpu.q), workloads.bf16_bits(cpu.k_logical),
+        workloads.bf16_bits(cpu.v_logical), cpu.kv_offsets.numpy(), cpu.seq_lens.numpy(),
+        cpu.query_start_loc.numpy(), 2, cpu.scale, True, alibi_slopes=sl.numpy(),
+        mask=mask.numpy().reshape(-1), mask_head_stride=t * ld, mask_token_stride=ld,
+        span_offsets=so.numpy(), spans=sp.numpy())
+    assert_attention_close(out, ref, what="spans + modifiers")
+    assert pa.get_error(ws) == (0, 0)

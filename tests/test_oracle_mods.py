@@ -166,3 +166,26 @@ def test_fully_masked_row_is_zero_and_partial_mask_drops_keys():
     ref9 = torch.nn.functional.scaled_dot_product_attention(
         q[:, 9:10], k[:, :40], v[:, :40], scale=case.scale)
     assert np.max(np.abs(got[9] - ref9[:, 0].numpy())) < 1e-10
+
+
+def test_modifiers_with_spans_match_sdpa():
+    # full-attention spans decide visibility; ALiBi and the mask add to the scores
+    lens = [200]
+    case = make(lens, lens, 4, 2, 64, True, seed=16)
+    spans = [(20, 60), (100, 180)]
+    sl = slopes_for(4)
+    ld = 200
+    mask = (np.random.default_rng(9).standard_normal(200 * ld) * 0.5).astype(np.float32)
+    got = run(case, alibi_slopes=sl, mask=mask, mask_head_stride=0, mask_token_stride=ld,
+              span_offsets=np.array([0, 2], np.int32), spans=np.array(spans, np.int32))
+    q, k, v = seq_parts(case, 0)
+    block = np.full(200, -1)
+    for b, (a, e) in enumerate(spans):
+        block[a:e] = b
+    i = np.arange(200)[:, None]
+    j = np.arange(200)[None, :]
+    vis = torch.from_numpy((j <= i) | ((block[:, None] == block[None, :]) & (block[:, None] >= 0)))
+    bias = alibi_bias(case, 0, sl) + mask_block(mask, case, 0, 0, ld)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q, k, v, attn_mask=bias.masked_fill(~vis, float("-inf")), scale=case.scale)
+    assert np.max(np.abs(got - ref.transpose(0, 1).numpy())) < 1e-10
