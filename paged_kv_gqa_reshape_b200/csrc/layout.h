@@ -28,7 +28,8 @@ struct SeqInfo {
 struct PlanHeader {
   int32_t num_prefill_tiles;   // entries in the prefill tile list
   int32_t total_decode_pages;  // 16-key pages over all single-query sequences
-  int32_t pad[62];
+  int32_t prefill_next;        // prefill work items handed out after the first round
+  int32_t pad[61];
 };
 
 struct WorkspaceLayout {

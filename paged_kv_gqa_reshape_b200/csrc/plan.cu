@@ -212,6 +212,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
     num_tiles = (int)min((long long)s_hist[kCostBuckets - 1], (long long)L.max_tiles);
     hdr->num_prefill_tiles = num_tiles;
     hdr->total_decode_pages = total_pages;
+    hdr->prefill_next = 0;
     if (s_err) atomicOr(err, s_err);
   }
 }

@@ -66,8 +66,9 @@ struct PrefillSmem {
   static constexpr int kRingOff = kQOff + 2 * kQBytes;
   static constexpr int kBarOff = kRingOff + kRing * kKVBytes;
   // barriers: q_full, q_empty, slot_full[kRing], slot_empty[kRing], s_full[2],
-  //           p_full[2], o_done[2]
-  static constexpr int kNumBars = 2 + 2 * kRing + 6;
+  //           p_full[2], o_done[2], item_full[kItemRing], item_empty[kItemRing]
+  static constexpr int kItemRing = 4;  // work-item indices in flight to the consumers
+  static constexpr int kNumBars = 2 + 2 * kRing + 6 + 2 * kItemRing;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 64;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B
@@ -133,8 +134,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = slot_empty + kRing;  // [2]: tile A, tile B
   uint64_t* p_full = s_full + 2;          // [2]
   uint64_t* o_done = p_full + 2;          // [2]
+  uint64_t* item_full = o_done + 2;       // [kItemRing]: index published
+  uint64_t* item_empty = item_full + SM::kItemRing;  // [kItemRing]: read by every consumer
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::kMiscOff + 4);
+  volatile int* s_item = reinterpret_cast<volatile int*>(smem + SM::kMiscOff + 8);  // [kItemRing]
 
   const uint32_t q_s = smem_u32(smem + SM::kQOff);
   const uint32_t ring_s = smem_u32(smem + SM::kRingOff);
@@ -146,6 +150,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int2* tiles = reinterpret_cast<const int2*>(ws + p.L.tiles);
   const int2* tile_n = reinterpret_cast<const int2*>(ws + p.L.tile_n);
   const int num_work = hdr->num_prefill_tiles * p.num_q_heads;
+  // Work distribution: the first item of a CTA is blockIdx.x; later ones are
+  // taken from a counter (sorted by descending cost, so the longest go first),
+  // so SMs that run faster take more items.  The producer publishes each item
+  // index in a small ring; the MMA thread and the softmax warps read it (-1:
+  // no more work).
+  int* next_item = const_cast<int*>(&hdr->prefill_next);
+  auto read_item = [&](int k, bool& ok) -> int {
+    const int slot = k % SM::kItemRing;
+    ok = ok && mbar_wait_bounded(item_full + slot, (uint32_t)((k / SM::kItemRing) & 1), abort_flag,
+                                 err);
+    return ok ? s_item[slot] : -1;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -158,6 +174,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(s_full + x, 1);
       mbar_init(p_full + x, 4 * 32);
       mbar_init(o_done + x, 1);
+    }
+    for (int i = 0; i < SM::kItemRing; ++i) {
+      mbar_init(item_full + i, 1);
+      mbar_init(item_empty + i, 1 + 8);  // the MMA thread and the 8 softmax warps
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -188,7 +208,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       // head-major q / cache swap two tensor-map coordinates (strided
       // instantiation only; the dense one keeps token-major order)
       const bool q_hnd = STRIDED && p.q_hnd != 0, kv_hnd = STRIDED && p.kv_hnd != 0;
-      for (int w = blockIdx.x; w < num_work && ok; w += gridDim.x) {
+      for (int k = 0; ok; ++k) {
+        int w = k == 0 ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(next_item, 1);
+        if (w >= num_work) w = -1;
+        const int slot = k % SM::kItemRing;
+        if (k >= SM::kItemRing)
+          ok = mbar_wait_bounded(item_empty + slot, (uint32_t)((k / SM::kItemRing - 1) & 1),
+                                 abort_flag, err);
+        if (!ok) break;
+        s_item[slot] = w;
+        mbar_arrive(item_full + slot);
+        if (w < 0) break;
         const Work wk = decode_work(w, tiles, tile_n, info, p.num_q_heads);
         if (wk.nmax == 0) continue;
         const int kvh = wk.head / p.group;
@@ -274,7 +304,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(o_done + x);
         ++pv_it[x];
       };
-      for (int w = blockIdx.x; w < num_work && ok; w += gridDim.x) {
+      for (int k = 0; ok; ++k) {
+        const int w = read_item(k, ok);
+        mbar_arrive(item_empty + k % SM::kItemRing);
+        if (w < 0) break;
         const Work wk = decode_work(w, tiles, tile_n, info, p.num_q_heads);
         if (wk.nmax == 0) continue;
         ok = mbar_wait_bounded(q_full, tcount & 1, abort_flag, err);
@@ -326,7 +359,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t o_col = tmem_o(x) + lane_base;
     int it = 0;  // S tiles of this query tile consumed so far (phase counter)
     bool ok = true;
-    for (int w = blockIdx.x; w < num_work && ok; w += gridDim.x) {
+    for (int k = 0; ok; ++k) {
+      const int w = read_item(k, ok);
+      ok = __all_sync(0xffffffffu, ok);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(item_empty + k % SM::kItemRing);
+      if (!ok || w < 0) break;
       const Work wk = decode_work(w, tiles, tile_n, info, p.num_q_heads);
       const int rows = wk.rows[x], n = wk.n[x];
       const int qrow = wk.row0 + x * BM + r;  // query index within the sequence
