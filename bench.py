@@ -42,8 +42,8 @@ WORKLOAD = ("decode_batch: 64 seqs x 1 query token, context U[256,4096], Hq 32 /
 # DRAM bytes (read + write) of one decode-kernel launch on the decode batch, from
 # one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), valid only
 # while the decode kernel's sources hash to the recorded value.
-DECODE_TRAFFIC = {"sources_sha256": "0a29665ba16ec5894d6e5a9094eed86b7fb554e4f0a3da803058f9effe231e27",
-                  "bytes_per_launch": 598869333}
+DECODE_TRAFFIC = {"sources_sha256": "232e848bf67035a6b26be84dd2272e9b7c8ba62e6d01b1931e99253fc906a3b7",
+                  "bytes_per_launch": 599628971}
 DECODE_SOURCES = ("decode.cu", "common.cuh", "layout.h")
 
 
@@ -653,18 +653,31 @@ def run_single_workload(args):
 def run_e2e(pa, case, args, dev, ws):
     """The same step through the public API with host-resident inputs/outputs."""
     names = ["q", "k_new", "v_new", "slot_mapping", "block_tables", "seq_lens", "query_start_loc"]
-    host = {n: getattr(case, n).cpu().pin_memory() for n in names}
-    devt = {n: torch.empty_like(getattr(case, n)) for n in names}
+    # the step's inputs packed in one pinned host buffer (each at a 256-byte
+    # offset) and copied with one transfer into one device buffer, whose
+    # typed views the library reads, as a serving loop stages its metadata
+    offs, off = {}, 0
+    for n in names:
+        t = getattr(case, n)
+        offs[n] = off
+        off += (t.numel() * t.element_size() + 255) // 256 * 256
+    host_buf = torch.empty(off, dtype=torch.uint8).pin_memory()
+    dev_buf = torch.empty(off, dtype=torch.uint8, device=dev)
+    devt = {}
+    for n in names:
+        t = getattr(case, n)
+        nbytes = t.numel() * t.element_size()
+        host_buf[offs[n]:offs[n] + nbytes].copy_(t.contiguous().view(torch.uint8).view(-1).cpu())
+        devt[n] = dev_buf[offs[n]:offs[n] + nbytes].view(t.dtype).view(t.shape)
     out_h = torch.empty(case.q.shape, dtype=case.q.dtype).pin_memory()
     out_d = torch.empty_like(case.q)
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    h2d = sum(getattr(case, n).numel() * getattr(case, n).element_size() for n in names)
     d2h = out_h.numel() * out_h.element_size()
     steps = max(1, min(args.steps, 500))
     mql, msl = case.max_query_len, case.max_seq_len  # host-side metadata, known before the step
 
     def step():
-        for n in names:
-            devt[n].copy_(host[n], non_blocking=True)
+        dev_buf.copy_(host_buf, non_blocking=True)
         pa.write_kv(devt["k_new"], devt["v_new"], devt["slot_mapping"], case.k_cache,
                     case.v_cache, workspace=ws)
         pa.attention_varlen(devt["q"], case.k_cache, case.v_cache, devt["block_tables"],
