@@ -95,6 +95,12 @@ typedef enum {
  *                error word receives PA_DEVERR_SLOT.
  * Two tokens naming the same slot is invalid input; the cache then holds one
  * of the candidate rows.  head_dim must be a multiple of 8.
+ * The kernel lets the next kernel in the stream start early when that one is
+ * launched with programmatic stream serialisation (the attention calls'
+ * decode kernel is, and waits for this grid before reading any input); an
+ * ordinary launch after it is not affected.  A successor from elsewhere
+ * launched that way must itself wait (griddepcontrol.wait) before reading
+ * the caches.
  */
 pa_status pa_write_kv(const void* k, const void* v, const int64_t* slot_mapping,
                       int64_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
