@@ -96,9 +96,25 @@ __global__ void __launch_bounds__(kBwdWarps * 32, kBwdBlocksPerSm)
   // phase A2, and each buffer takes the next item's rows once this lane has
   // used its own, so the next item's loads overlap this item's compute
 
+  // start an item's q, dO and weight rows towards L1 (one lane per 128-byte line)
+  auto prefetch_rows = [&](long long it) {
+    if (it >= total) return;
+    const int bb = (int)(it / p.num_kv_heads);
+    const int h0 = (int)(it - (long long)bb * p.num_kv_heads) * g;
+    for (int hl = sub; hl < g; hl += KPP) {
+      const size_t qrow = ((size_t)bb * p.num_q_heads + h0 + hl) * D;
+      if ((l & 7) == 0) {
+        prefetch_l1(p.q + qrow + l * 8);
+        prefetch_l1(p.dout + qrow + l * 8);
+      }
+      if (l == 0) prefetch_l1(p.weights + ((size_t)bb * p.num_q_heads + h0 + hl) * p.weights_len);
+    }
+  };
+
   long long item = (long long)blockIdx.x * (blockDim.x >> 5) + warp;
   int s1, n1;
   bounds(item, s1, n1);
+  prefetch_rows(item);
   copy_rows(sv, p.v, item, s1, n1);
   copy_rows(sk, p.k, item, s1, n1);
   for (; item < total; item += W) {
@@ -123,18 +139,13 @@ __global__ void __launch_bounds__(kBwdWarps * 32, kBwdBlocksPerSm)
       cp_async_wait<0>();
       copy_rows(sv, p.v, item + W, s1, n1);
       copy_rows(sk, p.k, item + W, s1, n1);
+      prefetch_rows(item + W);
       continue;
     }
     // the group's q, dO and weight rows are re-read per head and per key
-    // pass: start them towards L1 now (the K/V rows are already in flight)
-    for (int hl = sub; hl < g; hl += KPP) {
-      const size_t qrow = ((size_t)b * p.num_q_heads + head0 + hl) * D;
-      if ((l & 7) == 0) {  // one lane per 128-byte line
-        prefetch_l1(p.q + qrow + l * 8);
-        prefetch_l1(p.dout + qrow + l * 8);
-      }
-      if (l == 0) prefetch_l1(p.weights + ((size_t)b * p.num_q_heads + head0 + hl) * p.weights_len);
-    }
+    // pass: they depend only on the item, so the next item's rows are
+    // started towards L1 now (this item's were started one item ago)
+    prefetch_rows(item + W);
 
     auto run = [&](auto np_tag) {
       constexpr int NP = decltype(np_tag)::value;
