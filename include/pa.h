@@ -323,7 +323,9 @@ typedef struct pa_strides {
  * 16-byte aligned, entries finite or -inf; t is the packed query-token
  * index; mask_head_stride 0 shares one mask across heads; both strides are
  * multiples of 4; mask_len is the number of keys a mask row holds: a key at
- * or beyond it gets no mask value and raises PA_DEVERR_HINT.
+ * or beyond it gets no mask value and raises PA_DEVERR_HINT.  With any
+ * modifier on, scale must be > 0 (the kernels apply the modifiers to
+ * unscaled scores), else PA_ERR_INVALID_ARG.
  */
 typedef struct pa_score_mods {
   float softcap;

@@ -299,6 +299,7 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
   pa::ScoreMods mods{};
   rs = resolve_mods(score_mods, &mods);
   if (rs != PA_OK) return rs;
+  if (mods.any() && !(scale > 0.f)) return PA_ERR_INVALID_ARG;
   const WorkspaceLayout L =
       pa::make_layout(num_seqs, num_q_tokens, num_q_heads, num_kv_heads, head_dim);
   if (workspace_bytes < L.total) return PA_ERR_INVALID_ARG;

@@ -427,20 +427,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           // -inf below, so their mask values are not read.
           if (p.mods.softcap > 0.f) {
             const float a1 = p.scale / p.mods.softcap, capr = p.mods.softcap / p.scale;
+            const float ky = 2.f * kLog2e * a1;
+            const uint64_t ky2 = f2_pack(ky, ky), kk2 = f2_pack(2.f * capr, 2.f * capr),
+                           nk2 = f2_pack(-capr, -capr);
 #pragma unroll
-            for (int c = 0; c < BN; ++c)
-              sv[c] = __float_as_uint(capr * tanh_sfu(__uint_as_float(sv[c]) * a1));
+            for (int c = 0; c < BN; c += 2) {
+              const uint64_t y = f2_mul(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), ky2);
+              const uint64_t t = tanh2_scaled(y, kk2, nk2);
+              sv[c] = __float_as_uint(f2_lo(t));
+              sv[c + 1] = __float_as_uint(f2_hi(t));
+            }
           }
           if (slope != 0.f) {
             // + slope' (key0 - pos + c), slope' = slope / scale, on fp32 pairs
+            // The bias of pair c is carried in one of four running pairs
+            // (advanced by 8 keys per use) rather than rebuilt from c.
             const float sr = slope / p.scale;
-            const uint64_t step2 = f2_pack(sr, sr);
             const float b0 = sr * (float)(key0 - pos);
+            const uint64_t step8 = f2_pack(8.f * sr, 8.f * sr);
+            uint64_t bias[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              bias[i] = f2_pack(fmaf(sr, (float)(2 * i), b0), fmaf(sr, (float)(2 * i + 1), b0));
 #pragma unroll
             for (int c = 0; c < BN; c += 2) {
-              const uint64_t bias = f2_fma(step2, f2_pack((float)c, (float)(c + 1)), f2_pack(b0, b0));
-              const uint64_t v = f2_add(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
-                                        bias);
+              uint64_t& b = bias[(c / 2) % 4];
+              const uint64_t v = f2_add(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), b);
+              b = f2_add(b, step8);
               sv[c] = __float_as_uint(f2_lo(v));
               sv[c + 1] = __float_as_uint(f2_hi(v));
             }

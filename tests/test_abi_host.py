@@ -220,6 +220,10 @@ def test_varlen_mods_rejects_layouts_and_modifiers_before_launch():
     assert _mods_call(lib, None, M(0.0, None, 1 << 12, 0, 66, 64)) == 1        # row stride % 4
     assert _mods_call(lib, None, M(0.0, None, 1 << 12, 0, 64, 0)) == 1         # mask_len 0
     assert _mods_call(lib, None, M(0.0, None, None, 0, 0, 0), S=0) == 0       # empty batch
+    # a modifier with scale 0 (the kernels work in unscaled-score units)
+    assert _mods_call(lib, None, M(30.0, None, None, 0, 0, 0), scale=0.0) == 1
+    assert _mods_call(lib, None, M(0.0, 1 << 12, None, 0, 0, 0), scale=0.0) == 1
+    assert _mods_call(lib, None, M(0.0, None, 1 << 12, 0, 64, 64), scale=0.0) == 1
 
 
 def test_write_kv_strided_rejects_before_launch():
