@@ -57,27 +57,6 @@ constexpr int BN = kPrefillTileN;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows by > 2^8
 
-// k * tanh(x) on a packed fp32 pair, given y = 2 x log2(e), with one SFU
-// operation per element.  tanh x = sign(x) (2 r - 1) with r = 1 / w,
-// w = 1 + e^{-2|x|}; the exponential runs on the SFU, and since w lies in
-// [1, 2] the reciprocal needs no range reduction: the minimax quadratic for
-// 1/w on [1, 2] (relative error 1/99, coefficients 70/33, -48/33, 32/99)
-// followed by two Newton steps r <- r + r (1 - w r) gives r to ~1e-8 on the
-// FMA pipe.  Absolute error of tanh ~3e-7 (fp32 rounding); saturates
-// exactly (u = 0 for large |x|, so r = 1).  kk = (2k, 2k), nk = (-k, -k).
-__device__ __forceinline__ uint64_t tanh2_scaled(uint64_t y, uint64_t kk, uint64_t nk) {
-  constexpr float c0 = 70.f / 33.f, c1 = -48.f / 33.f, c2 = 32.f / 99.f;
-  const uint64_t m1 = f2_pack(-1.f, -1.f), one = f2_pack(1.f, 1.f);
-  const float u0 = fast_exp2(-fabsf(f2_lo(y))), u1 = fast_exp2(-fabsf(f2_hi(y)));
-  const uint64_t nw = f2_fma(f2_pack(u0, u1), m1, m1);  // -w
-  // c0 + c1 w + c2 w^2, in -w
-  uint64_t r = f2_fma(f2_fma(f2_pack(c2, c2), nw, f2_pack(-c1, -c1)), nw, f2_pack(c0, c0));
-#pragma unroll
-  for (int i = 0; i < 2; ++i) r = f2_fma(r, f2_fma(nw, r, one), r);
-  const uint64_t t = f2_fma(r, kk, nk);  // k (2 r - 1) = k tanh|x|
-  return t ^ (y & 0x8000000080000000ull);
-}
-
 template <int D>
 struct PrefillSmem {
   static constexpr int kQBytes = BM * D * 2;   // one 128-row Q tile
@@ -448,16 +427,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           // -inf below, so their mask values are not read.
           if (p.mods.softcap > 0.f) {
             const float a1 = p.scale / p.mods.softcap, capr = p.mods.softcap / p.scale;
-            const float ky = 2.f * kLog2e * a1;
-            const uint64_t ky2 = f2_pack(ky, ky), kk2 = f2_pack(2.f * capr, 2.f * capr),
-                           nk2 = f2_pack(-capr, -capr);
 #pragma unroll
-            for (int c = 0; c < BN; c += 2) {
-              const uint64_t y = f2_mul(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), ky2);
-              const uint64_t t = tanh2_scaled(y, kk2, nk2);
-              sv[c] = __float_as_uint(f2_lo(t));
-              sv[c + 1] = __float_as_uint(f2_hi(t));
-            }
+            for (int c = 0; c < BN; ++c)
+              sv[c] = __float_as_uint(capr * tanh_sfu(__uint_as_float(sv[c]) * a1));
           }
           if (slope != 0.f) {
             // + slope' (key0 - pos + c), slope' = slope / scale, on fp32 pairs
