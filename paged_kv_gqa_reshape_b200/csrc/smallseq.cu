@@ -39,6 +39,7 @@ struct SmallSeqItem {
   static constexpr int LPK = D / 8;        // lanes per key row
   static constexpr int KPP = 32 / LPK;     // keys per pass
   static constexpr int PASSES = 16 / KPP;  // passes for the 16-key maximum
+  static_assert(PASSES <= LPK, "one lane per pass in each key group");
   uint4 q;
   uint4 k[PASSES], v[PASSES];
   int n;  // keys of the entry (clamped)
@@ -184,15 +185,15 @@ __global__ void __launch_bounds__(256, 3) smallseq_kernel(SmallSeqParams p) {
       const float winv = sum > 0.f ? 1.f / sum : 0.f;
       uint16_t* wrow = p.weights + ((size_t)b * p.num_q_heads + h) * p.weights_len;
       if (cur.n > p.weights_len && lane == 0) raise_error(p.err, PA_DEVERR_HINT);
-      // lane t writes weight t (one coalesced row store): key t's weight is
-      // pass t / KPP of key group t % KPP, whose lanes all hold it
-      float wt = 0.f;
-      const int src = (lane % KPP) * LPK;
+      // lane t writes weight t (one coalesced row store).  Key t is pass
+      // t / KPP of key group t % KPP, whose lanes all hold its weight: lane
+      // pp of each group (PASSES <= LPK) offers its pass-pp weight, and one
+      // shuffle brings key t's to lane t (lanes past the last pass read 0).
+      float mine = 0.f;
 #pragma unroll
-      for (int pp = 0; pp < PASSES; ++pp) {
-        const float v = __shfl_sync(0xffffffffu, pwv[pp], src);
-        if (lane / KPP == pp) wt = v;
-      }
+      for (int pp = 0; pp < PASSES; ++pp)
+        if (l == pp) mine = pwv[pp];
+      const float wt = __shfl_sync(0xffffffffu, mine, (lane % KPP) * LPK + lane / KPP);
       for (int t = lane; t < p.weights_len; t += 32)
         wrow[t] = (t < cur.n && t == lane) ? ebits<H>(wt * winv) : (uint16_t)0;
     }
