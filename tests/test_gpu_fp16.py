@@ -79,3 +79,21 @@ def test_smallseq_fp16(d, hq, hkv):
                                 hkv, cpu.scale, 1)
     assert_attention_close(out, ref, what="smallseq fp16")
     assert pa.get_error(ws) == (0, 0)
+
+
+def test_fp16_prefill_and_decode_configs_full_size():
+    # the benchmark's fp16 legs: varlen_prefill on sampled rows, decode_batch
+    # on every row
+    pre = workloads.varlen_prefill(dtype=F16)
+    out, _, _, ws = run_varlen(case_to(pre, "cuda"))
+    assert pa.get_error(ws) == (0, 0)
+    qsl = pre.query_start_loc.tolist()
+    rows = sorted({qsl[s] + i for s in range(pre.num_seqs) for i in (0, 127, 128, 2047)
+                   if qsl[s] + i < qsl[s + 1]} | {qsl[s + 1] - 1 for s in range(pre.num_seqs)})
+    rows = np.array(rows, dtype=np.int64)
+    assert_attention_close(out, oracle_f16(pre, rows=rows), rows=rows,
+                           what="fp16 prefill full (sampled)")
+    dec = workloads.decode_batch(dtype=F16)
+    out, _, _, ws = run_varlen(case_to(dec, "cuda"))
+    assert pa.get_error(ws) == (0, 0)
+    assert_attention_close(out, oracle_f16(dec), what="fp16 decode full")

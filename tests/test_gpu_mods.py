@@ -254,3 +254,49 @@ def test_spans_with_modifiers():
         span_offsets=so.numpy(), spans=sp.numpy())
     assert_attention_close(out, ref, what="spans + modifiers")
     assert pa.get_error(ws) == (0, 0)
+
+
+# ---------------------------------------------------------------------------
+# the modifier workloads the benchmark times, at full size, on sampled rows
+# ---------------------------------------------------------------------------
+
+def sampled_rows(case):
+    """Tile edges, the middle and the last two rows of every sequence."""
+    qsl = case.query_start_loc.tolist()
+    rows = set()
+    for s in range(case.num_seqs):
+        for i in (0, 1, 127, 128, 129, 1000, 2047):
+            if qsl[s] + i < qsl[s + 1]:
+                rows.add(qsl[s] + i)
+        rows.update((qsl[s + 1] - 1, qsl[s + 1] - 2))
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def test_alibi_softcap_prefill_config_full_size_sampled_rows():
+    # varlen_prefill (4 causal sequences up to 8192 tokens, Hq 32 / Hkv 8,
+    # D 128) with the geometric slopes and the TANH30 soft-cap
+    cpu = workloads.varlen_prefill()
+    sl = slopes_for(cpu.num_q_heads)
+    out, ws = run_mods(case_to(cpu, "cuda"), softcap=30.0, alibi_slopes=sl.cuda())
+    assert pa.get_error(ws) == (0, 0)
+    rows = sampled_rows(cpu)
+    ref = oracle.attention_varlen_mods(
+        workloads.bf16_bits(cpu.q), workloads.bf16_bits(cpu.k_logical),
+        workloads.bf16_bits(cpu.v_logical), cpu.kv_offsets.numpy(), cpu.seq_lens.numpy(),
+        cpu.query_start_loc.numpy(), cpu.num_kv_heads, cpu.scale, cpu.causal, 0,
+        softcap=30.0, alibi_slopes=sl.numpy(), rows=rows)
+    assert_attention_close(out, ref, rows=rows, what="prefill + ALiBi + TANH30 full (sampled)")
+
+
+def test_hnd_mask_decode_config_full_size():
+    # decode_batch (64 sequences, context 256-4096) over head-major caches
+    # with one additive mask shared by all heads, every row checked
+    cpu = workloads.decode_batch()
+    dev = case_to(cpu, "cuda")
+    import dataclasses
+    hnd = dataclasses.replace(dev, k_cache=hnd_cache(dev.k_cache), v_cache=hnd_cache(dev.v_cache))
+    mlen = (cpu.max_seq_len + 3) // 4 * 4
+    mask = torch.randn(cpu.num_q_tokens, mlen, generator=workloads._gen(1008, "cpu"))
+    out, ws = run_mods(hnd, mask=mask.cuda())
+    assert pa.get_error(ws) == (0, 0)
+    assert_attention_close(out, oracle_mods(cpu, mask=mask), what="decode HND + mask full")

@@ -259,3 +259,24 @@ def test_backward_full_size_sampled():
     for got, ref, extra, name in ((dq[pick], rq, eq, "dq"), (gk, rk, ek, "dk"),
                                   (gv, rv, ev, "dv")):
         assert_chain_close(got, ref, extra, UNIT[BF16], name)
+
+
+def test_weights_full_size_sampled():
+    # the benchmark's forward with the weights output (batch 30720, width 16):
+    # sampled entries against the oracle on their sub-batch, and zeros past
+    # every entry's keys over the whole output
+    ss = workloads.smallseq_batch(device="cuda")
+    out, w, ws = gpu_forward(ss, 16)
+    assert pa.get_error(ws) == (0, 0)
+    cu = ss.cu_seqlens_kv.cpu()
+    lens = (cu[1:] - cu[:-1]).to("cuda")
+    past = torch.arange(16, device="cuda")[None, None, :] >= lens[:, None, None]
+    assert torch.count_nonzero(w.masked_select(past)) == 0
+    cu = cu.tolist()
+    rng = np.random.default_rng(94)
+    pick = sorted(set(rng.integers(0, ss.batch, size=300).tolist()) | {0, ss.batch - 1})
+    kk = torch.cat([ss.k[cu[b]:cu[b + 1]] for b in pick]).cpu()
+    sub_cu = np.concatenate([[0], np.cumsum([cu[b + 1] - cu[b] for b in pick])]).astype(np.int32)
+    ref = oracle.smallseq_weights(bits(ss.q[pick]), bits(kk), sub_cu, ss.num_kv_heads, ss.scale,
+                                  16, dtype=0)
+    assert_rel_close(w[pick], ref, UNIT[BF16], 1e-5, "weights full (sampled)")
