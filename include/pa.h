@@ -321,7 +321,9 @@ typedef struct pa_strides {
  * keys enter the softmax, and a row whose visible scores are all -inf gives
  * zeros.  alibi_slopes: NULL or [num_q_heads] fp32.  mask: NULL or fp32,
  * 16-byte aligned, entries finite or -inf; t is the packed query-token
- * index; mask_head_stride 0 shares one mask across heads; both strides are
+ * index; the buffer must hold every (h, t) row a call addresses (the
+ * library cannot check its extent, only the row length below);
+ * mask_head_stride 0 shares one mask across heads; both strides are
  * multiples of 4; mask_len is the number of keys a mask row holds: a key at
  * or beyond it gets no mask value and raises PA_DEVERR_HINT.  With any
  * modifier on, scale must be > 0 (the kernels apply the modifiers to

@@ -140,9 +140,9 @@ def version() -> str:
     return load().pa_version().decode()
 
 
-def _stream(stream) -> Optional[int]:
+def _stream(stream, device=None) -> Optional[int]:
     if stream is None:
-        return torch.cuda.current_stream().cuda_stream
+        return torch.cuda.current_stream(device).cuda_stream
     if isinstance(stream, torch.cuda.Stream):
         return stream.cuda_stream
     return int(stream)
@@ -159,6 +159,13 @@ def _check(t: torch.Tensor, name: str, dtype, ndim: Optional[int] = None):
         raise ValueError(f"{name} must be contiguous")
     if ndim is not None and t.dim() != ndim:
         raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+
+
+def _same_device(device, **tensors):
+    """Every tensor argument of a call lives on the device its kernels run on."""
+    for name, t in tensors.items():
+        if t is not None and t.device != device:
+            raise ValueError(f"{name} is on {t.device}, the call's tensors on {device}")
 
 
 def _raise(status: int, where: str):
@@ -260,22 +267,30 @@ def write_kv(k, v, slot_mapping, k_cache, v_cache, workspace=None, stream=None):
     nb, bs, hkv_c, d_c = k_cache.shape
     if hkv_c != hkv or d_c != d:
         raise ValueError("cache shape does not match k/v")
+    dev = k.device
+    _same_device(dev, v=v, slot_mapping=slot_mapping, k_cache=k_cache, v_cache=v_cache,
+                 workspace=workspace)
     ws = workspace.data_ptr() if workspace is not None else None
-    if _dense_rows(cstr, hkv, d):
-        st = load().pa_write_kv_ex(k.data_ptr(), v.data_ptr(), slot_mapping.data_ptr(), t, hkv,
-                                   d, k_cache.data_ptr(), v_cache.data_ptr(), nb, bs, cstr[0],
-                                   _DTYPES[dt], ws, _stream(stream))
-        _raise(st, "pa_write_kv_ex")
-        return
-    strides = _Strides(0, 0, 0, 0, *cstr)
-    st = load().pa_write_kv_strided(k.data_ptr(), v.data_ptr(), slot_mapping.data_ptr(), t, hkv,
-                                    d, k_cache.data_ptr(), v_cache.data_ptr(), nb, bs,
-                                    ctypes.byref(strides), _DTYPES[dt], ws, _stream(stream))
+    with torch.cuda.device(dev):
+        if _dense_rows(cstr, hkv, d):
+            st = load().pa_write_kv_ex(k.data_ptr(), v.data_ptr(), slot_mapping.data_ptr(), t,
+                                       hkv, d, k_cache.data_ptr(), v_cache.data_ptr(), nb, bs,
+                                       cstr[0], _DTYPES[dt], ws, _stream(stream, dev))
+            _raise(st, "pa_write_kv_ex")
+            return
+        strides = _Strides(0, 0, 0, 0, *cstr)
+        st = load().pa_write_kv_strided(k.data_ptr(), v.data_ptr(), slot_mapping.data_ptr(), t,
+                                        hkv, d, k_cache.data_ptr(), v_cache.data_ptr(), nb, bs,
+                                        ctypes.byref(strides), _DTYPES[dt], ws,
+                                        _stream(stream, dev))
     _raise(st, "pa_write_kv_strided")
 
 
-def _score_mods(softcap, alibi_slopes, mask, hq):
-    """pa_score_mods for the call, or None when every modifier is off."""
+def _score_mods(softcap, alibi_slopes, mask, hq, t, device):
+    """pa_score_mods for the call, or None when every modifier is off.  The
+    mask must hold a row for each of the call's t query tokens (and each
+    query head, if 3-D): the library reads those rows and checks only their
+    length."""
     if not softcap and alibi_slopes is None and mask is None:
         return None
     m = _ScoreMods(float(softcap or 0.0), None, None, 0, 0, 0)
@@ -287,10 +302,14 @@ def _score_mods(softcap, alibi_slopes, mask, hq):
     if mask is not None:
         if not isinstance(mask, torch.Tensor) or mask.dtype != torch.float32 or not mask.is_cuda:
             raise TypeError("mask must be a float32 CUDA tensor")
+        if mask.device != device:
+            raise ValueError("mask must be on q's device")
         if mask.dim() not in (2, 3) or mask.stride(-1) != 1:
             raise ValueError("mask must be [T, L] or [Hq, T, L] with L contiguous")
         if mask.dim() == 3 and mask.shape[0] != hq:
             raise ValueError("a 3-D mask must be [num_q_heads, T, L]")
+        if mask.shape[-2] < t:
+            raise ValueError("the mask needs a row for every query token")
         m.mask = mask.data_ptr()
         m.mask_token_stride = mask.stride(-2)
         m.mask_head_stride = mask.stride(0) if mask.dim() == 3 else 0
@@ -329,27 +348,33 @@ def _varlen_ex(q, k_cache, v_cache, block_tables, seq_lens, query_start_loc, num
     mb = block_tables.shape[1]
     mql = t if max_query_len is None else int(max_query_len)
     msl = mb * bs if max_seq_len is None else int(max_seq_len)
+    dev = q.device
+    _same_device(dev, k_cache=k_cache, v_cache=v_cache, block_tables=block_tables,
+                 seq_lens=seq_lens, query_start_loc=query_start_loc, out=out,
+                 span_offsets=span_offsets, spans=spans, workspace=workspace,
+                 alibi_slopes=alibi_slopes, mask=mask)
     if workspace is None:
-        workspace = varlen_workspace(s, t, hq, hkv, d, device=q.device)
-    mods = _score_mods(softcap, alibi_slopes, mask, hq)
+        workspace = varlen_workspace(s, t, hq, hkv, d, device=dev)
+    mods = _score_mods(softcap, alibi_slopes, mask, hq, t, dev)
     dense = qstr == (hq * d, d) and ostr == (hq * d, d) and _dense_rows(cstr, hkv, d)
-    if dense and mods is None:
-        st = load().pa_attention_varlen_ex(
+    with torch.cuda.device(dev):
+        if dense and mods is None:
+            st = load().pa_attention_varlen_ex(
+                q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(),
+                mb, seq_lens.data_ptr(), query_start_loc.data_ptr(), s, t, hq, hkv, d, bs, nb,
+                cstr[0], _DTYPES[dt], mql, msl, float(scale), int(bool(causal)), so_ptr, sp_ptr,
+                n_spans, out.data_ptr(), workspace.data_ptr(),
+                workspace.numel() * workspace.element_size(), _stream(stream, dev))
+            _raise(st, what)
+            return out
+        strides = _Strides(*qstr, *ostr, *cstr)
+        st = load().pa_attention_varlen_mods(
             q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(), mb,
-            seq_lens.data_ptr(), query_start_loc.data_ptr(), s, t, hq, hkv, d, bs, nb, cstr[0],
+            seq_lens.data_ptr(), query_start_loc.data_ptr(), s, t, hq, hkv, d, bs, nb,
             _DTYPES[dt], mql, msl, float(scale), int(bool(causal)), so_ptr, sp_ptr, n_spans,
+            ctypes.byref(strides), ctypes.byref(mods) if mods is not None else None,
             out.data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-            _stream(stream))
-        _raise(st, what)
-        return out
-    strides = _Strides(*qstr, *ostr, *cstr)
-    st = load().pa_attention_varlen_mods(
-        q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(), mb,
-        seq_lens.data_ptr(), query_start_loc.data_ptr(), s, t, hq, hkv, d, bs, nb, _DTYPES[dt],
-        mql, msl, float(scale), int(bool(causal)), so_ptr, sp_ptr, n_spans,
-        ctypes.byref(strides), ctypes.byref(mods) if mods is not None else None,
-        out.data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-        _stream(stream))
+            _stream(stream, dev))
     _raise(st, "pa_attention_varlen_mods")
     return out
 
@@ -425,10 +450,14 @@ def attention_varlen_static(q, k_cache, v_cache, block_tables, seq_lens, query_s
     mb = block_tables.shape[1]
     mql = t if max_query_len is None else int(max_query_len)
     msl = mb * bs if max_seq_len is None else int(max_seq_len)
-    st = load().pa_attention_varlen_static(
-        q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(), mb,
-        seq_lens.data_ptr(), query_start_loc.data_ptr(), s, t, hq, hkv, d, bs, nb, mql, msl,
-        float(scale), int(bool(causal)), out.data_ptr(), _stream(stream))
+    dev = q.device
+    _same_device(dev, k_cache=k_cache, v_cache=v_cache, block_tables=block_tables,
+                 seq_lens=seq_lens, query_start_loc=query_start_loc, out=out)
+    with torch.cuda.device(dev):
+        st = load().pa_attention_varlen_static(
+            q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(), mb,
+            seq_lens.data_ptr(), query_start_loc.data_ptr(), s, t, hq, hkv, d, bs, nb, mql, msl,
+            float(scale), int(bool(causal)), out.data_ptr(), _stream(stream, dev))
     _raise(st, "pa_attention_varlen_static")
     return out
 
@@ -453,11 +482,15 @@ def attention_smallseq(q, k, v, cu_seqlens_kv, scale, out, max_seqlen_kv=16, wor
         if weights.shape[:2] != (b, hq):
             raise ValueError("weights must be [batch, num_q_heads, W]")
         wp, wlen = weights.data_ptr(), weights.shape[2]
+    dev = q.device
+    _same_device(dev, k=k, v=v, cu_seqlens_kv=cu_seqlens_kv, out=out, weights=weights,
+                 workspace=workspace)
     ws = workspace.data_ptr() if workspace is not None else None
-    st = load().pa_attention_smallseq_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                         cu_seqlens_kv.data_ptr(), b, hq, hkv, d,
-                                         int(max_seqlen_kv), float(scale), _DTYPES[dt],
-                                         out.data_ptr(), wp, wlen, ws, _stream(stream))
+    with torch.cuda.device(dev):
+        st = load().pa_attention_smallseq_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                             cu_seqlens_kv.data_ptr(), b, hq, hkv, d,
+                                             int(max_seqlen_kv), float(scale), _DTYPES[dt],
+                                             out.data_ptr(), wp, wlen, ws, _stream(stream, dev))
     _raise(st, "pa_attention_smallseq_ex")
     return out
 
@@ -476,12 +509,16 @@ def attention_smallseq_bwd(q, k, v, dout, weights, cu_seqlens_kv, scale, dq, dk,
             or dout.shape != q.shape or dq.shape != q.shape or weights.shape[:2] != (b, hq)
             or cu_seqlens_kv.shape[0] != b + 1):
         raise ValueError("inconsistent small-seq backward shapes")
+    dev = q.device
+    _same_device(dev, k=k, v=v, dout=dout, weights=weights, cu_seqlens_kv=cu_seqlens_kv, dq=dq,
+                 dk=dk, dv=dv, workspace=workspace)
     ws = workspace.data_ptr() if workspace is not None else None
-    st = load().pa_attention_smallseq_bwd(
-        q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), weights.data_ptr(),
-        weights.shape[2], cu_seqlens_kv.data_ptr(), b, hq, hkv, d, int(max_seqlen_kv),
-        float(scale), _DTYPES[dt], dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws,
-        _stream(stream))
+    with torch.cuda.device(dev):
+        st = load().pa_attention_smallseq_bwd(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), weights.data_ptr(),
+            weights.shape[2], cu_seqlens_kv.data_ptr(), b, hq, hkv, d, int(max_seqlen_kv),
+            float(scale), _DTYPES[dt], dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws,
+            _stream(stream, dev))
     _raise(st, "pa_attention_smallseq_bwd")
     return dq, dk, dv
 
@@ -489,5 +526,7 @@ def attention_smallseq_bwd(q, k, v, dout, weights, cu_seqlens_kv, scale, dq, dk,
 def get_error(workspace, stream=None):
     """Synchronise, read and clear the workspace's device error word: (status, bits)."""
     bits = ctypes.c_uint32(0)
-    st = load().pa_get_error(workspace.data_ptr(), _stream(stream), ctypes.byref(bits))
+    with torch.cuda.device(workspace.device):
+        st = load().pa_get_error(workspace.data_ptr(), _stream(stream, workspace.device),
+                                 ctypes.byref(bits))
     return int(st), int(bits.value)
