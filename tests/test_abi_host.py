@@ -168,6 +168,14 @@ def test_python_binding_rejects_cpu_and_wrong_dtypes():
         pa.write_kv(q.float(), q, torch.zeros(4, dtype=torch.int64), kc, kc)
 
 
+def test_python_binding_device_agreement():
+    # every tensor of a call must sit on the device its kernels run on
+    a, b = torch.zeros(1), torch.zeros(1, device="meta")
+    pa._same_device(torch.device("cpu"), x=a, y=None)
+    with pytest.raises(ValueError, match="y is on meta"):
+        pa._same_device(torch.device("cpu"), x=a, y=b)
+
+
 def test_struct_layouts_match_the_header(tmp_path):
     # the C structs of include/pa.h, laid out by the C compiler, against the
     # ctypes mirrors the binding passes by pointer
