@@ -1,7 +1,7 @@
 /*
  * pa.h — C ABI of the B200 (sm_100a) paged KV attention library (libpa.so).
  *
- * Three operations, all asynchronous on the caller's CUDA stream:
+ * Operations, all asynchronous on the caller's CUDA stream:
  *
  *   pa_write_kv            scatter this step's K/V rows into a block-paged cache
  *   pa_attention_varlen    softmax attention of packed variable-length queries
@@ -16,7 +16,9 @@
  * Conventions shared by every call
  * --------------------------------
  *  - Element type: bfloat16 for every Q/K/V/cache/output tensor (passed as
- *    void*, 2 bytes per element).  Index tensors are int32 unless stated.
+ *    void*, 2 bytes per element), or fp16 where a call takes a pa_dtype (the
+ *    _ex, _strided, _mods and small-seq _bwd forms); one type per call.
+ *    Index tensors are int32 unless stated.
  *  - Layout (every entry point but the _mods / _strided ones, which take
  *    pa_strides): token-major ("NHD"), dense, innermost dimension last:
  *      q, out           [num_tokens, num_q_heads, head_dim]
