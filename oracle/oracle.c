@@ -308,8 +308,13 @@ static int varlen_driver(const uint16_t *q, const uint16_t *k_base,
 #pragma omp parallel
     {
         double *scratch = (double *)malloc(sizeof(double) * (size_t)max_len);
+        /* one task per (query token, query head): rows are independent, and
+           so are the heads of a row, so a single decode row still spreads
+           over every thread */
 #pragma omp for schedule(dynamic, 1)
-        for (int64_t r = 0; r < todo; ++r) {
+        for (int64_t task = 0; task < todo * num_q_heads; ++task) {
+            int64_t r = task / num_q_heads;
+            int h = (int)(task % num_q_heads);
             int64_t t = rows ? rows[r] : r;
             int s = 0;
             while (s < num_seqs && query_start_loc[s + 1] <= t) ++s;
@@ -323,40 +328,38 @@ static int varlen_driver(const uint16_t *q, const uint16_t *k_base,
                 n_vis = visible_keys_spans((len_kv - len_q) + i, len_kv,
                                            spans + 2 * a, b > a ? b - a : 0);
             }
-            for (int h = 0; h < num_q_heads; ++h) {
-                kv_view kview = {0}, vview = {0};
-                kview.num_kv_heads = vview.num_kv_heads = num_kv_heads;
-                kview.head_dim = vview.head_dim = head_dim;
-                kview.kv_head = vview.kv_head = h / group;
-                kview.widen = vview.widen = widen;
-                kview.base = k_base;
-                vview.base = v_base;
-                if (block_tables) {
-                    const int32_t *tab = block_tables + (int64_t)s * max_blocks_per_seq;
-                    kview.table = vview.table = tab;
-                    kview.block_size = vview.block_size = block_size;
-                    kview.num_blocks = vview.num_blocks = num_blocks;
-                } else {
-                    kview.first_row = vview.first_row = kv_offsets[s];
-                }
-                const uint16_t *qr = q + (t * num_q_heads + h) * (int64_t)head_dim;
-                double *o = out + (t * num_q_heads + h) * (int64_t)head_dim;
-                row_mods rm, *rmp = NULL;
-                if (sm) {
-                    rm.softcap = sm->softcap;
-                    rm.has_alibi = sm->alibi_slopes != NULL;
-                    rm.slope = sm->alibi_slopes ? (double)sm->alibi_slopes[h] : 0.0;
-                    rm.pos = (len_kv - len_q) + i;
-                    rm.mask_row = sm->mask ? sm->mask + h * sm->mask_head_stride +
-                                                 t * sm->mask_token_stride
-                                           : NULL;
-                    rmp = &rm;
-                }
-                if (attention_row(qr, &kview, &vview, n_vis, head_dim, scale, rmp, o,
-                                  NULL, scratch) != 0) {
+            kv_view kview = {0}, vview = {0};
+            kview.num_kv_heads = vview.num_kv_heads = num_kv_heads;
+            kview.head_dim = vview.head_dim = head_dim;
+            kview.kv_head = vview.kv_head = h / group;
+            kview.widen = vview.widen = widen;
+            kview.base = k_base;
+            vview.base = v_base;
+            if (block_tables) {
+                const int32_t *tab = block_tables + (int64_t)s * max_blocks_per_seq;
+                kview.table = vview.table = tab;
+                kview.block_size = vview.block_size = block_size;
+                kview.num_blocks = vview.num_blocks = num_blocks;
+            } else {
+                kview.first_row = vview.first_row = kv_offsets[s];
+            }
+            const uint16_t *qr = q + (t * num_q_heads + h) * (int64_t)head_dim;
+            double *o = out + (t * num_q_heads + h) * (int64_t)head_dim;
+            row_mods rm, *rmp = NULL;
+            if (sm) {
+                rm.softcap = sm->softcap;
+                rm.has_alibi = sm->alibi_slopes != NULL;
+                rm.slope = sm->alibi_slopes ? (double)sm->alibi_slopes[h] : 0.0;
+                rm.pos = (len_kv - len_q) + i;
+                rm.mask_row = sm->mask ? sm->mask + h * sm->mask_head_stride +
+                                             t * sm->mask_token_stride
+                                       : NULL;
+                rmp = &rm;
+            }
+            if (attention_row(qr, &kview, &vview, n_vis, head_dim, scale, rmp, o,
+                              NULL, scratch) != 0) {
 #pragma omp atomic write
-                    status = -2;
-                }
+                status = -2;
             }
         }
         free(scratch);

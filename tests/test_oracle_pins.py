@@ -385,3 +385,39 @@ def test_smallseq_equals_varlen_with_one_query():
         v = case.v[cu[b]:cu[b] + n].double().repeat_interleave(2, dim=1).transpose(0, 1)
         o = torch.nn.functional.scaled_dot_product_attention(q, k, v, scale=case.scale)
         assert np.allclose(out[b], o.transpose(0, 1)[0].numpy(), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_scale_zero_gives_mean_of_visible_values(causal):
+    """Closed form (pin i with every score equal): at scale 0 each visible key
+    has weight 1/|V_i|, so the output is the plain mean of the visible V rows.
+    Visible set of query i of a sequence with Lq queries over Lkv keys: all
+    Lkv keys, or with causality the first Lkv - Lq + i + 1 (vllm-omni PR
+    #9244, kernel-semantics review)."""
+    case = workloads.build_varlen_case("pin", [9, 30, 1, 17], [9, 4, 1, 17], 6, 3, 64, causal,
+                                       seed=31, scale=0.0)
+    out = run_logical(case)
+    qsl = case.query_start_loc.tolist()
+    g = case.num_q_heads // case.num_kv_heads
+    for s in range(case.num_seqs):
+        lkv = int(case.seq_lens[s])
+        lq = qsl[s + 1] - qsl[s]
+        vals = case.v_logical[int(case.kv_offsets[s]):int(case.kv_offsets[s]) + lkv].double()
+        for i in range(lq):
+            n = (lkv - lq + i + 1) if causal else lkv
+            mean = vals[:n].mean(dim=0).repeat_interleave(g, dim=0).numpy()   # [Hq, D]
+            assert np.allclose(out[qsl[s] + i], mean, rtol=0, atol=1e-12)
+
+
+def test_smallseq_scale_zero_gives_mean_of_values():
+    case = workloads.build_smallseq_case("pin", [3, 0, 16, 1], 4, 2, 64, seed=12, scale=0.0)
+    out = oracle.attention_smallseq(workloads.bf16_bits(case.q), workloads.bf16_bits(case.k),
+                                    workloads.bf16_bits(case.v), case.cu_seqlens_kv.numpy(),
+                                    2, 0.0)
+    cu = case.cu_seqlens_kv.tolist()
+    for b in range(case.batch):
+        if cu[b + 1] == cu[b]:
+            assert np.all(out[b] == 0.0)
+            continue
+        mean = case.v[cu[b]:cu[b + 1]].double().mean(dim=0).repeat_interleave(2, dim=0)
+        assert np.allclose(out[b], mean.numpy(), rtol=0, atol=1e-12)
