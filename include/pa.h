@@ -28,7 +28,10 @@
  *  - The caller owns every buffer, including the workspace.  The library
  *    allocates no device memory and keeps no state between calls beyond a
  *    per-device table of attributes (SM count) and lazily-resolved driver
- *    entry points.
+ *    entry points, with one exception: the PA_STATIC_SCRATCH_BYTES device
+ *    array behind pa_attention_varlen_static, which every GPU that loads the
+ *    library holds, and which carries that entry point's scratch (its
+ *    split-KV arrival counters among it) from one call to the next.
  *  - `stream` is a cudaStream_t passed as void*; NULL means the legacy default
  *    stream.  No call synchronises except pa_get_error.
  *  - `out` must not alias any input.
@@ -112,9 +115,12 @@ pa_status pa_write_kv(const void* k, const void* v, const int64_t* slot_mapping,
 /*
  * pa_attention_varlen_workspace_size — bytes of workspace pa_attention_varlen
  * needs for these sizes (a function of the arguments only).  The workspace
- * must be zero-initialised once before its first use (the error word must
- * start at zero); afterwards it can be reused by consecutive calls on the
- * same stream without clearing.
+ * must be zero-initialised once before its first use (the error word and the
+ * split-KV arrival counters must start at zero); afterwards it can be reused
+ * without clearing by consecutive calls on the same stream, whatever their
+ * sizes (as long as it is large enough for each): the counters sit at a fixed
+ * offset in a region used for nothing else, and every call leaves them at
+ * zero.
  */
 size_t pa_attention_varlen_workspace_size(int32_t num_seqs, int64_t num_q_tokens,
                                           int32_t num_q_heads, int32_t num_kv_heads,
@@ -272,9 +278,15 @@ pa_status pa_attention_varlen_ex(const void* q, const void* k_cache, const void*
  *    PA_STATIC_SCRATCH_BYTES return PA_ERR_UNSUPPORTED before any launch.
  *  - The first call on a device looks up the array's device address with
  *    that device current; make it before any stream capture.
- *  - All calls share the array (it keeps the last call's contents; each call
- *    rebuilds what it needs).  Calls whose executions overlap on the GPU race
- *    on it: issue them on one stream, one host thread at a time.
+ *  - All calls share the array, which keeps the last call's contents.  Each
+ *    call rebuilds its plan lists and partial results; the split-KV arrival
+ *    counters, the one part that must start at zero, sit in a region used for
+ *    nothing else, zero when the module loads and returned to zero by every
+ *    call (the merge that uses a counter resets it; the plan kernel, when it
+ *    runs, zeroes them first).  Calls whose executions overlap on the GPU
+ *    race on the array: issue them on one stream, one host thread at a time.
+ *  - Bad arguments are reported as pa_attention_varlen reports them, before
+ *    the size limit below is applied and before any CUDA call.
  *  - Device-side index errors are handled as in pa_attention_varlen but
  *    cannot be read back (there is no caller workspace for pa_get_error).
  */
@@ -457,6 +469,21 @@ const char* pa_status_string(pa_status status);
 
 /* Library version string, e.g. "pa 0.1 sm_100a". */
 const char* pa_version(void);
+
+/*
+ * pa_set_wait_limit_ns — a test hook for the failure path of the tensor-core
+ * prefill (an addition of this library: the pages it follows have no
+ * counterpart).  Every wait of that kernel on one of its own pipeline
+ * barriers is bounded in wall time; after the limit it raises
+ * PA_DEVERR_TIMEOUT in the workspace's error word, lets the copies and MMAs
+ * it already issued land, releases its tensor memory and exits (its rows are
+ * left unwritten), so a lost arrival never hangs the GPU.  The default limit,
+ * one second, is far beyond any legitimate wait.  This call sets the limit
+ * for prefill launches made from now on, process-wide; ns = 0 restores the
+ * default.  A short limit makes ordinary waits give up, which is how a test
+ * reaches the timeout path; production code has no reason to call it.
+ */
+void pa_set_wait_limit_ns(uint64_t ns);
 
 #ifdef __cplusplus
 }

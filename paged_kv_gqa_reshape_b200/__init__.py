@@ -29,13 +29,16 @@ __all__ = [
     "attention_smallseq_bwd",
     "attention_varlen_static", "attention_varlen_spans", "STATIC_SCRATCH_BYTES",
     "varlen_workspace_size", "varlen_workspace", "error_workspace", "get_error",
-    "status_string", "version", "EXPORTED_SYMBOLS",
+    "status_string", "version", "set_wait_limit_ns", "EXPORTED_SYMBOLS", "PA_OK", "PA_ERR_INVALID_ARG",
+    "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA", "PA_ERR_DEVICE_INDEX", "PA_ERR_TIMEOUT",
     "DEVERR_SLOT", "DEVERR_BLOCK", "DEVERR_LENGTHS", "DEVERR_QLEN", "DEVERR_HINT",
     "DEVERR_TIMEOUT", "DEVERR_SPANS", "ERROR_WORD_BYTES", "DTYPE_BF16", "DTYPE_FP16",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-PA_OK = 0
+PA_OK = 0  # pa_status values of include/pa.h
+PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA = 1, 2, 3
+PA_ERR_DEVICE_INDEX, PA_ERR_TIMEOUT = 4, 5
 DEVERR_SLOT, DEVERR_BLOCK, DEVERR_LENGTHS = 0x1, 0x2, 0x4
 DEVERR_QLEN, DEVERR_HINT, DEVERR_TIMEOUT = 0x8, 0x10, 0x20
 DEVERR_SPANS = 0x40
@@ -47,7 +50,7 @@ EXPORTED_SYMBOLS = (
     "pa_attention_smallseq", "pa_get_error", "pa_status_string", "pa_version",
     "pa_attention_varlen_static", "pa_attention_varlen_spans", "pa_write_kv_ex",
     "pa_attention_varlen_ex", "pa_attention_smallseq_ex", "pa_attention_smallseq_bwd",
-    "pa_write_kv_strided", "pa_attention_varlen_mods",
+    "pa_write_kv_strided", "pa_attention_varlen_mods", "pa_set_wait_limit_ns",
 )
 DTYPE_BF16, DTYPE_FP16 = 0, 1
 
@@ -128,6 +131,8 @@ def load(build_if_missing: bool = True):
         lib.pa_status_string.argtypes = [ctypes.c_int]
         lib.pa_version.restype = ctypes.c_char_p
         lib.pa_version.argtypes = []
+        lib.pa_set_wait_limit_ns.restype = None
+        lib.pa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         _lib = lib
     return _lib
 
@@ -138,6 +143,14 @@ def status_string(status: int) -> str:
 
 def version() -> str:
     return load().pa_version().decode()
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Test hook: bound every pipeline-barrier wait of prefill launches made
+    from now on to `ns` nanoseconds (0 restores the 1 s default).  A short
+    limit makes ordinary waits give up, raising DEVERR_TIMEOUT; only tests of
+    that failure path should call this."""
+    load().pa_set_wait_limit_ns(int(ns))
 
 
 def _stream(stream, device=None) -> Optional[int]:

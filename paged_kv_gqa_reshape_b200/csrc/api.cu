@@ -4,7 +4,9 @@
 // written (the reject-before-write rule of TensorRT-LLM PR "CSA2 Vanilla
 // sparse attention", description).  The library allocates no device memory;
 // its only state is a per-device SM count and the lazily resolved driver
-// entry point used to encode TMA tensor maps.
+// entry point used to encode TMA tensor maps — apart from the fixed device
+// array of pa_attention_varlen_static (api_static.cu), which every GPU that
+// loads the library holds and which keeps that entry point's scratch.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -13,6 +15,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/pa.h"
@@ -48,6 +51,10 @@ bool log_enabled() {
   }
   return v == 1;
 }
+
+// Bound of the prefill kernel's mbarrier waits for launches from now on
+// (0: the kernel's 1 s default); set only through pa_set_wait_limit_ns.
+std::atomic<unsigned long long> g_wait_limit_ns{0};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -196,6 +203,8 @@ const char* pa_status_string(pa_status s) {
 
 const char* pa_version(void) { return "pa 0.1 sm_100a"; }
 
+void pa_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns, std::memory_order_relaxed); }
+
 pa_status pa_write_kv(const void* k, const void* v, const int64_t* slot_mapping,
                       int64_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
                       void* k_cache, void* v_cache, int64_t num_blocks, int32_t block_size,
@@ -255,6 +264,57 @@ size_t pa_attention_varlen_workspace_size(int32_t num_seqs, int64_t num_q_tokens
 
 namespace {
 
+// Every host-visible check of a varlen call, in order; nothing is launched or
+// written.  On PA_OK, *sd, *mods and *L hold the resolved strides, modifiers
+// and workspace layout.  *nothing_to_do is set when the call has no rows (the
+// pointers are then not examined).  The workspace size is not compared here.
+pa_status varlen_checks(const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* block_tables, int32_t max_blocks_per_seq,
+                        const int32_t* seq_lens, const int32_t* query_start_loc,
+                        int32_t num_seqs, int64_t num_q_tokens, int32_t num_q_heads,
+                        int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                        int64_t num_blocks, const pa_strides* strides, int32_t dtype,
+                        int32_t max_query_len, int32_t max_seq_len, float scale, int32_t causal,
+                        const int32_t* span_offsets, const int32_t* spans, int32_t num_spans,
+                        const pa_score_mods* score_mods, const void* out, const void* workspace,
+                        Strides* sd, pa::ScoreMods* mods, WorkspaceLayout* L,
+                        bool* nothing_to_do) {
+  *nothing_to_do = false;
+  if (dtype != PA_DTYPE_BF16 && dtype != PA_DTYPE_FP16) return PA_ERR_INVALID_ARG;
+  if (num_seqs < 0 || num_q_tokens < 0 || num_q_tokens > 0x7fffffffll || num_q_heads <= 0 ||
+      num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || max_blocks_per_seq <= 0 ||
+      num_blocks <= 0 || num_blocks > 0x7fffffffll || max_query_len < 0 || max_seq_len < 0 ||
+      (causal != 0 && causal != 1) || !isfinite(scale) || scale < 0.f)
+    return PA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (block_size != pa::kPageKeys) return PA_ERR_UNSUPPORTED;
+  if (num_q_heads / num_kv_heads > 16) return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0 || num_q_tokens == 0) {
+    *nothing_to_do = true;
+    return PA_OK;
+  }
+  if (!q || !k_cache || !v_cache || !block_tables || !seq_lens || !query_start_loc || !out ||
+      !workspace)
+    return PA_ERR_INVALID_ARG;
+  if (span_offsets && (num_spans < 0 || (num_spans > 0 && !spans) ||
+                       (reinterpret_cast<uintptr_t>(span_offsets) & 3u) ||
+                       (reinterpret_cast<uintptr_t>(spans) & 3u)))
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+      (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(query_start_loc) & 3u))
+    return PA_ERR_INVALID_ARG;
+  pa_status rs = resolve_strides(strides, num_q_tokens, num_q_heads, num_kv_heads, head_dim,
+                                 block_size, sd);
+  if (rs != PA_OK) return rs;
+  rs = resolve_mods(score_mods, mods);
+  if (rs != PA_OK) return rs;
+  if (mods->any() && !(scale > 0.f)) return PA_ERR_INVALID_ARG;
+  *L = pa::make_layout(num_seqs, num_q_tokens, num_q_heads, num_kv_heads, head_dim);
+  return PA_OK;
+}
+
 // pa_attention_varlen and pa_attention_varlen_spans (span_offsets non-null)
 pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* v_cache,
                                 const int32_t* block_tables, int32_t max_blocks_per_seq,
@@ -268,41 +328,19 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
                                 const pa_score_mods* score_mods, void* out,
                                 void* workspace, size_t workspace_bytes, void* stream) {
   // ---- host-visible checks (nothing launched yet) ----
-  if (dtype != PA_DTYPE_BF16 && dtype != PA_DTYPE_FP16) return PA_ERR_INVALID_ARG;
-  const bool fp16 = dtype == PA_DTYPE_FP16;
-  if (num_seqs < 0 || num_q_tokens < 0 || num_q_tokens > 0x7fffffffll || num_q_heads <= 0 ||
-      num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || max_blocks_per_seq <= 0 ||
-      num_blocks <= 0 || num_blocks > 0x7fffffffll || max_query_len < 0 || max_seq_len < 0 ||
-      (causal != 0 && causal != 1) || !isfinite(scale) || scale < 0.f)
-    return PA_ERR_INVALID_ARG;
-  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
-  if (block_size != pa::kPageKeys) return PA_ERR_UNSUPPORTED;
-  const int group = num_q_heads / num_kv_heads;
-  if (group > 16) return PA_ERR_UNSUPPORTED;
-  if (num_seqs == 0 || num_q_tokens == 0) return PA_OK;
-  if (!q || !k_cache || !v_cache || !block_tables || !seq_lens || !query_start_loc || !out ||
-      !workspace)
-    return PA_ERR_INVALID_ARG;
-  if (span_offsets && (num_spans < 0 || (num_spans > 0 && !spans) ||
-                       (reinterpret_cast<uintptr_t>(span_offsets) & 3u) ||
-                       (reinterpret_cast<uintptr_t>(spans) & 3u)))
-    return PA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
-      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
-      (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
-      (reinterpret_cast<uintptr_t>(query_start_loc) & 3u))
-    return PA_ERR_INVALID_ARG;
   Strides sd{};
-  pa_status rs = resolve_strides(strides, num_q_tokens, num_q_heads, num_kv_heads, head_dim,
-                                 block_size, &sd);
-  if (rs != PA_OK) return rs;
   pa::ScoreMods mods{};
-  rs = resolve_mods(score_mods, &mods);
-  if (rs != PA_OK) return rs;
-  if (mods.any() && !(scale > 0.f)) return PA_ERR_INVALID_ARG;
-  const WorkspaceLayout L =
-      pa::make_layout(num_seqs, num_q_tokens, num_q_heads, num_kv_heads, head_dim);
+  WorkspaceLayout L{};
+  bool nothing = false;
+  pa_status rs = varlen_checks(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                               query_start_loc, num_seqs, num_q_tokens, num_q_heads, num_kv_heads,
+                               head_dim, block_size, num_blocks, strides, dtype, max_query_len,
+                               max_seq_len, scale, causal, span_offsets, spans, num_spans,
+                               score_mods, out, workspace, &sd, &mods, &L, &nothing);
+  if (rs != PA_OK || nothing) return rs;
   if (workspace_bytes < L.total) return PA_ERR_INVALID_ARG;
+  const bool fp16 = dtype == PA_DTYPE_FP16;
+  const int group = num_q_heads / num_kv_heads;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
@@ -338,8 +376,11 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
   }
 
   // decode CTAs compute their page ranges themselves for up to
-  // kSelfPlanMaxSeqs sequences; beyond that the plan kernel writes the prefix
-  const bool self_plan = num_seqs <= pa::kSelfPlanMaxSeqs;
+  // kSelfPlanMaxSeqs sequences whose arrival counters fit the fixed counter
+  // region (kept zero between calls); beyond that the plan kernel writes the
+  // prefix and zeroes the counters
+  const bool self_plan = num_seqs <= pa::kSelfPlanMaxSeqs &&
+                         (int64_t)num_seqs * num_kv_heads <= pa::kFixedCounterSlots;
   cudaError_t e = cudaSuccess;
   if (run_prefill || !self_plan) {
     pa::launch_plan(query_start_loc, seq_lens, num_seqs, num_q_tokens, max_blocks_per_seq,
@@ -372,6 +413,7 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
     pp.out = static_cast<uint16_t*>(out);
     pp.ws = ws;
     pp.L = L;
+    pp.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
     e = pa::launch_prefill(pp, q_map, k_map, v_map, head_dim, fp16, nsm, st);
     if (e != cudaSuccess) return PA_ERR_CUDA;
   }
@@ -414,6 +456,34 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
 }
 
 }  // namespace
+
+}  // extern "C"
+
+namespace pa {
+
+pa_status check_varlen_args(const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq,
+                            const int32_t* seq_lens, const int32_t* query_start_loc,
+                            int32_t num_seqs, int64_t num_q_tokens, int32_t num_q_heads,
+                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                            int64_t num_blocks, int32_t max_query_len, int32_t max_seq_len,
+                            float scale, int32_t causal, const void* out, const void* workspace,
+                            size_t* workspace_bytes, bool* nothing_to_do) {
+  Strides sd{};
+  ScoreMods mods{};
+  WorkspaceLayout L{};
+  const pa_status rs = varlen_checks(
+      q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, query_start_loc, num_seqs,
+      num_q_tokens, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, nullptr,
+      PA_DTYPE_BF16, max_query_len, max_seq_len, scale, causal, nullptr, nullptr, 0, nullptr, out,
+      workspace, &sd, &mods, &L, nothing_to_do);
+  *workspace_bytes = (rs == PA_OK && !*nothing_to_do) ? L.total : 0;
+  return rs;
+}
+
+}  // namespace pa
+
+extern "C" {
 
 pa_status pa_attention_varlen(const void* q, const void* k_cache, const void* v_cache,
                               const int32_t* block_tables, int32_t max_blocks_per_seq,

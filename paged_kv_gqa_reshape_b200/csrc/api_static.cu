@@ -15,23 +15,30 @@
 //  - The first call on a device looks up the array's device address
 //    (cudaGetSymbolAddress) with that device current, and caches it; make that
 //    first call before any stream capture.
-//  - All calls share the one array, which keeps the last call's contents.  The
-//    plan kernel rebuilds every list and zeroes every split-KV counter at the
-//    start of each call, and this entry point clears the error word, so no
-//    state leaks from one call to the next; but calls whose executions
-//    overlap on the GPU (different streams, or different host threads) race
-//    on the array and must not be issued.
+//  - All calls share the one array, which keeps the last call's contents.
+//    What a call needs at zero is its split-KV arrival counters: they sit in
+//    a region of the array that only ever holds counters, which starts at
+//    zero (a __device__ array is zero-initialised when the module loads) and
+//    is returned to zero by every merge that uses a counter; when the plan
+//    kernel runs (any batch with a multi-query sequence, or too many
+//    sequences for the decode CTAs to plan for themselves) it also zeroes
+//    them.  The plan lists and partial results are rebuilt by each call.
+//    Calls whose executions overlap on the GPU (different streams, or
+//    different host threads) race on the array and must not be issued.
 //  - Device-side index errors are handled as in pa_attention_varlen (rows
 //    skipped, reads zero-filled) but cannot be read back: the error word lives
-//    in the shared array, not in a caller buffer.
-//  - Sizes whose workspace would exceed PA_STATIC_SCRATCH_BYTES are rejected
-//    with PA_ERR_UNSUPPORTED before anything is launched.
+//    in the shared array, which nothing reads.
+//  - Bad arguments are reported exactly as pa_attention_varlen reports them;
+//    then sizes whose workspace would exceed PA_STATIC_SCRATCH_BYTES are
+//    rejected with PA_ERR_UNSUPPORTED.  Both happen before anything is
+//    launched or written.
 // Nothing here calls cudaMalloc, cudaFree or any allocating library routine.
 #include <cuda_runtime.h>
 
 #include <mutex>
 
 #include "../../include/pa.h"
+#include "kernels.h"
 
 namespace {
 
@@ -67,16 +74,21 @@ extern "C" pa_status pa_attention_varlen_static(
     int32_t num_seqs, int64_t num_q_tokens, int32_t num_q_heads, int32_t num_kv_heads,
     int32_t head_dim, int32_t block_size, int64_t num_blocks, int32_t max_query_len,
     int32_t max_seq_len, float scale, int32_t causal, void* out, void* stream) {
-  const size_t need = pa_attention_varlen_workspace_size(num_seqs, num_q_tokens, num_q_heads,
-                                                         num_kv_heads, head_dim);
+  // The arguments are checked first, with the array's alignment standing in
+  // for the workspace pointer (the array is 256-byte aligned, so that check
+  // passes for it), so that a bad call is reported before any CUDA call.
+  const void* aligned_stand_in = reinterpret_cast<const void*>(uintptr_t(256));
+  size_t need = 0;
+  bool nothing = false;
+  pa_status st = pa::check_varlen_args(
+      q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, query_start_loc, num_seqs,
+      num_q_tokens, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, max_query_len,
+      max_seq_len, scale, causal, out, aligned_stand_in, &need, &nothing);
+  if (st != PA_OK || nothing) return st;
   if (need > (size_t)PA_STATIC_SCRATCH_BYTES) return PA_ERR_UNSUPPORTED;
   void* scratch = nullptr;
-  pa_status st = scratch_address(&scratch);
+  st = scratch_address(&scratch);
   if (st != PA_OK) return st;
-  if (need > 0 && num_seqs > 0 && num_q_tokens > 0 &&
-      cudaMemsetAsync(scratch, 0, sizeof(uint32_t), static_cast<cudaStream_t>(stream)) !=
-          cudaSuccess)
-    return PA_ERR_CUDA;
   return pa_attention_varlen(q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
                              query_start_loc, num_seqs, num_q_tokens, num_q_heads, num_kv_heads,
                              head_dim, block_size, num_blocks, max_query_len, max_seq_len, scale,

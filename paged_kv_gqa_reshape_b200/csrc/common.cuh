@@ -3,8 +3,8 @@
 // Thin inline-PTX wrappers for the instructions the kernels issue directly:
 // cp.async (Ampere-style 16-byte async copies), ldmatrix, mma.sync bf16,
 // mbarrier, TMA tensor loads and the tcgen05 family.  Every wait on an
-// mbarrier is bounded in wall time (mbar_wait_bounded): after one second it
-// gives up, raises PA_DEVERR_TIMEOUT in the caller's error word and returns
+// mbarrier is bounded in wall time (mbar_wait_bounded): after one second (or
+// a shorter limit a test sets) it gives up, raises PA_DEVERR_TIMEOUT in the caller's error word and returns
 // false, so a lost arrival can never hang the GPU.
 #pragma once
 
@@ -313,17 +313,21 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Wait for an mbarrier phase, bounded in wall time.  On timeout (or when
-// another role of the CTA already gave up) returns false; the first role to
-// time out raises PA_DEVERR_TIMEOUT and sets the CTA's abort flag.
+// Default limit of a bounded wait: 1 s, far beyond any legitimate wait.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+
+// Wait for an mbarrier phase, bounded in wall time (limit_ns).  On timeout (or
+// when another role of the CTA already gave up) returns false; the first role
+// to time out raises PA_DEVERR_TIMEOUT and sets the CTA's abort flag.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort_flag, uint32_t* err) {
+                                                  volatile int* abort_flag, uint32_t* err,
+                                                  uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > 1000000000ull) {  // 1 s: no legitimate wait is this long
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       raise_error(err, PA_DEVERR_TIMEOUT);
       return false;

@@ -6,9 +6,24 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/pa.h"
 #include "layout.h"
 
 namespace pa {
+
+// ---- host-side argument checks ---------------------------------------------
+// Every host-visible check pa_attention_varlen makes, without launching or
+// writing anything and without comparing a workspace size.  On PA_OK,
+// *workspace_bytes is the workspace the call needs (0 when it has no rows, in
+// which case *nothing_to_do is set and the pointers were not examined).
+pa_status check_varlen_args(const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq,
+                            const int32_t* seq_lens, const int32_t* query_start_loc,
+                            int32_t num_seqs, int64_t num_q_tokens, int32_t num_q_heads,
+                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                            int64_t num_blocks, int32_t max_query_len, int32_t max_seq_len,
+                            float scale, int32_t causal, const void* out, const void* workspace,
+                            size_t* workspace_bytes, bool* nothing_to_do);
 
 // ---- KV scatter ------------------------------------------------------------
 // Cache destination of vector c of head h of slot s: (s / block_size) *
@@ -92,6 +107,7 @@ struct PrefillParams {
   uint16_t* out;  // elements of the kernel's type (bf16 or fp16)
   unsigned char* ws;
   WorkspaceLayout L;
+  unsigned long long wait_limit_ns;  // bound of every mbarrier wait; 0: the 1 s default
 };
 // Tensor maps are built by the host layer (they need the driver entry point).
 cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& q_map,

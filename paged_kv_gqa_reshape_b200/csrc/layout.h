@@ -15,6 +15,12 @@ constexpr int kPageKeys = 16;           // block_size this build supports
 constexpr int kDecodeMaxWarps = 4096;   // bound on decode warps in one launch (8 per SM)
 constexpr int kCostBuckets = 4096;      // prefill tiles are sorted by KV-tile count
 constexpr int kSelfPlanMaxSeqs = 1024;  // decode CTAs plan for themselves up to this many sequences
+// Split-KV arrival counters live at a fixed offset, in a region no layout
+// uses for anything else, at least this many int32 long.  Each merge resets
+// its counter after use, so once the workspace has been zeroed the region
+// stays zero between calls whatever their sizes; a call that plans for itself
+// (no plan kernel to zero them) must fit its counters in this region.
+constexpr int kFixedCounterSlots = 65536;
 
 // Sanitised geometry of one sequence, written by the plan kernel.  The
 // attention kernels read lengths only from here, never from the raw inputs.
@@ -39,7 +45,8 @@ struct WorkspaceLayout {
   size_t tiles;      // int2[max_tiles]   (seq, first query row of a 256-row work item)
   size_t tile_n;     // int2[max_tiles]   KV tiles its two 128-row query tiles visit
   size_t page_pfx;   // int32[num_seqs + 1]  exclusive prefix of decode pages
-  size_t counters;   // int32[num_seqs * num_kv_heads]  split-KV arrival counters
+  size_t counters;   // int32[max(num_seqs * num_kv_heads, kFixedCounterSlots)]  split-KV
+                     // arrival counters, at a fixed offset (see kFixedCounterSlots)
   size_t lse;        // float[max_slots * num_q_heads]   log2-sum-exp per partial
   size_t partial;    // float[max_slots * num_q_heads * head_dim]
   size_t total;
@@ -57,6 +64,11 @@ inline WorkspaceLayout make_layout(int64_t num_seqs, int64_t num_q_tokens, int64
   off += 256;
   L.header = off;
   off += sizeof(PlanHeader);
+  L.counters = off;  // fixed offset: the same in every layout
+  const int64_t counter_slots = num_seqs * num_kv_heads > kFixedCounterSlots
+                                    ? num_seqs * num_kv_heads
+                                    : (int64_t)kFixedCounterSlots;
+  off = align_up(off + 4 * (size_t)counter_slots, 256);
   L.seq_info = off;
   off = align_up(off + sizeof(SeqInfo) * (size_t)num_seqs, 256);
   L.max_tiles = (num_q_tokens + kPrefillItemRows - 1) / kPrefillItemRows + num_seqs;
@@ -69,8 +81,6 @@ inline WorkspaceLayout make_layout(int64_t num_seqs, int64_t num_q_tokens, int64
   L.max_slots = (kDecodeMaxWarps + num_kv_heads - 1) / num_kv_heads + num_seqs;
   L.page_pfx = off;
   off = align_up(off + 4 * (size_t)(num_seqs + 1), 256);
-  L.counters = off;
-  off = align_up(off + 4 * (size_t)(num_seqs * num_kv_heads), 256);
   L.lse = off;
   off = align_up(off + 4 * (size_t)(L.max_slots * num_q_heads), 256);
   L.partial = off;

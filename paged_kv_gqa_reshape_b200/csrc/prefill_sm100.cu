@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int2* tiles = reinterpret_cast<const int2*>(ws + p.L.tiles);
   const int2* tile_n = reinterpret_cast<const int2*>(ws + p.L.tile_n);
   const int num_work = hdr->num_prefill_tiles * p.num_q_heads;
+  const uint64_t wlim = p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs;
   // Work distribution: the first item of a CTA is blockIdx.x; later ones are
   // taken from a counter (sorted by descending cost, so the longest go first),
   // so SMs that run faster take more items.  The producer publishes each item
@@ -159,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto read_item = [&](int k, bool& ok) -> int {
     const int slot = k % SM::kItemRing;
     ok = ok && mbar_wait_bounded(item_full + slot, (uint32_t)((k / SM::kItemRing) & 1), abort_flag,
-                                 err);
+                                 err, wlim);
     return ok ? s_item[slot] : -1;
   };
 
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int slot = k % SM::kItemRing;
         if (k >= SM::kItemRing)
           ok = mbar_wait_bounded(item_empty + slot, (uint32_t)((k / SM::kItemRing - 1) & 1),
-                                 abort_flag, err);
+                                 abort_flag, err, wlim);
         if (!ok) break;
         s_item[slot] = w;
         mbar_arrive(item_full + slot);
@@ -223,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (wk.nmax == 0) continue;
         const int kvh = wk.head / p.group;
         const int kv_c1 = kv_hnd ? 0 : kvh, kv_c2 = kv_hnd ? kvh : 0;  // (head, slot) or (slot, head)
-        if (tcount > 0) ok = mbar_wait_bounded(q_empty, (tcount - 1) & 1, abort_flag, err);
+        if (tcount > 0) ok = mbar_wait_bounded(q_empty, (tcount - 1) & 1, abort_flag, err, wlim);
         if (!ok) break;
         mbar_arrive_expect_tx(q_full, 2 * SM::kQBytes);
 #pragma unroll
@@ -253,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kv = 0; kv < 2; ++kv, ++ld) {  // K_j, then V_j
             const int st = (int)(ld % kRing);
             const long long round = ld / kRing;
-            if (round > 0) ok = mbar_wait_bounded(slot_empty + st, (round - 1) & 1, abort_flag, err);
+            if (round > 0) ok = mbar_wait_bounded(slot_empty + st, (round - 1) & 1, abort_flag, err, wlim);
             if (!ok) break;
             mbar_arrive_expect_tx(slot_full + st, SM::kKVBytes);
             const void* map = kv == 0 ? (const void*)&k_map : (const void*)&v_map;
@@ -279,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       auto wait_tile = [&](long long idx) {
         return mbar_wait_bounded(slot_full + (int)(idx % kRing), (uint32_t)((idx / kRing) & 1),
-                                 abort_flag, err);
+                                 abort_flag, err, wlim);
       };
       auto issue_s = [&](int x, long long kidx) {
         const uint32_t kb = ring_s + (int)(kidx % kRing) * SM::kKVBytes;
@@ -310,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (w < 0) break;
         const Work wk = decode_work(w, tiles, tile_n, info, p.num_q_heads);
         if (wk.nmax == 0) continue;
-        ok = mbar_wait_bounded(q_full, tcount & 1, abort_flag, err);
+        ok = mbar_wait_bounded(q_full, tcount & 1, abort_flag, err, wlim);
         if (!ok) break;
         tc_fence_after();
         const long long base = ld;  // K_j = base + 2j, V_j = base + 2j + 1
@@ -326,14 +327,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
             if (j >= wk.n[x]) continue;
-            ok = mbar_wait_bounded(p_full + x, pv_it[x] & 1, abort_flag, err);
+            ok = mbar_wait_bounded(p_full + x, pv_it[x] & 1, abort_flag, err, wlim);
             if (ok) ok = wait_tile(vj);
             if (!ok) break;
             tc_fence_after();
             issue_pv(x, vj, j > 0);
             if (j + 1 < wk.n[x]) {
               // S_x(j+1) overwrites the columns P_x(j) occupies: let P_x(j).V finish
-              ok = mbar_wait_bounded(o_done + x, (pv_it[x] - 1) & 1, abort_flag, err);
+              ok = mbar_wait_bounded(o_done + x, (pv_it[x] - 1) & 1, abort_flag, err, wlim);
               if (ok) ok = wait_tile(kn);
               if (!ok) break;
               tc_fence_after();
@@ -401,14 +402,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // S_x(j) has landed.  P_x(j-1).V was issued before S_x(j) by the same
         // thread, so waiting for it here (P buffer free, O stable) costs nothing
         // and lets P be stored as it is computed.
-        ok = mbar_wait_bounded(s_full + x, cur & 1, abort_flag, err);
-        if (ok && cur > 0) ok = mbar_wait_bounded(o_done + x, (cur - 1) & 1, abort_flag, err);
+        ok = mbar_wait_bounded(s_full + x, cur & 1, abort_flag, err, wlim);
+        if (ok && cur > 0) ok = mbar_wait_bounded(o_done + x, (cur - 1) & 1, abort_flag, err, wlim);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
         // The row's 128 raw scores come into registers with four TMEM loads and
         // one wait; the max and the exponentials both work from those registers.
-        // The scale is applied after the max (scale_log2 > 0, so the max
+        // The scale is applied after the max (scale_log2 >= 0, so the max
         // commutes with it) and in the exponent's FFMA.  Reductions use
         // independent partials (short trees, not 128-long dependency chains).
         const int key0 = j * BN;
@@ -504,11 +505,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         // Tiles crossing the diagonal or the sequence end set hidden keys to
-        // -inf once; the others skip every per-key test.
+        // -inf once; the others skip every per-key test.  A masked tile is
+        // scaled here, before the -inf goes in, and then runs with unit scale
+        // below: with scale 0 the product -inf * 0 would be NaN, whereas
+        // scaling first gives 0 for every visible key (a uniform softmax)
+        // and keeps the hidden ones at -inf.
+        float tile_scale = p.scale_log2;
         if (masked_tile) {
+          tile_scale = 1.f;
 #pragma unroll
           for (int c = 0; c < BN; ++c)
-            if (c >= valid) sv[c] = __float_as_uint(-INFINITY);
+            sv[c] = __float_as_uint(c >= valid ? -INFINITY : __uint_as_float(sv[c]) * p.scale_log2);
         }
         constexpr int NP = 4;
         float mp[NP];
@@ -521,7 +528,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int wdt = NP / 2; wdt >= 1; wdt >>= 1)
 #pragma unroll
           for (int i = 0; i < wdt; ++i) mp[i] = fmaxf(mp[i], mp[i + wdt]);
-        const float m_tile = mp[0] * p.scale_log2;  // scale_log2 > 0: max commutes with it
+        // tile_scale >= 0, so the max commutes with it; on an unmasked tile
+        // every score is finite, so scale 0 gives 0 here, not NaN
+        const float m_tile = mp[0] * tile_scale;
         const float m_old = m_use;
         const bool grow =
             m_tile > m_old + kRescaleThreshold || (m_old == -INFINITY && m_tile > -INFINITY);
@@ -532,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // p = 2^(scale_log2 * s - base), rounded to bf16 and written to TMEM as
         // the A operand of O += P.V.  Scaling and row sums run on packed fp32
         // pairs; the exponentials on the SFU.
-        const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t scale2 = f2_pack(tile_scale, tile_scale);
         const uint64_t nbase2 = f2_pack(-base, -base);
         uint64_t rs2[NP / 2];
 #pragma unroll
@@ -578,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       // epilogue: O / l -> bf16 -> global
       const int last = it + n - 1;
-      ok = mbar_wait_bounded(o_done + x, last & 1, abort_flag, err);
+      ok = mbar_wait_bounded(o_done + x, last & 1, abort_flag, err, wlim);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();

@@ -237,26 +237,41 @@ def test_mixed_small():
     assert pa.get_error(ws) == (0, 0)
 
 
-def test_mixed_config_full_size_sampled():
+def test_mixed_config_full_size():
+    """The full mixed chunked-prefill + decode step: every decode row, and every
+    prefill chunk at its tile-edge rows (0, 1, 127-129, 255, 256, the last)
+    plus every 37th row, each against the oracle.  The sequences are handed to
+    the oracle a few at a time so that the host holds a slice of the 17 GB of
+    logical K/V, not all of it."""
     dev = workloads.mixed_step(device="cuda")
     out, _, _, ws = run_varlen(dev)
     assert pa.get_error(ws) == (0, 0)
-    # two prefill chunks (16 rows each) and six decodes, checked one by one
-    picks = [0, 5, 8, 50, 100, 150, 200, 255]
-    sub = sub_case(dev, picks)
     qsl_full = dev.query_start_loc.cpu().tolist()
-    sub_rows, full_rows = [], []
-    sq = sub.query_start_loc.tolist()
-    for k, s in enumerate(picks):
-        n = qsl_full[s + 1] - qsl_full[s]
-        take = range(n) if n <= 1 else sorted(set(list(range(0, n, 37)) + [n - 1]))
-        for i in take:
-            sub_rows.append(sq[k] + i)
-            full_rows.append(qsl_full[s] + i)
-    sub_rows = np.array(sub_rows, np.int64)
-    ref = oracle_varlen(sub, rows=sub_rows)[sub_rows]
-    got = out[torch.tensor(full_rows, device=out.device)]
-    assert_attention_close(got, ref, what="mixed full (sampled)")
+    n_seq = dev.num_seqs
+    edges = (0, 1, 127, 128, 129, 255, 256, 383, 384, 511)
+    got_all, ref_all = [], []
+    batch = 32
+    for first in range(0, n_seq, batch):
+        picks = list(range(first, min(n_seq, first + batch)))
+        sub = sub_case(dev, picks)
+        sq = sub.query_start_loc.tolist()
+        sub_rows, full_rows = [], []
+        for k, s in enumerate(picks):
+            n = qsl_full[s + 1] - qsl_full[s]
+            take = range(n) if n <= 1 else sorted(
+                {i for i in edges if i < n} | set(range(0, n, 37)) | {n - 1})
+            for i in take:
+                sub_rows.append(sq[k] + i)
+                full_rows.append(qsl_full[s] + i)
+        sub_rows = np.array(sub_rows, np.int64)
+        ref_all.append(oracle_varlen(sub, rows=sub_rows)[sub_rows])
+        got_all.append(out[torch.tensor(full_rows, device=out.device)].cpu())
+        del sub
+    got = torch.cat(got_all)
+    ref = np.concatenate(ref_all)
+    assert got.shape[0] == 248 + sum(
+        len({i for i in edges if i < 512} | set(range(0, 512, 37)) | {511}) for _ in range(8))
+    assert_attention_close(got, ref, what="mixed full (every decode, chunk edges)")
 
 
 # ---------------------------------------------------------------------------
@@ -357,3 +372,22 @@ def test_decode_repeated_calls_reuse_counters():
     for o in outs:
         assert_attention_close(o, ref, what="repeated decode")
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+
+
+def test_workspace_reused_across_batch_shapes():
+    # One workspace, sized for the largest call, reused by calls of different
+    # shapes in a row: a few long split-KV decodes (their partials fill the
+    # workspace's scratch), then a larger pure-decode batch that plans for
+    # itself, then a mixed batch, then the larger decode batch again.  The
+    # arrival counters must read zero at the start of every call.
+    a = build([5000, 4000, 3000, 6000, 2500, 4500, 3500, 5500], [1] * 8, 32, 8, 128, seed=21)
+    rng = np.random.default_rng(22)
+    lens_b = rng.integers(1, 3000, size=200).tolist()
+    b = build(lens_b, [1] * 200, 32, 8, 128, seed=22)
+    c = build([700, 40, 300, 1, 2000, 17, 5, 129], [64, 1, 300, 1, 1, 17, 1, 100], 32, 8, 128,
+              seed=23)
+    ws = pa.varlen_workspace(256, 1024, 32, 8, 128)
+    for case in (a, b, c, b):
+        out, _, _, _ = run_varlen(case_to(case, "cuda"), workspace=ws)
+        assert_attention_close(out, oracle_varlen(case), what=f"reused workspace S={case.num_seqs}")
+    assert pa.get_error(ws) == (0, 0)
