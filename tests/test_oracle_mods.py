@@ -189,3 +189,26 @@ def test_modifiers_with_spans_match_sdpa():
     ref = torch.nn.functional.scaled_dot_product_attention(
         q, k, v, attn_mask=bias.masked_fill(~vis, float("-inf")), scale=case.scale)
     assert np.max(np.abs(got - ref.transpose(0, 1).numpy())) < 1e-10
+
+
+def test_golden_softcap_saturation():
+    """Hand-derived worked example (tests/golden/softcap_saturation.json): scores
+    of +-1000 under a cap of 2 saturate to exactly +-2, so the output is the
+    closed form (1/(1+e^-4), e^-4/(1+e^-4), 0, 0); without the cap, or with the
+    cap placed after the softmax, the second weight would be 0."""
+    from tests.conftest import load_golden
+    g = load_golden("softcap_saturation")
+
+    def bits(x):
+        t = torch.tensor(np.asarray(x, dtype=np.float32)).to(torch.bfloat16)
+        assert torch.equal(t.float(), torch.tensor(np.asarray(x, dtype=np.float32)))
+        return t.view(torch.int16).numpy().view(np.uint16)
+    out = oracle.attention_varlen_mods(
+        bits(g["q"]), bits(g["k"]), bits(g["v"]), np.array([0], np.int64),
+        np.array([2], np.int32), np.array([0, 1], np.int32), 1, g["scale"], g["causal"],
+        softcap=g["softcap"])
+    assert np.allclose(out, np.array(g["expected"]), rtol=0, atol=1e-15)
+    uncapped = oracle.attention_varlen_mods(
+        bits(g["q"]), bits(g["k"]), bits(g["v"]), np.array([0], np.int64),
+        np.array([2], np.int32), np.array([0, 1], np.int32), 1, g["scale"], g["causal"])
+    assert np.array_equal(uncapped[0, 0], np.array([1.0, 0.0, 0.0, 0.0]))
