@@ -44,7 +44,7 @@ WORKLOAD = ("decode_batch: 64 seqs x 1 query token, context U[256,4096], Hq 32 /
 # while the decode kernel's sources hash to the recorded value.
 DECODE_TRAFFIC = {"sources_sha256": "232e848bf67035a6b26be84dd2272e9b7c8ba62e6d01b1931e99253fc906a3b7",
                   "bytes_per_launch": 599628971}
-DECODE_SOURCES = ("decode.cu", "common.cuh", "layout.h")
+DECODE_SOURCES = ("decode.cu", "decode.cuh", "common.cuh", "layout.h")
 
 
 def decode_sources_sha() -> str:

@@ -165,8 +165,12 @@ size_t pa_attention_varlen_workspace_size(int32_t num_seqs, int64_t num_q_tokens
  *  out              [num_q_tokens, num_q_heads, head_dim] bf16, written for
  *                   every token that belongs to a sequence
  *  workspace        device buffer of >= workspace_size bytes (see above)
- * Supported: head_dim in {64, 128}; block_size == 16;
- * num_q_heads / num_kv_heads <= 16 (decode packs a GQA group into one tile).
+ * Supported: head_dim in {64, 128}; block_size a multiple of 16, up to 512
+ * (the kernels fetch and count keys in 16-slot pages; a block holds
+ * block_size / 16 of them);
+ * num_q_heads / num_kv_heads <= 128 (a decode warp serves up to 16 query heads
+ * of a GQA group; larger groups are cut into 16-head slices, up to 8 warps
+ * sharing the KV head's pages).
  */
 pa_status pa_attention_varlen(const void* q, const void* k_cache, const void* v_cache,
                               const int32_t* block_tables, int32_t max_blocks_per_seq,

@@ -8,8 +8,9 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpa.so")
-SOURCES = ["api.cu", "api_static.cu", "plan.cu", "scatter.cu", "smallseq.cu", "smallseq_bwd.cu", "decode.cu", "prefill_sm100.cu"]
-HEADERS = ["common.cuh", "kernels.h", "layout.h", "spans.cuh"]
+SOURCES = ["api.cu", "api_static.cu", "plan.cu", "scatter.cu", "smallseq.cu", "smallseq_bwd.cu",
+           "decode.cu", "decode_sliced.cu", "prefill_sm100.cu"]
+HEADERS = ["common.cuh", "decode.cuh", "kernels.h", "layout.h", "spans.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

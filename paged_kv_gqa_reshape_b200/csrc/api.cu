@@ -287,8 +287,10 @@ pa_status varlen_checks(const void* q, const void* k_cache, const void* v_cache,
       (causal != 0 && causal != 1) || !isfinite(scale) || scale < 0.f)
     return PA_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
-  if (block_size != pa::kPageKeys) return PA_ERR_UNSUPPORTED;
-  if (num_q_heads / num_kv_heads > 16) return PA_ERR_UNSUPPORTED;
+  if (block_size < pa::kPageKeys || block_size > pa::kMaxBlockSize ||
+      (block_size & (block_size - 1)) != 0)
+    return PA_ERR_UNSUPPORTED;
+  if (num_q_heads / num_kv_heads > pa::kMaxGroup) return PA_ERR_UNSUPPORTED;
   if (num_seqs == 0 || num_q_tokens == 0) {
     *nothing_to_do = true;
     return PA_OK;
@@ -379,12 +381,14 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
   // kSelfPlanMaxSeqs sequences whose arrival counters fit the fixed counter
   // region (kept zero between calls); beyond that the plan kernel writes the
   // prefix and zeroes the counters
-  const bool self_plan = num_seqs <= pa::kSelfPlanMaxSeqs &&
-                         (int64_t)num_seqs * num_kv_heads <= pa::kFixedCounterSlots;
+  const bool self_plan =
+      num_seqs <= pa::kSelfPlanMaxSeqs &&
+      pa::counter_slots_needed(num_seqs, num_q_heads, num_kv_heads) <= pa::kFixedCounterSlots;
   cudaError_t e = cudaSuccess;
   if (run_prefill || !self_plan) {
     pa::launch_plan(query_start_loc, seq_lens, num_seqs, num_q_tokens, max_blocks_per_seq,
-                    block_size, max_query_len, max_seq_len, causal, num_kv_heads, span_offsets,
+                    block_size, max_query_len, max_seq_len, causal,
+                    pa::counter_slots_needed(num_seqs, num_q_heads, num_kv_heads), span_offsets,
                     spans, num_spans, ws, L, st);
     e = cudaGetLastError();
     if (e != cudaSuccess) return PA_ERR_CUDA;
@@ -394,6 +398,8 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
     pa::PrefillParams pp{};
     pp.block_tables = block_tables;
     pp.max_blocks_per_seq = max_blocks_per_seq;
+    pp.block_size = block_size;
+    pp.ppb_shift = pa::log2_pages_per_block(block_size);
     pp.num_q_heads = num_q_heads;
     pp.num_kv_heads = num_kv_heads;
     pp.group = group;
@@ -429,11 +435,13 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
   dp.num_q_tokens = num_q_tokens;
   dp.max_query_len = max_query_len;
   dp.max_blocks_per_seq = max_blocks_per_seq;
+  dp.ppb_shift = pa::log2_pages_per_block(block_size);
   dp.max_seq_len = max_seq_len;
   dp.self_plan = self_plan ? 1 : 0;
   dp.num_q_heads = num_q_heads;
   dp.num_kv_heads = num_kv_heads;
   dp.group = group;
+  dp.slices = pa::decode_slices(group);
   dp.num_blocks = num_blocks;
   dp.block_stride = sd.cb;
   dp.c_slot = sd.cs;

@@ -38,7 +38,7 @@ cudaError_t launch_write_kv(const void* k, const void* v, const int64_t* slot_ma
 // ---- plan ------------------------------------------------------------------
 void launch_plan(const int32_t* query_start_loc, const int32_t* seq_lens, int num_seqs,
                  long long num_q_tokens, int max_blocks_per_seq, int block_size,
-                 int max_query_len, int max_seq_len, int causal, int num_kv_heads,
+                 int max_query_len, int max_seq_len, int causal, long long num_counters,
                  const int32_t* span_offsets, const int32_t* spans, int num_spans,
                  unsigned char* ws, const WorkspaceLayout& L, cudaStream_t stream);
 
@@ -63,11 +63,13 @@ struct DecodeParams {
   int num_seqs;
   long long num_q_tokens;
   int max_blocks_per_seq;
+  int ppb_shift;     // log2(block_size / 16): a cache block holds 1 << ppb_shift 16-key pages
   int max_query_len; // host hint, checked
   int max_seq_len;   // host hint, checked
   int num_q_heads;
   int num_kv_heads;
-  int group;  // num_q_heads / num_kv_heads, <= 16
+  int group;   // num_q_heads / num_kv_heads, <= kMaxGroup
+  int slices;  // warps per KV head: decode_slices(group)
   long long num_blocks;
   long long block_stride;  // elements between consecutive cache blocks
   long long c_slot, c_head;  // elements between slots of a block / KV heads of a slot
@@ -84,11 +86,16 @@ struct DecodeParams {
 // Persistent launch: one resident wave, num_sms from the device.
 cudaError_t launch_decode(const DecodeParams& p, int head_dim, bool fp16, int num_sms,
                           cudaStream_t stream);
+// The same for slices > 1 (GQA groups of more than 16 query heads).
+cudaError_t launch_decode_sliced(const DecodeParams& p, int head_dim, bool fp16, int num_sms,
+                                 cudaStream_t stream);
 
 // ---- tcgen05 prefill ------------------------------------------------------
 struct PrefillParams {
   const int32_t* block_tables;
   int max_blocks_per_seq;
+  int block_size;   // slots per cache block: 16 << ppb_shift
+  int ppb_shift;    // log2(block_size / 16)
   int num_q_heads;
   int num_kv_heads;
   int group;

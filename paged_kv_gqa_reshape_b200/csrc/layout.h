@@ -11,7 +11,15 @@ namespace pa {
 constexpr int kPrefillTileM = 128;      // query rows per prefill tile (tcgen05 M)
 constexpr int kPrefillItemRows = 256;   // query rows per prefill work item: two tiles
 constexpr int kPrefillTileN = 128;      // keys per prefill KV tile (tcgen05 N)
-constexpr int kPageKeys = 16;           // block_size this build supports
+constexpr int kPageKeys = 16;           // keys per page: the unit the kernels fetch and count
+constexpr int kMaxBlockSize = 512;      // block_size: a power of two from kPageKeys up to this
+
+// log2 of the 16-key pages in a cache block of block_size slots (a power of two >= 16).
+inline int log2_pages_per_block(int block_size) {
+  int s = 0;
+  while ((kPageKeys << s) < block_size) ++s;
+  return s;
+}
 constexpr int kDecodeMaxWarps = 4096;   // bound on decode warps in one launch (8 per SM)
 constexpr int kCostBuckets = 4096;      // prefill tiles are sorted by KV-tile count
 constexpr int kSelfPlanMaxSeqs = 1024;  // decode CTAs plan for themselves up to this many sequences
@@ -21,6 +29,17 @@ constexpr int kSelfPlanMaxSeqs = 1024;  // decode CTAs plan for themselves up to
 // stays zero between calls whatever their sizes; a call that plans for itself
 // (no plan kernel to zero them) must fit its counters in this region.
 constexpr int kFixedCounterSlots = 65536;
+
+constexpr int kMaxGroup = 128;          // largest GQA group (num_q_heads / num_kv_heads)
+
+// Warps of the decode kernel that share one KV head: one warp serves up to 16
+// query heads of its GQA group, so larger groups are cut into 16-head slices;
+// a power of two (1, 2, 4 or 8) so that the slices tile a CTA's warps.
+inline int decode_slices(int64_t group) {
+  int s = 1;
+  while (s * 16 < group) s *= 2;
+  return s;
+}
 
 // Sanitised geometry of one sequence, written by the plan kernel.  The
 // attention kernels read lengths only from here, never from the raw inputs.
@@ -45,8 +64,8 @@ struct WorkspaceLayout {
   size_t tiles;      // int2[max_tiles]   (seq, first query row of a 256-row work item)
   size_t tile_n;     // int2[max_tiles]   KV tiles its two 128-row query tiles visit
   size_t page_pfx;   // int32[num_seqs + 1]  exclusive prefix of decode pages
-  size_t counters;   // int32[max(num_seqs * num_kv_heads, kFixedCounterSlots)]  split-KV
-                     // arrival counters, at a fixed offset (see kFixedCounterSlots)
+  size_t counters;   // int32[max(num_seqs * num_kv_heads * slices, kFixedCounterSlots)]
+                     // split-KV arrival counters, at a fixed offset (see kFixedCounterSlots)
   size_t lse;        // float[max_slots * num_q_heads]   log2-sum-exp per partial
   size_t partial;    // float[max_slots * num_q_heads * head_dim]
   size_t total;
@@ -55,6 +74,11 @@ struct WorkspaceLayout {
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Split-KV arrival counters a call uses: one per (sequence, KV head, slice).
+inline int64_t counter_slots_needed(int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads) {
+  return num_seqs * num_kv_heads * decode_slices(num_q_heads / num_kv_heads);
+}
 
 inline WorkspaceLayout make_layout(int64_t num_seqs, int64_t num_q_tokens, int64_t num_q_heads,
                                    int64_t num_kv_heads, int64_t head_dim) {
@@ -65,9 +89,8 @@ inline WorkspaceLayout make_layout(int64_t num_seqs, int64_t num_q_tokens, int64
   L.header = off;
   off += sizeof(PlanHeader);
   L.counters = off;  // fixed offset: the same in every layout
-  const int64_t counter_slots = num_seqs * num_kv_heads > kFixedCounterSlots
-                                    ? num_seqs * num_kv_heads
-                                    : (int64_t)kFixedCounterSlots;
+  const int64_t need = counter_slots_needed(num_seqs, num_q_heads, num_kv_heads);
+  const int64_t counter_slots = need > kFixedCounterSlots ? need : (int64_t)kFixedCounterSlots;
   off = align_up(off + 4 * (size_t)counter_slots, 256);
   L.seq_info = off;
   off = align_up(off + sizeof(SeqInfo) * (size_t)num_seqs, 256);

@@ -82,7 +82,7 @@ __device__ __forceinline__ int2 item_tiles(const SeqInfo& si, int row0, int caus
 __global__ void __launch_bounds__(kPlanThreads, 1)
     plan_kernel(const int32_t* __restrict__ query_start_loc, const int32_t* __restrict__ seq_lens,
                 int num_seqs, long long num_q_tokens, int max_blocks_per_seq, int block_size,
-                int max_query_len, int max_seq_len, int causal, int num_kv_heads,
+                int max_query_len, int max_seq_len, int causal, long long num_counters,
                 const int32_t* __restrict__ span_offsets, const int32_t* __restrict__ spans,
                 int num_spans, unsigned char* ws, WorkspaceLayout L) {
   uint32_t* err = reinterpret_cast<uint32_t*>(ws + L.err);
@@ -101,8 +101,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
   const int tid = threadIdx.x;
   if (tid == 0) s_err = 0;
   for (int i = tid; i < kCostBuckets; i += blockDim.x) s_hist[i] = 0;
-  for (long long i = tid; i < (long long)num_seqs * num_kv_heads; i += blockDim.x)
-    counters[i] = 0;
+  for (long long i = tid; i < num_counters; i += blockDim.x) counters[i] = 0;
   __syncthreads();
 
   // ---- pass 1: sanitise lengths, total decode keys -------------------------
@@ -219,12 +218,12 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
 
 void launch_plan(const int32_t* query_start_loc, const int32_t* seq_lens, int num_seqs,
                  long long num_q_tokens, int max_blocks_per_seq, int block_size,
-                 int max_query_len, int max_seq_len, int causal, int num_kv_heads,
+                 int max_query_len, int max_seq_len, int causal, long long num_counters,
                  const int32_t* span_offsets, const int32_t* spans, int num_spans,
                  unsigned char* ws, const WorkspaceLayout& L, cudaStream_t stream) {
   plan_kernel<<<1, kPlanThreads, 0, stream>>>(query_start_loc, seq_lens, num_seqs, num_q_tokens,
                                               max_blocks_per_seq, block_size, max_query_len,
-                                              max_seq_len, causal, num_kv_heads, span_offsets,
+                                              max_seq_len, causal, num_counters, span_offsets,
                                               spans, num_spans, ws, L);
 }
 

@@ -14,7 +14,8 @@
 //    that share every K/V tile;
 //  * warp 0 (one lane): TMA producer.  Q tiles via a 3-D map over
 //    [tokens, Hq, D]; each 128-key K/V tile as eight 16-key pages fetched
-//    through the block table with a 4-D map over [blocks, 16, Hkv, D]
+//    through the block table with a 4-D map over [blocks, block_size, Hkv,
+//    D] (a block of 16k slots holds k pages)
 //    (a page past the sequence end, or a bad block id, is fetched at an
 //    out-of-range coordinate, i.e. as zeros).  128-byte swizzle, no
 //    multicast.  K and V tiles go through one ring (4 slots for D = 128,
@@ -112,7 +113,10 @@ __device__ __forceinline__ size_t out_offset(const PrefillParams& p, int t, int 
   return ((size_t)t * p.num_q_heads + h) * D;
 }
 
-template <int D, bool H, bool MODS, bool STRIDED>
+// PG: cache blocks of more than 16 slots (block_size = 16 << p.ppb_shift), so
+// a 16-key page sits at a slot offset inside its block; 16-slot blocks take the
+// plain path, in which a page is a whole block.
+template <int D, bool H, bool MODS, bool STRIDED, bool PG>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(PrefillParams p, const __grid_constant__ CUtensorMap q_map,
                    const __grid_constant__ CUtensorMap k_map,
@@ -236,19 +240,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                         q_hnd ? wk.head : wk.q_start + wk.row0 + x * BM);
         const int32_t* table = p.block_tables + (size_t)wk.seq * p.max_blocks_per_seq;
         for (int j = 0; j < wk.nmax && ok; ++j) {
+          // page pg (16 keys) of the tile: block blk, and with PG slots
+          // [slot, slot + 16) of it
           int blk[BN / kPageKeys];
+          [[maybe_unused]] int slot[BN / kPageKeys];
 #pragma unroll
           for (int pg = 0; pg < BN / kPageKeys; ++pg) {
             const int key0 = j * BN + pg * kPageKeys;
             int b = (int)p.num_blocks;  // out of range => zero fill
             if (key0 < wk.kv_len) {
-              const int t = table[key0 / kPageKeys];
+              const int t = PG ? table[key0 >> (p.ppb_shift + 4)] : table[key0 / kPageKeys];
               if (t >= 0 && t < p.num_blocks)
                 b = t;
               else
                 raise_error(err, PA_DEVERR_BLOCK);
             }
             blk[pg] = b;
+            if constexpr (PG) slot[pg] = key0 & (p.block_size - 1);
           }
 #pragma unroll
           for (int kv = 0; kv < 2; ++kv, ++ld) {  // K_j, then V_j
@@ -261,9 +269,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int pg = 0; pg < BN / kPageKeys; ++pg)
 #pragma unroll
-              for (int dh = 0; dh < D / 64; ++dh)
-                tma_load_4d(ring_s + st * SM::kKVBytes + dh * (BN * 128) + pg * (kPageKeys * 128),
-                            map, slot_full + st, dh * 64, kv_c1, kv_c2, blk[pg]);
+              for (int dh = 0; dh < D / 64; ++dh) {  // coordinates (d, head, slot) or (d, slot, head)
+                const uint32_t dst = ring_s + st * SM::kKVBytes + dh * (BN * 128) + pg * (kPageKeys * 128);
+                if constexpr (PG)
+                  tma_load_4d(dst, map, slot_full + st, dh * 64, kv_hnd ? slot[pg] : kvh,
+                              kv_hnd ? kvh : slot[pg], blk[pg]);
+                else
+                  tma_load_4d(dst, map, slot_full + st, dh * 64, kv_c1, kv_c2, blk[pg]);
+              }
           }
         }
         ++tcount;
@@ -628,17 +641,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool H, bool MODS, bool STRIDED>
-static cudaError_t launch_prefill_m(const PrefillParams& p, const CUtensorMap& q_map,
+template <int D, bool H, bool MODS, bool STRIDED, bool PG>
+static cudaError_t launch_prefill_b(const PrefillParams& p, const CUtensorMap& q_map,
                                     const CUtensorMap& k_map, const CUtensorMap& v_map, int grid,
                                     cudaStream_t stream) {
   using SM = PrefillSmem<D>;
-  auto kernel = prefill_kernel<D, H, MODS, STRIDED>;
+  auto kernel = prefill_kernel<D, H, MODS, STRIDED, PG>;
   cudaError_t e =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc);
   if (e != cudaSuccess) return e;
   kernel<<<grid, kThreads, SM::kAlloc, stream>>>(p, q_map, k_map, v_map);
   return cudaGetLastError();
+}
+
+template <int D, bool H, bool MODS, bool STRIDED>
+static cudaError_t launch_prefill_m(const PrefillParams& p, const CUtensorMap& q_map,
+                                    const CUtensorMap& k_map, const CUtensorMap& v_map, int grid,
+                                    cudaStream_t stream) {
+  return p.ppb_shift > 0
+             ? launch_prefill_b<D, H, MODS, STRIDED, true>(p, q_map, k_map, v_map, grid, stream)
+             : launch_prefill_b<D, H, MODS, STRIDED, false>(p, q_map, k_map, v_map, grid, stream);
 }
 
 template <int D, bool H>

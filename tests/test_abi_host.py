@@ -58,8 +58,10 @@ def _varlen(lib, **over):
     (dict(Hq=6, Hkv=4), 1),           # Hq % Hkv != 0
     (dict(Hkv=0), 1),
     (dict(D=96), 2),                  # unsupported head_dim
-    (dict(BS=32), 2),                 # unsupported block size
-    (dict(Hq=34, Hkv=2), 2),          # GQA group > 16
+    (dict(BS=24), 2),                 # block size not a multiple of 16
+    (dict(BS=8), 2),
+    (dict(BS=1024), 2),               # above the largest block size
+    (dict(Hq=258, Hkv=2), 2),         # GQA group > 128
     (dict(causal=2), 1),
     (dict(scale=float("nan")), 1),
     (dict(scale=-0.125), 1),          # negative scale
