@@ -43,6 +43,62 @@ int sm_count() {
   return g_sm_count[dev];
 }
 
+// Per-device resources for running a call's decode kernel beside its prefill
+// kernel: a side stream (non-blocking) and the two events that fork it from
+// and join it back to the caller's stream.  Created by the first call that
+// can use them outside a stream capture; the mutex keeps each call's
+// record / wait pairs together when several host threads share a device.
+// Inside a capture the fork and join are recorded as graph dependencies (the
+// side stream joins the capture), so a replay runs the two kernels side by
+// side as an eager call does, with the same results.
+struct SideStream {
+  std::mutex mu;
+  bool tried = false;
+  bool ok = false;
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+SideStream g_side[kMaxDevices];
+
+// The current device's side stream, or nullptr (the call then launches the
+// two kernels one after the other on the caller's stream): no device,
+// creation failed, the caller's stream is being captured before the side
+// stream exists (creating it inside a capture is avoided), or the side stream
+// is already part of a different, still open capture.
+SideStream* side_stream(cudaStream_t caller) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  unsigned long long cap_id = 0;
+  if (cudaStreamGetCaptureInfo(caller, &cap, &cap_id) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  SideStream* s = &g_side[dev];
+  std::lock_guard<std::mutex> lock(s->mu);
+  if (s->tried && s->ok) {
+    cudaStreamCaptureStatus side_cap = cudaStreamCaptureStatusNone;
+    unsigned long long side_id = 0;
+    if (cudaStreamGetCaptureInfo(s->stream, &side_cap, &side_id) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return nullptr;
+    }
+    if (side_cap != cudaStreamCaptureStatusNone &&
+        (cap != cudaStreamCaptureStatusActive || side_id != cap_id))
+      return nullptr;
+    return s;
+  }
+  if (cap != cudaStreamCaptureStatusNone) return nullptr;
+  if (!s->tried) {
+    s->tried = true;
+    s->ok = cudaStreamCreateWithFlags(&s->stream, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&s->fork, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&s->join, cudaEventDisableTiming) == cudaSuccess;
+    if (!s->ok) (void)cudaGetLastError();
+  }
+  return s->ok ? s : nullptr;
+}
+
 bool log_enabled() {
   static int v = -1;
   if (v < 0) {
@@ -384,14 +440,31 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
   const bool self_plan =
       num_seqs <= pa::kSelfPlanMaxSeqs &&
       pa::counter_slots_needed(num_seqs, num_q_heads, num_kv_heads) <= pa::kFixedCounterSlots;
+  // A call with multi-query sequences runs its decode kernel on a side stream
+  // beside the prefill kernel, each on the share of the SMs the plan kernel
+  // picks (the prefill is tensor-bound and the decode HBM-bound, so the two
+  // overlap); the side stream forks from the caller's stream after the plan
+  // and joins it again before the call returns.
+  SideStream* side = run_prefill ? side_stream(st) : nullptr;
+  std::unique_lock<std::mutex> side_lock;
+  if (side) side_lock = std::unique_lock<std::mutex>(side->mu);
+  pa::SplitShape split{};
+  if (side) split = pa::SplitShape{nsm, num_q_heads, num_kv_heads, head_dim};
   cudaError_t e = cudaSuccess;
   if (run_prefill || !self_plan) {
     pa::launch_plan(query_start_loc, seq_lens, num_seqs, num_q_tokens, max_blocks_per_seq,
                     block_size, max_query_len, max_seq_len, causal,
                     pa::counter_slots_needed(num_seqs, num_q_heads, num_kv_heads), span_offsets,
-                    spans, num_spans, ws, L, st);
+                    spans, num_spans, ws, L, split, st);
     e = cudaGetLastError();
     if (e != cudaSuccess) return PA_ERR_CUDA;
+  }
+  cudaStream_t dec_st = st;
+  if (side) {
+    if (cudaEventRecord(side->fork, st) != cudaSuccess ||
+        cudaStreamWaitEvent(side->stream, side->fork, 0) != cudaSuccess)
+      return PA_ERR_CUDA;
+    dec_st = side->stream;
   }
 
   if (run_prefill) {
@@ -420,8 +493,8 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
     pp.ws = ws;
     pp.L = L;
     pp.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+    pp.split = side ? 1 : 0;
     e = pa::launch_prefill(pp, q_map, k_map, v_map, head_dim, fp16, nsm, st);
-    if (e != cudaSuccess) return PA_ERR_CUDA;
   }
 
   pa::DecodeParams dp{};
@@ -438,6 +511,7 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
   dp.ppb_shift = pa::log2_pages_per_block(block_size);
   dp.max_seq_len = max_seq_len;
   dp.self_plan = self_plan ? 1 : 0;
+  dp.split_sms = side ? nsm : 0;
   dp.num_q_heads = num_q_heads;
   dp.num_kv_heads = num_kv_heads;
   dp.group = group;
@@ -456,7 +530,15 @@ pa_status attention_varlen_impl(const void* q, const void* k_cache, const void* 
   dp.out = static_cast<uint16_t*>(out);
   dp.ws = ws;
   dp.L = L;
-  e = pa::launch_decode(dp, head_dim, fp16, nsm, st);
+  const cudaError_t e_dec = e == cudaSuccess ? pa::launch_decode(dp, head_dim, fp16, nsm, dec_st) : e;
+  if (side) {
+    // join even after a failed launch, so the caller's stream never runs ahead
+    // of work queued on the side stream
+    const bool joined = cudaEventRecord(side->join, side->stream) == cudaSuccess &&
+                        cudaStreamWaitEvent(st, side->join, 0) == cudaSuccess;
+    if (!joined && e_dec == cudaSuccess) return PA_ERR_CUDA;
+  }
+  e = e_dec;
   if (log_enabled())
     fprintf(stderr, "[pa] varlen S=%d T=%lld Hq=%d Hkv=%d D=%d prefill=%d sms=%d\n", num_seqs,
             (long long)num_q_tokens, num_q_heads, num_kv_heads, head_dim, (int)run_prefill, nsm);

@@ -100,7 +100,14 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
   const int S = p.num_seqs;
   const int hg = blockIdx.x % groups;           // KV-head group of this CTA
   const long long c = blockIdx.x / groups;      // page range of this CTA
-  const long long G = gridDim.x / groups;       // page ranges per group
+  // page ranges per group: one per CTA of the grid, or, beside the prefill,
+  // the plan's share of the grid (the other CTAs leave at once)
+  long long G = gridDim.x / groups;
+  if (p.split_sms > 0) {
+    const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(p.ws + p.L.header);
+    G = max(1ll, G * min(hdr->decode_sms, p.split_sms) / p.split_sms);
+    if (c >= G) return;
+  }
   const int kvl = warp / SL;                    // this warp's KV head within the CTA
   const int slice = warp - kvl * SL;            // and its slice of the GQA group
   const int kvh = hg * hpc + kvl;               // this warp's KV head

@@ -36,11 +36,18 @@ cudaError_t launch_write_kv(const void* k, const void* v, const int64_t* slot_ma
                             int num_sms, cudaStream_t stream);
 
 // ---- plan ------------------------------------------------------------------
+// What the plan needs to split the machine between the prefill and the decode
+// kernel when they run side by side (sms = 0: they do not).
+struct SplitShape {
+  int sms;
+  int num_q_heads, num_kv_heads, head_dim;
+};
 void launch_plan(const int32_t* query_start_loc, const int32_t* seq_lens, int num_seqs,
                  long long num_q_tokens, int max_blocks_per_seq, int block_size,
                  int max_query_len, int max_seq_len, int causal, long long num_counters,
                  const int32_t* span_offsets, const int32_t* spans, int num_spans,
-                 unsigned char* ws, const WorkspaceLayout& L, cudaStream_t stream);
+                 unsigned char* ws, const WorkspaceLayout& L, const SplitShape& split,
+                 cudaStream_t stream);
 
 // ---- split-KV decode -------------------------------------------------------
 // Score modifiers of a varlen call (soft-cap, ALiBi, additive mask), as the
@@ -79,6 +86,7 @@ struct DecodeParams {
   ScoreMods mods;
   float scale_log2;  // scale * log2(e)
   int self_plan;     // 1: every CTA plans the decode work itself (num_seqs <= kSelfPlanMaxSeqs)
+  int split_sms;     // > 0: runs beside the prefill, on the plan's decode_sms of these SMs
   uint16_t* out;     // elements of the kernel's type (bf16 or fp16)
   unsigned char* ws;
   WorkspaceLayout L;
@@ -115,6 +123,7 @@ struct PrefillParams {
   unsigned char* ws;
   WorkspaceLayout L;
   unsigned long long wait_limit_ns;  // bound of every mbarrier wait; 0: the 1 s default
+  int split;  // 1: runs beside the decode kernel, on the plan's prefill_sms SMs
 };
 // Tensor maps are built by the host layer (they need the driver entry point).
 cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& q_map,

@@ -54,8 +54,24 @@ struct PlanHeader {
   int32_t num_prefill_tiles;   // entries in the prefill tile list
   int32_t total_decode_pages;  // 16-key pages over all single-query sequences
   int32_t prefill_next;        // prefill work items handed out after the first round
-  int32_t pad[61];
+  // When the prefill and decode kernels of a call run side by side, the SMs
+  // each may use (the plan's split of the machine; see plan.cu)
+  int32_t prefill_sms;
+  int32_t decode_sms;
+  int32_t pad[59];
 };
+
+// Cost model of the side-by-side split, measured on B200 at 1965 MHz:
+// a prefill work item's 128-row tile visiting one 128-key KV tile of one head
+// costs about kPrefillTileVisitUs SM-microseconds at head_dim 128 (prefill
+// time x SMs / tile visits on the varlen and mixed-step workloads: 1.14 and
+// 1.20); a decode CTA streams at most kDecodeSmBytesPerUs bytes per
+// microsecond (about 59 GB/s per SM, from runs on 24 to 96 SMs), and the
+// decode kernel as a whole at most kDecodeHbmBytesPerUs (7.2 TB/s, the
+// mixed step's 17 GB of decode reads on all SMs).
+constexpr double kPrefillTileVisitUs = 1.15;
+constexpr double kDecodeSmBytesPerUs = 59.0e3;
+constexpr double kDecodeHbmBytesPerUs = 7.2e6;
 
 struct WorkspaceLayout {
   size_t err;        // uint32 error word (PA_ERROR_WORD_BYTES reserved)

@@ -9,11 +9,15 @@
 //  - the exclusive prefix of 16-key pages over the single-query (decode)
 //    sequences, from which the decode CTAs cut their balanced page ranges
 //    when there are too many sequences for them to plan themselves;
-//  - zeroed split-KV arrival counters.
+//  - zeroed split-KV arrival counters;
+//  - when the call runs its prefill and decode kernels side by side, the
+//    share of the SMs each gets, from a cost model of the two kinds of work
+//    (prefill tile visits against decode bytes; see split_machine).
 // This plays the role of the device-side runtime length reduction of
 // ROCm/TransformerEngine PR #461 (description: the real maximum is found on
 // the device before routing), without any host synchronisation.
 #include "common.cuh"
+#include "kernels.h"
 #include "layout.h"
 #include "spans.cuh"
 
@@ -77,6 +81,42 @@ __device__ __forceinline__ int2 item_tiles(const SeqInfo& si, int row0, int caus
   return n;
 }
 
+// The SMs the prefill and the decode kernel each use when they run side by
+// side on split.sms SMs (both 0 when split.sms is 0: one after the other, each
+// on the whole machine).  With only one kind of work, each may take every SM.
+// Otherwise the prefill gets the P SMs that minimise the later finish time:
+// the prefill's work spread over P SMs, against the decode's bytes streamed by
+// the other SMs at no more than kDecodeSmBytesPerUs each and
+// kDecodeHbmBytesPerUs in all.  Called by one whole warp: each lane tries
+// every 32nd P, then the warp keeps the best (the smallest P on a tie).
+__device__ int2 split_machine(const SplitShape& split, float visits, float pages) {
+  if (split.sms <= 1) return make_int2(0, 0);
+  const float wp = visits * split.num_q_heads * (float)kPrefillTileVisitUs * split.head_dim / 128.f;
+  const float bytes = pages * kPageKeys * split.num_kv_heads * split.head_dim * 4.f;
+  if (!(wp > 0.f) || !(bytes > 0.f)) return make_int2(split.sms, split.sms);
+  const float t_hbm = bytes / (float)kDecodeHbmBytesPerUs;
+  float best_t = INFINITY;
+  int best_p = split.sms;
+  for (int p = 1 + (threadIdx.x & 31); p < split.sms; p += 32) {
+    const float t = fmaxf(wp / p, fmaxf(bytes / ((split.sms - p) * (float)kDecodeSmBytesPerUs), t_hbm));
+    if (t < best_t) {
+      best_t = t;
+      best_p = p;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ot = __shfl_xor_sync(0xffffffffu, best_t, o);
+    const int op = __shfl_xor_sync(0xffffffffu, best_p, o);
+    if (ot < best_t || (ot == best_t && op < best_p)) {
+      best_t = ot;
+      best_p = op;
+    }
+  }
+  if (best_p >= split.sms) best_p = split.sms / 2;
+  return make_int2(best_p, split.sms - best_p);
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kPlanThreads, 1)
@@ -84,7 +124,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
                 int num_seqs, long long num_q_tokens, int max_blocks_per_seq, int block_size,
                 int max_query_len, int max_seq_len, int causal, long long num_counters,
                 const int32_t* __restrict__ span_offsets, const int32_t* __restrict__ spans,
-                int num_spans, unsigned char* ws, WorkspaceLayout L) {
+                int num_spans, unsigned char* ws, WorkspaceLayout L, SplitShape split) {
   uint32_t* err = reinterpret_cast<uint32_t*>(ws + L.err);
   PlanHeader* hdr = reinterpret_cast<PlanHeader*>(ws + L.header);
   SeqInfo* info = reinterpret_cast<SeqInfo*>(ws + L.seq_info);
@@ -97,9 +137,13 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
   __shared__ int s_hist[kCostBuckets];
   __shared__ int s_carry;
   __shared__ uint32_t s_err;
+  __shared__ float s_visits;  // prefill tile visits (128-row tile x KV tile), summed per warp
 
   const int tid = threadIdx.x;
-  if (tid == 0) s_err = 0;
+  if (tid == 0) {
+    s_err = 0;
+    s_visits = 0.f;
+  }
   for (int i = tid; i < kCostBuckets; i += blockDim.x) s_hist[i] = 0;
   for (long long i = tid; i < num_counters; i += blockDim.x) counters[i] = 0;
   __syncthreads();
@@ -138,6 +182,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
   // ---- pass 2: decode page prefix, tile histogram --------------------------
   if (tid == 0) s_carry = 0;
   __syncthreads();
+  int my_visits = 0;  // this thread's prefill tile visits
   for (int base = 0; base < num_seqs; base += blockDim.x) {
     const int s = base + tid;
     int pages = 0;
@@ -153,6 +198,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
           bad |= bad_r;
           const int c = n.x + n.y;
           atomicAdd(&s_hist[kCostBuckets - 1 - min(c, kCostBuckets - 1)], 1);
+          my_visits += c;
         }
         if (bad) atomicOr(&s_err, PA_DEVERR_SPANS);
       }
@@ -166,6 +212,12 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
   }
   if (tid == 0) page_pfx[num_seqs] = s_carry;
   const int total_pages = s_carry;
+  {
+    float v = (float)my_visits;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((tid & 31) == 0 && v > 0.f) atomicAdd(&s_visits, v);
+  }
 
   // ---- pass 3: counting sort of prefill tiles by descending cost -----------
   // exclusive scan of the histogram (bucket 0 = most expensive)
@@ -206,6 +258,13 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
     }
   }
   __syncthreads();
+  if (tid < 32) {
+    const int2 sms = split_machine(split, s_visits, (float)total_pages);
+    if (tid == 0) {
+      hdr->prefill_sms = sms.x;
+      hdr->decode_sms = sms.y;
+    }
+  }
   if (tid == 0) {
     // the last bucket's running cursor ends at the number of tiles
     num_tiles = (int)min((long long)s_hist[kCostBuckets - 1], (long long)L.max_tiles);
@@ -220,11 +279,12 @@ void launch_plan(const int32_t* query_start_loc, const int32_t* seq_lens, int nu
                  long long num_q_tokens, int max_blocks_per_seq, int block_size,
                  int max_query_len, int max_seq_len, int causal, long long num_counters,
                  const int32_t* span_offsets, const int32_t* spans, int num_spans,
-                 unsigned char* ws, const WorkspaceLayout& L, cudaStream_t stream) {
+                 unsigned char* ws, const WorkspaceLayout& L, const SplitShape& split,
+                 cudaStream_t stream) {
   plan_kernel<<<1, kPlanThreads, 0, stream>>>(query_start_loc, seq_lens, num_seqs, num_q_tokens,
                                               max_blocks_per_seq, block_size, max_query_len,
                                               max_seq_len, causal, num_counters, span_offsets,
-                                              spans, num_spans, ws, L);
+                                              spans, num_spans, ws, L, split);
 }
 
 }  // namespace pa

@@ -155,6 +155,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int2* tile_n = reinterpret_cast<const int2*>(ws + p.L.tile_n);
   const int num_work = hdr->num_prefill_tiles * p.num_q_heads;
   const uint64_t wlim = p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs;
+  // Beside the decode kernel only the plan's share of the CTAs (one per SM)
+  // takes work: the others are handed no item and leave, freeing their SMs.
+  const int ctas = p.split ? min((int)gridDim.x, max(1, hdr->prefill_sms)) : (int)gridDim.x;
   // Work distribution: the first item of a CTA is blockIdx.x; later ones are
   // taken from a counter (sorted by descending cost, so the longest go first),
   // so SMs that run faster take more items.  The producer publishes each item
@@ -214,7 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // instantiation only; the dense one keeps token-major order)
       const bool q_hnd = STRIDED && p.q_hnd != 0, kv_hnd = STRIDED && p.kv_hnd != 0;
       for (int k = 0; ok; ++k) {
-        int w = k == 0 ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(next_item, 1);
+        int w = k == 0 ? ((int)blockIdx.x < ctas ? (int)blockIdx.x : num_work)
+                       : ctas + atomicAdd(next_item, 1);
         if (w >= num_work) w = -1;
         const int slot = k % SM::kItemRing;
         if (k >= SM::kItemRing)
