@@ -156,6 +156,21 @@ __device__ __forceinline__ void cp_async_16n(uint32_t dst, const void* src, int 
                "r"(src_bytes)
                : "memory");
 }
+// cp.async of 16 bytes (zero-filled when !valid) under an L2 eviction policy
+// made by createpolicy, e.g. evict-first for data read once.
+__device__ __forceinline__ void cp_async_16_hint(uint32_t dst, const void* src, bool valid,
+                                                 uint64_t policy) {
+  int src_bytes = valid ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;\n" ::"r"(dst),
+               "l"(src), "r"(src_bytes), "l"(policy)
+               : "memory");
+}
+// L2 policy: lines this thread reads under it are the first to be evicted.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;\n" ::: "memory");
 }

@@ -234,6 +234,10 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
   int p_kv = seq_kv(seq_p);
   [[maybe_unused]] int p_tok = MODS ? seq_q(seq_p) : 0;  // the sequence's query token
   long long x = b0;  // consumer position
+  // Each K/V page is read once per call: streaming it evict-first keeps the
+  // lines that are read again (the partials a split-KV merge reads back, q,
+  // the tables) in L2 while the stream passes through.
+  const uint64_t kv_policy = policy_evict_first();
   auto issue_page = [&]() {
     const int stage = (int)((x_p - b0) % NSTAGE);
     const int page = (int)(x_p - p_first);  // 16-key page of the sequence
@@ -282,8 +286,8 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
       const bool ok = block_ok && (key0 + r < p_kv);
       const size_t src = base + (size_t)r * p.c_slot + (size_t)h * p.c_head + cc * 8;
       const int dst = (h * kPageKeys + r) * D + ((cc ^ (r & 7)) * 8);
-      cp_async_16(smem_u32(kdst + dst), p.k_cache + (ok ? src : 0), ok);
-      cp_async_16(smem_u32(vdst + dst), p.v_cache + (ok ? src : 0), ok);
+      cp_async_16_hint(smem_u32(kdst + dst), p.k_cache + (ok ? src : 0), ok, kv_policy);
+      cp_async_16_hint(smem_u32(vdst + dst), p.v_cache + (ok ? src : 0), ok, kv_policy);
     }
     cp_async_commit();
     ++x_p;
