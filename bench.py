@@ -650,9 +650,29 @@ def run_single_workload(args):
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / args.steps
     v = work / (ms * 1e-3) / scale_div
-    return {"workload": name, "value": round(v, 2), "unit": unit, "ms_per_step": round(ms, 5),
-            "steps": args.steps, "warmup": args.warmup, "frac": round(v / peak, 4),
-            "peak": peak, "peak_kind": peak_kind}
+    res = {"workload": name, "value": round(v, 2), "unit": unit, "ms_per_step": round(ms, 5),
+           "steps": args.steps, "warmup": args.warmup, "frac": round(v / peak, 4),
+           "peak": peak, "peak_kind": peak_kind}
+    if args.timeline:
+        res["timeline"] = kernel_timeline(step)
+    return res
+
+
+def kernel_timeline(step):
+    """Start and end (µs, from the first kernel's start) of every kernel one
+    call of `step` launches, from the CUDA activity records of torch.profiler:
+    shows which kernels of a call ran side by side."""
+    torch.cuda.synchronize()
+    with torch.profiler.profile(activities=[torch.profiler.ProfilerActivity.CUDA]) as prof:
+        step()
+        torch.cuda.synchronize()
+    ev = [e for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
+    if not ev:
+        return []
+    t0 = min(e.time_range.start for e in ev)
+    return [{"kernel": e.name.split("(")[0][:80], "start_us": round(e.time_range.start - t0, 1),
+             "end_us": round(e.time_range.end - t0, 1)}
+            for e in sorted(ev, key=lambda e: e.time_range.start)]
 
 
 def run_e2e(pa, case, args, dev, ws):
@@ -853,6 +873,8 @@ def main():
                     choices=sorted(list(workloads.NAMED) + ["spans_prefill", "smallseq_bwd",
                                                            "scatter_varlen"]),
                     help="decode_batch is the headline; the others time one workload alone")
+    ap.add_argument("--timeline", action="store_true",
+                    help="with --workload: also list one step's kernels with start / end times")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per dominant-kernel launch from an ncu capture, if current")
     args = ap.parse_args()

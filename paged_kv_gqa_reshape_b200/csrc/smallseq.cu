@@ -194,8 +194,9 @@ __global__ void __launch_bounds__(256, 3) smallseq_kernel(SmallSeqParams p) {
       for (int pp = 0; pp < PASSES; ++pp)
         if (l == pp) mine = pwv[pp];
       const float wt = __shfl_sync(0xffffffffu, mine, (lane % KPP) * LPK + lane / KPP);
-      for (int t = lane; t < p.weights_len; t += 32)
-        wrow[t] = (t < cur.n && t == lane) ? ebits<H>(wt * winv) : (uint16_t)0;
+      for (int t = lane; t < p.weights_len; t += 32)  // written once, not read back here
+        __stcs(reinterpret_cast<unsigned short*>(wrow + t),
+               (t < cur.n && t == lane) ? ebits<H>(wt * winv) : (unsigned short)0);
     }
     if (sub == 0) {
       const float inv = sum > 0.f ? 1.f / sum : 0.f;  // an empty entry writes zeros
