@@ -86,6 +86,10 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
   // resident before it ends and wait here, before reading any input, until
   // it has completed and its writes are visible.
   griddep_wait();
+  // The next kernel on the stream, if launched the same way (the next step's
+  // cache scatter is), may become resident now; it waits for this grid to
+  // complete before it touches anything.
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int tid = threadIdx.x;

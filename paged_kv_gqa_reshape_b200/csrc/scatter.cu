@@ -29,6 +29,12 @@ __global__ void __launch_bounds__(256) write_kv_kernel(const uint4* __restrict__
   // the attention call that follows reads the caches only after this grid has
   // completed (griddep_wait); its planning may overlap this scatter
   griddep_launch_dependents();
+  // Launched with programmatic stream serialisation: when the previous kernel
+  // lets this one start early (the decode kernel does, so that the next
+  // step's scatter is resident before it ends), wait here, before touching
+  // any input or the caches, until it has completed and its writes are
+  // visible (it may still be reading the cache rows this grid overwrites).
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
   for (long long t = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -87,11 +93,21 @@ cudaError_t launch_write_kv(const void* k, const void* v, const int64_t* slot_ma
   long long blocks = (warps_needed + (threads / 32) - 1) / (threads / 32);
   const long long cap = (long long)num_sms * 8;  // 8 resident 256-thread CTAs per SM
   if (blocks > cap) blocks = cap;
-  write_kv_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
-      static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping, num_tokens,
-      row_vecs, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), num_slots, block_size,
-      block_vecs, slot_vecs, head_vecs, dshift, err);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, write_kv_kernel, static_cast<const uint4*>(k),
+                            static_cast<const uint4*>(v), slot_mapping, (long long)num_tokens,
+                            row_vecs, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+                            (long long)num_slots, block_size, (long long)block_vecs,
+                            (long long)slot_vecs, (long long)head_vecs, dshift, err);
 }
 
 }  // namespace pa
