@@ -42,8 +42,8 @@ WORKLOAD = ("decode_batch: 64 seqs x 1 query token, context U[256,4096], Hq 32 /
 # DRAM bytes (read + write) of one decode-kernel launch on the decode batch, from
 # one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), valid only
 # while the decode kernel's sources hash to the recorded value.
-DECODE_TRAFFIC = {"sources_sha256": "77d78743a5dafd09846b6cb1e4435b4edefd45fd75e0872bd1774db12ea59cf9",
-                  "bytes_per_launch": 597421312}
+DECODE_TRAFFIC = {"sources_sha256": "28c9cd251130f5f91c40fef6d44655321d2e76565e75b424a5e1b6f6a8cdbf2e",
+                  "bytes_per_launch": 597274965}
 DECODE_SOURCES = ("decode.cu", "decode.cuh", "common.cuh", "layout.h")
 
 

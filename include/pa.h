@@ -31,9 +31,14 @@
  *    entry points, with one exception: the PA_STATIC_SCRATCH_BYTES device
  *    array behind pa_attention_varlen_static, which every GPU that loads the
  *    library holds, and which carries that entry point's scratch (its
- *    split-KV arrival counters among it) from one call to the next.
+ *    split-KV arrival counters among it) from one call to the next.  Besides
+ *    memory, each device gets one library-owned side stream and two events
+ *    (created on the first varlen call with multi-query sequences made
+ *    outside a stream capture; see pa_attention_varlen).
  *  - `stream` is a cudaStream_t passed as void*; NULL means the legacy default
- *    stream.  No call synchronises except pa_get_error.
+ *    stream.  No call synchronises except pa_get_error.  Every call is
+ *    ordered on `stream` as one unit: work a call runs on the side stream is
+ *    forked from `stream` and joined back to it before the call returns.
  *  - `out` must not alias any input.
  *
  * Errors
@@ -145,7 +150,16 @@ size_t pa_attention_varlen_workspace_size(int32_t num_seqs, int64_t num_q_tokens
  * sparse attention", description: an empty selection gives zeros).
  * seq_lens counts every key of the sequence, this step's tokens included.
  * Sequences with Lq == 1 take the split-KV decode kernel; all others the
- * tensor-core prefill kernel; both may appear in one call.
+ * tensor-core prefill kernel; both may appear in one call.  When the prefill
+ * kernel runs, the decode kernel runs beside it on the device's side stream
+ * (forked from `stream` after the planning kernel, joined back before the
+ * call returns), each on the share of the SMs the planning kernel picks for
+ * this batch.  Inside a stream capture the fork and join are captured too,
+ * once the side stream exists (the first such call outside a capture makes
+ * it); until then, or while the side stream belongs to another open capture,
+ * the two kernels run one after the other on `stream`.  Results are the same
+ * either way up to rounding (the decode's split-KV partition follows the
+ * share of SMs it gets).
  *
  *  q                [num_q_tokens, num_q_heads, head_dim] bf16
  *  k_cache, v_cache [num_blocks, block_size, num_kv_heads, head_dim] bf16
