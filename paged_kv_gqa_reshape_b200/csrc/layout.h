@@ -66,11 +66,12 @@ struct PlanHeader {
 // costs about kPrefillTileVisitUs SM-microseconds at head_dim 128 (prefill
 // time x SMs / tile visits on the varlen and mixed-step workloads: 1.14 and
 // 1.20); a decode CTA streams at most kDecodeSmBytesPerUs bytes per
-// microsecond (about 59 GB/s per SM, from runs on 24 to 96 SMs), and the
-// decode kernel as a whole at most kDecodeHbmBytesPerUs (7.2 TB/s, the
+// microsecond (about 59 GB/s per SM alone, from runs on 24 to 96 SMs; 56 GB/s
+// beside the prefill, from the mixed step's 17 GB on 105 SMs in 2.90 ms), and
+// the decode kernel as a whole at most kDecodeHbmBytesPerUs (7.2 TB/s, the
 // mixed step's 17 GB of decode reads on all SMs).
 constexpr double kPrefillTileVisitUs = 1.15;
-constexpr double kDecodeSmBytesPerUs = 59.0e3;
+constexpr double kDecodeSmBytesPerUs = 56.0e3;
 constexpr double kDecodeHbmBytesPerUs = 7.2e6;
 
 struct WorkspaceLayout {
