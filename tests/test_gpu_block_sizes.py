@@ -195,3 +195,50 @@ def test_large_group_with_modifiers():
         mask_head_stride=t * ld, mask_token_stride=ld)
     assert_attention_close(out, ref, what="g=32 with modifiers")
     assert pa.get_error(ws) == (0, 0)
+
+
+# ---------------------------------------------------------------------------
+# large blocks with the other features: full-attention spans and an additive
+# mask (prefill, chunked prefill and decode rows in one batch)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bs", [32, 128])
+def test_spans_with_large_blocks(bs):
+    from tests.test_gpu_spans import oracle_spans, run_spans
+    lens = [700, 300, 129, 1000, 40]
+    qlens = [700, 300, 129, 400, 1]
+    spans_per_seq = [[(0, 100), (100, 300), (517, 700)], [(128, 256)], [],
+                     [(610, 900), (900, 901), (950, 1000)], [(0, 40)]]
+    cpu = build(lens, qlens, 8, 2, 128, bs, seed=60 + bs)
+    offs = np.cumsum([0] + [len(x) for x in spans_per_seq])
+    flat = [p for x in spans_per_seq for p in x]
+    out, ws = run_spans(case_to(cpu, "cuda"), offs, flat)
+    assert_attention_close(out, oracle_spans(cpu, offs, flat), what=f"spans bs={bs}")
+    assert pa.get_error(ws) == (0, 0)
+
+
+@pytest.mark.parametrize("bs", [32, 64])
+def test_additive_mask_with_large_blocks(bs):
+    lens, qlens = [400, 33, 129, 1000], [400, 1, 64, 1]
+    cpu = build(lens, qlens, 8, 2, 64, bs, seed=70 + bs)
+    dev = case_to(cpu, "cuda")
+    t, ld = cpu.num_q_tokens, 1024
+    g = torch.Generator().manual_seed(71)
+    mask = torch.randn((8, t, ld), generator=g) * 2
+    mask[torch.rand((8, t, ld), generator=g) < 0.05] = float("-inf")
+    kc, vc = dev.k_cache.clone(), dev.v_cache.clone()
+    ws = pa.varlen_workspace(dev.num_seqs, t, 8, 2, 64)
+    pa.write_kv(dev.k_new, dev.v_new, dev.slot_mapping, kc, vc, workspace=ws)
+    out = torch.full_like(dev.q, float("nan"))
+    pa.attention_varlen(dev.q, kc, vc, dev.block_tables, dev.seq_lens, dev.query_start_loc, 2,
+                        dev.scale, True, out, max_query_len=dev.max_query_len,
+                        max_seq_len=dev.max_seq_len, workspace=ws, mask=mask.cuda())
+    torch.cuda.synchronize()
+    ref = oracle.attention_varlen_mods(
+        workloads.bf16_bits(cpu.q), workloads.bf16_bits(cpu.k_logical),
+        workloads.bf16_bits(cpu.v_logical), cpu.kv_offsets.numpy(), cpu.seq_lens.numpy(),
+        cpu.query_start_loc.numpy(), 2, cpu.scale, True, 0,
+        mask=mask.contiguous().numpy().reshape(-1), mask_head_stride=t * ld,
+        mask_token_stride=ld)
+    assert_attention_close(out, ref, what=f"mask bs={bs}")
+    assert pa.get_error(ws) == (0, 0)
