@@ -132,6 +132,7 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
   constexpr int kMaskHeads = HPC * NGT * 8;
   constexpr int kMaskStage = MODS ? kMaskHeads * kPageKeys : 0;  // floats per stage
   float* mring = reinterpret_cast<float*>(smem + Shape::kRingBytes);
+  [[maybe_unused]] const bool mask_shared = MODS && p.mods.mask_head == 0;
   int* s_pg = reinterpret_cast<int*>(smem + Shape::kRingBytes + NSTAGE * kMaskStage * 4);  // [S + 1] page prefix
   int* s_kv = s_pg + kSelfPlanMaxSeqs + 1;                       // [S] decode kv_len or -1
   __shared__ uint32_t s_err;
@@ -257,11 +258,14 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
     if constexpr (MODS) {
       if (p.mods.mask) {
         // the page's mask values: 16 keys (4 chunks of 4) for each query-head
-        // slot (warp w's local head hl) of the CTA; keys past the sequence
+        // slot (warp w's local head hl) of the CTA, or once when every head
+        // shares the mask (head stride 0: one copy, not one identical
+        // request per head to the same L2 line); keys past the sequence
         // end or the mask row read nothing and are zero-filled
         float* mdst = mring + (size_t)stage * kMaskStage;
         const long long lim = min((long long)p_kv, p.mods.mask_len);
-        for (int ci = tid; ci < kMaskHeads * 4; ci += NT) {
+        const int mask_slots = mask_shared ? 1 : kMaskHeads;
+        for (int ci = tid; ci < mask_slots * 4; ci += NT) {
           const int hs = ci >> 2, q4 = ci & 3;
           const int w = hs / (NGT * 8), hl = hs - w * (NGT * 8);  // warp w's local head hl
           const int wsl = w % SL, wh0 = (hg * hpc + w / SL) * g + wsl * 16;
@@ -404,12 +408,13 @@ __global__ void __launch_bounds__(HPC * 32, 8 / HPC) decode_kernel(DecodeParams 
           // this page's mask values (log2 units) from the ring stage
           float mv[4] = {0.f, 0.f, 0.f, 0.f};
           if (p.mods.mask) {
+            const int hstride = mask_shared ? 0 : kPageKeys;  // floats between head slots
             const float* mst = mring + (size_t)((x - b0) % NSTAGE) * kMaskStage +
-                               (size_t)(warp * NGT * 8 + nt * 8 + 2 * tq) * kPageKeys + gq;
+                               (size_t)(warp * NGT * 8 + nt * 8 + 2 * tq) * hstride + gq;
             mv[0] = mst[0] * kLog2e;
-            mv[1] = mst[kPageKeys] * kLog2e;
+            mv[1] = mst[hstride] * kLog2e;
             mv[2] = mst[8] * kLog2e;
-            mv[3] = mst[kPageKeys + 8] * kLog2e;
+            mv[3] = mst[hstride + 8] * kLog2e;
           }
           s0 = ok0 ? mod(sc[nt][0], msl[nt][0], mv[0], key0 + gq) : -INFINITY;
           s1 = ok0 ? mod(sc[nt][1], msl[nt][1], mv[1], key0 + gq) : -INFINITY;

@@ -167,17 +167,20 @@ def test_large_group_equals_repeat_interleaved_heads():
     assert (out_g.float() - out_m.float()).abs().max().item() <= 2e-2
 
 
-def test_large_group_with_modifiers():
+@pytest.mark.parametrize("per_head", [True, False])
+def test_large_group_with_modifiers(per_head):
+    # per_head False: one mask row per token shared by every head (head stride 0)
     lens = [300, 1, 2000, 129]
     qlens = [300, 1, 1, 64]
     hq, hkv = 64, 2
     cpu = build(lens, qlens, hq, hkv, 128, 32, seed=77)
     dev = case_to(cpu, "cuda")
     slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / hq) for h in range(hq)], dtype=torch.float32)
-    t, ld = cpu.num_q_tokens, 2048  # per-head mask rows longer than every sequence
+    t, ld = cpu.num_q_tokens, 2048  # mask rows longer than every sequence
     g = torch.Generator().manual_seed(8)
-    mask = torch.randn((hq, t, ld), generator=g)
-    mask[torch.rand((hq, t, ld), generator=g) < 0.05] = float("-inf")
+    shape = (hq, t, ld) if per_head else (t, ld)
+    mask = torch.randn(shape, generator=g)
+    mask[torch.rand(shape, generator=g) < 0.05] = float("-inf")
     kc, vc = dev.k_cache.clone(), dev.v_cache.clone()
     ws = pa.varlen_workspace(dev.num_seqs, t, hq, hkv, 128)
     pa.write_kv(dev.k_new, dev.v_new, dev.slot_mapping, kc, vc, workspace=ws)
@@ -192,8 +195,8 @@ def test_large_group_with_modifiers():
         workloads.bf16_bits(cpu.v_logical), cpu.kv_offsets.numpy(), cpu.seq_lens.numpy(),
         cpu.query_start_loc.numpy(), hkv, cpu.scale, True, 0, softcap=30.0,
         alibi_slopes=slopes.numpy(), mask=mask.contiguous().numpy().reshape(-1),
-        mask_head_stride=t * ld, mask_token_stride=ld)
-    assert_attention_close(out, ref, what="g=32 with modifiers")
+        mask_head_stride=t * ld if per_head else 0, mask_token_stride=ld)
+    assert_attention_close(out, ref, what=f"g=32 with modifiers, per-head mask {per_head}")
     assert pa.get_error(ws) == (0, 0)
 
 
