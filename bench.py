@@ -542,7 +542,7 @@ def run_ours(args, rank, world, local_rank):
     value = whole_job_gbs(bytes_step, args.steps, world, max_ms)
 
     # end to end through the public API: pinned host inputs in, output back, every step
-    e2e = run_e2e(pa, case, args, dev, ws)
+    e2e = run_e2e(pa, case, args, dev, ws, expected=out)
     e2e["ms"] = max_over_ranks(e2e["ms"], world, dev)
     e2e_value = whole_job_gbs(bytes_step, args.steps, world, e2e["ms"])
 
@@ -555,7 +555,8 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic (seeded N(0,1) bf16; per-rank seed 1002+rank)",
         "config": headline_config(world, args.graph),
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
-                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                "mode": e2e["mode"]},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                      "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                      "traffic": args.traffic if args.traffic is not None else recorded_traffic(),
@@ -675,8 +676,17 @@ def kernel_timeline(step):
             for e in sorted(ev, key=lambda e: e.time_range.start)]
 
 
-def run_e2e(pa, case, args, dev, ws):
-    """The same step through the public API with host-resident inputs/outputs."""
+def run_e2e(pa, case, args, dev, ws, expected=None):
+    """The same step through the public API with host-resident inputs/outputs.
+
+    Default (pipelined, as a serving loop runs it): each step's inputs are
+    copied in on a host-to-device stream one step ahead, into one of two
+    device buffers, and its output goes back on a device-to-host stream from
+    one of two output buffers, so both transfers overlap the neighbouring
+    steps' kernels; events order every buffer's reuse.  `--e2e-serial` runs
+    copy in, kernels, copy out one after another on one stream instead (the
+    only form `--graph` captures).  Either way every step copies all of its
+    inputs in and its output back inside the timed region."""
     names = ["q", "k_new", "v_new", "slot_mapping", "block_tables", "seq_lens", "query_start_loc"]
     # the step's inputs packed in one pinned host buffer (each at a 256-byte
     # offset) and copied with one transfer into one device buffer, whose
@@ -687,52 +697,112 @@ def run_e2e(pa, case, args, dev, ws):
         offs[n] = off
         off += (t.numel() * t.element_size() + 255) // 256 * 256
     host_buf = torch.empty(off, dtype=torch.uint8).pin_memory()
-    dev_buf = torch.empty(off, dtype=torch.uint8, device=dev)
-    devt = {}
     for n in names:
         t = getattr(case, n)
         nbytes = t.numel() * t.element_size()
         host_buf[offs[n]:offs[n] + nbytes].copy_(t.contiguous().view(torch.uint8).view(-1).cpu())
-        devt[n] = dev_buf[offs[n]:offs[n] + nbytes].view(t.dtype).view(t.shape)
+    serial = args.e2e_serial or args.graph
+    nbuf = 1 if serial else 2
+    dev_bufs, devts, outs_d = [], [], []
+    for _ in range(nbuf):
+        buf = torch.empty(off, dtype=torch.uint8, device=dev)
+        devt = {}
+        for n in names:
+            t = getattr(case, n)
+            nbytes = t.numel() * t.element_size()
+            devt[n] = buf[offs[n]:offs[n] + nbytes].view(t.dtype).view(t.shape)
+        dev_bufs.append(buf)
+        devts.append(devt)
+        outs_d.append(torch.empty_like(case.q))
     out_h = torch.empty(case.q.shape, dtype=case.q.dtype).pin_memory()
-    out_d = torch.empty_like(case.q)
     h2d = sum(getattr(case, n).numel() * getattr(case, n).element_size() for n in names)
     d2h = out_h.numel() * out_h.element_size()
     steps = max(1, min(args.steps, 500))
     mql, msl = case.max_query_len, case.max_seq_len  # host-side metadata, known before the step
 
-    def step():
-        dev_buf.copy_(host_buf, non_blocking=True)
+    def kernels(b):
+        devt = devts[b]
         pa.write_kv(devt["k_new"], devt["v_new"], devt["slot_mapping"], case.k_cache,
                     case.v_cache, workspace=ws)
         pa.attention_varlen(devt["q"], case.k_cache, case.v_cache, devt["block_tables"],
                             devt["seq_lens"], devt["query_start_loc"], case.num_kv_heads,
-                            case.scale, case.causal, out_d, max_query_len=mql,
+                            case.scale, case.causal, outs_d[b], max_query_len=mql,
                             max_seq_len=msl, workspace=ws)
-        out_h.copy_(out_d, non_blocking=True)
 
-    for _ in range(3):
-        step()
+    comp = torch.cuda.current_stream(dev)
+    if serial:
+        def step(i):
+            dev_bufs[0].copy_(host_buf, non_blocking=True)
+            kernels(0)
+            out_h.copy_(outs_d[0], non_blocking=True)
+    else:
+        h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev = lambda: [torch.cuda.Event() for _ in range(nbuf)]
+        staged, computed, returned = ev(), ev(), ev()
+        used = [False] * nbuf
+
+        def step(i):
+            b = i % nbuf
+            with torch.cuda.stream(h2d_s):
+                if used[b]:
+                    h2d_s.wait_event(computed[b])  # step i-2's kernels have read buffer b
+                dev_bufs[b].copy_(host_buf, non_blocking=True)
+                staged[b].record(h2d_s)
+            comp.wait_event(staged[b])
+            if used[b]:
+                comp.wait_event(returned[b])  # step i-2's output has left buffer b
+            kernels(b)
+            computed[b].record(comp)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(computed[b])
+                out_h.copy_(outs_d[b], non_blocking=True)
+                returned[b].record(d2h_s)
+            used[b] = True
+
+        def drain():
+            for b in range(nbuf):
+                if used[b]:
+                    comp.wait_event(returned[b])
+
+    for i in range(3):
+        step(i)
+    if not serial:
+        drain()
     torch.cuda.synchronize()
-    # with --graph: one CUDA graph of the whole step (the host-to-device copies
-    # of its inputs, the two library calls, the copy of the output back)
-    g = capture_graph(step, 1) if args.graph else None
+    # with --graph: one CUDA graph of the whole serial step (the host-to-device
+    # copy of its inputs, the two library calls, the copy of the output back)
+    g = capture_graph(lambda: step(0), 1) if args.graph else None
     if g is not None:
         for _ in range(3):
             g.replay()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(steps):
+    a.record(comp)
+    if not serial:
+        h2d_s.wait_event(a)  # no copy of the timed steps starts before the first event
+        d2h_s.wait_event(a)
+        used = [False] * nbuf
+    for i in range(steps):
         if g is not None:
             g.replay()
         else:
-            step()
-    b.record()
+            step(i)
+    if not serial:
+        drain()  # the last outputs are back on the host before the end event
+    b.record(comp)
     torch.cuda.synchronize()
     del g
     ms = a.elapsed_time(b) * args.steps / steps
-    return {"ms": ms, "h2d": h2d, "d2h": d2h}
+    st, bits = pa.get_error(ws)
+    if st != 0:
+        raise RuntimeError(f"device error word {bits:#x} in the end-to-end leg")
+    # the output that came back is the device-resident path's, bit for bit
+    if expected is not None and not torch.equal(out_h, expected.cpu()):
+        raise RuntimeError("end-to-end output differs from the device-resident step's")
+    mode = ("serial: copy in, kernels, copy out on one stream" if serial else
+            "pipelined: inputs copied in one step ahead on a copy stream, outputs copied "
+            "back on another, two device buffers each")
+    return {"ms": ms, "h2d": h2d, "d2h": d2h, "mode": mode}
 
 
 # ---------------------------------------------------------------------------
@@ -867,6 +937,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-components", action="store_true")
+    ap.add_argument("--e2e-serial", action="store_true",
+                    help="end-to-end leg: copy in, kernels, copy out serially on one stream")
     ap.add_argument("--graph", action="store_true",
                     help="time the step (and the end-to-end leg) as replays of a CUDA graph")
     ap.add_argument("--workload", default="decode_batch",
