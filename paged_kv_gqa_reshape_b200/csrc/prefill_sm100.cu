@@ -335,8 +335,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = wait_tile(base);
         if (!ok) break;
         tc_fence_after();
-        if (wk.n[0] > 0) issue_s(0, base);
-        if (wk.n[1] > 0) issue_s(1, base);
+        // S_x(0) overwrites the columns the previous item's last P_x occupied:
+        // let that P_x.V finish first (MMAs on different accumulators are
+        // not ordered by their issue)
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if (wk.n[x] == 0) continue;
+          if (pv_it[x] > 0) {
+            ok = mbar_wait_bounded(o_done + x, (pv_it[x] - 1) & 1, abort_flag, err, wlim);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          issue_s(x, base);
+        }
+        if (!ok) break;
         tc_commit(slot_empty + (int)(base % kRing));  // K_0 read by both S MMAs
         if (wk.nmax == 1) tc_commit(q_empty);
         for (int j = 0; j < wk.nmax && ok; ++j) {
