@@ -353,18 +353,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (wk.nmax == 1) tc_commit(q_empty);
         for (int j = 0; j < wk.nmax && ok; ++j) {
           const long long kn = base + 2 * (j + 1), vj = base + 2 * j + 1;
+          if constexpr (MODS) {
+            // the modifiers' longer softmax leaves V_j and K_{j+1} landed long
+            // before P_x(j) is ready: check both first, off the P -> P.V -> S
+            // chain (in the plain kernel this order measured slower)
+            ok = wait_tile(vj);
+            if (ok && j + 1 < wk.nmax) ok = wait_tile(kn);
+            if (!ok) break;
+          }
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
             if (j >= wk.n[x]) continue;
             ok = mbar_wait_bounded(p_full + x, pv_it[x] & 1, abort_flag, err, wlim);
-            if (ok) ok = wait_tile(vj);
+            if (!MODS && ok) ok = wait_tile(vj);
             if (!ok) break;
             tc_fence_after();
             issue_pv(x, vj, j > 0);
             if (j + 1 < wk.n[x]) {
               // S_x(j+1) overwrites the columns P_x(j) occupies: let P_x(j).V finish
               ok = mbar_wait_bounded(o_done + x, (pv_it[x] - 1) & 1, abort_flag, err, wlim);
-              if (ok) ok = wait_tile(kn);
+              if (!MODS && ok) ok = wait_tile(kn);
               if (!ok) break;
               tc_fence_after();
               issue_s(x, kn);
